@@ -1,0 +1,101 @@
+/*
+ * bi.h -- C ABI of libbi.so: batch-invariant forward kernels for NVIDIA B200 (sm_100a).
+ *
+ * Batch invariance: for fixed weights and fixed shape parameters (H, N, K, r, D,
+ * chunk, eps, scale), the bits of output row m depend only on input row m.  They
+ * do not depend on the batch size M, on the row's position in the batch, or on
+ * the other rows.  Every kernel gets this by construction.  Its launch plan,
+ * reduction tree, tile shape and split counts are functions of the shape
+ * parameters alone, never of M.  No kernel uses floating-point atomics.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" must point to device memory (or memory the device
+ *     can address) on the current CUDA device.  Pointers marked "host" are read
+ *     by the CPU before the call returns.
+ *   - The caller allocates and owns every buffer, workspaces included.  The
+ *     library never allocates, frees or synchronises, except where an entry point
+ *     says otherwise.
+ *   - `stream` is a cudaStream_t passed as void*.  NULL means the legacy default
+ *     stream.  Work is enqueued asynchronously on it.
+ *   - Shapes, dtypes, alignment and workspace are checked on the host before any
+ *     launch.  A failed check returns a status and launches nothing.  A failed
+ *     launch returns BI_ERR_CUDA.  Kernels that wait on on-chip barriers give up
+ *     after a bounded number of polls.  They record a code in a device error word,
+ *     read back by bi_get_device_error().
+ *   - An empty batch (M == 0 or B == 0) is a valid no-op and returns BI_OK.
+ *   - Base pointers and row strides must be 16-byte aligned.  Otherwise the call
+ *     returns BI_ERR_MISALIGNED.
+ *   - Calls are thread-safe as long as their output buffers do not overlap.
+ *
+ * dtype codes: BI_F32 = IEEE binary32, BI_BF16 = bfloat16 (round to nearest even
+ * on output).
+ */
+#ifndef BI_H
+#define BI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bi_status {
+    BI_OK = 0,
+    BI_ERR_INVALID_ARG = 1,       /* null pointer, negative size, unknown dtype      */
+    BI_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside what the kernel is built for      */
+    BI_ERR_MISALIGNED = 3,        /* pointer or stride not 16-byte aligned           */
+    BI_ERR_WORKSPACE = 4,         /* workspace missing or smaller than required      */
+    BI_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed            */
+    BI_ERR_TIMEOUT = 6            /* a device-side bounded wait ran out              */
+} bi_status;
+
+typedef enum bi_dtype { BI_F32 = 0, BI_BF16 = 1 } bi_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* bi_status_str(int status);
+
+/* ABI version of this header: 1. */
+int bi_abi_version(void);
+
+/*
+ * Device error word.  Kernels that spin on an mbarrier or a cluster barrier stop
+ * after a bounded number of polls.  They OR a cause bit into a per-library device
+ * word and return early, and their outputs are then undefined.
+ * bi_get_device_error() synchronises `stream`, then reads the word into *code
+ * (0 = no error).  Return value: BI_OK, BI_ERR_TIMEOUT if *code != 0, or
+ * BI_ERR_CUDA.  bi_clear_device_error() zeroes the word, ordered on `stream`.
+ */
+int bi_get_device_error(uint32_t* code, void* stream);
+int bi_clear_device_error(void* stream);
+
+/*
+ * bi_rmsnorm -- y[m, :] = x[m, :] / sqrt(mean_j x[m, j]^2 + eps) * w
+ *
+ * Source: "Defeating Nondeterminism in LLM Inference" (Spanish summary), section
+ * "Diseño de kernels invariantes al batch", RMSNorm.  It uses a data-parallel
+ * strategy: each batch element is handled by one core, with the same strategy at
+ * every batch size.  The page prints no formula.  The Llama form is read here:
+ * the mean is over H, eps is inside the square root, and the weight w is applied
+ * as is.
+ *
+ *   x    device, [M, H] row-major, row stride ldx elements, dtype io_dtype
+ *   w    device, [H], dtype w_dtype
+ *   y    device, [M, H] row-major, row stride ldy elements, dtype io_dtype.
+ *        y may alias x only if ldy == ldx (in-place).
+ *   M    rows (>= 0).  H: row length, > 0, a multiple of 16 bytes' worth of
+ *        elements (8 for bf16, 4 for fp32), at most 32768 (bf16) / 16384 (fp32).
+ *   eps  added to the mean square inside the square root.
+ *
+ * Arithmetic: fp32.  Each row is reduced by one CTA.  The tree is fixed by H:
+ * thread -> warp shuffle -> CTA.  Then inv = rsqrt_rn(sum/H + eps) and
+ * y = (x * inv) * w, rounded once to io_dtype.
+ */
+int bi_rmsnorm(const void* x, const void* w, void* y, int64_t M, int64_t H, int64_t ldx, int64_t ldy,
+               float eps, int io_dtype, int w_dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BI_H */

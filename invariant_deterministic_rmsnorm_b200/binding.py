@@ -1,0 +1,120 @@
+"""Thin ctypes binding over libbi.so, with the same names as the C ABI (include/bi.h).
+
+Argument marshalling only: every step of every op runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors; PyTorch provides device memory and
+the stream (the current stream by default).  If libbi.so is missing, loading
+raises an error.  There is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbi.so")
+
+BI_F32 = 0
+BI_BF16 = 1
+STATUS = {0: "BI_OK", 1: "BI_ERR_INVALID_ARG", 2: "BI_ERR_UNSUPPORTED_SHAPE", 3: "BI_ERR_MISALIGNED",
+          4: "BI_ERR_WORKSPACE", 5: "BI_ERR_CUDA", 6: "BI_ERR_TIMEOUT"}
+
+
+class BIError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Load libbi.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libbi.so not found at {LIB_PATH}; build it with "
+                               "`python -m invariant_deterministic_rmsnorm_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        _declare(lib)
+        _lib = lib
+    return _lib
+
+
+def _declare(lib: ctypes.CDLL) -> None:
+    P, I64, I32, F, Z = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    C = ctypes.c_int
+    sig = {
+        "bi_status_str": ([C], ctypes.c_char_p),
+        "bi_abi_version": ([], C),
+        "bi_get_device_error": ([P, P], C),
+        "bi_clear_device_error": ([P], C),
+        "bi_rmsnorm": ([P, P, P, I64, I64, I64, I64, F, C, C, P], C),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise BIError(fn, status)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return BI_F32
+    if t.dtype == torch.bfloat16:
+        return BI_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float32 or bfloat16")
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _rows(t: torch.Tensor, name: str) -> None:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with unit stride along the last dimension")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+# ------------------------------------------------------------------ ops
+def bi_rmsnorm(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, eps: float = 1e-6,
+               stream=None) -> torch.Tensor:
+    """y = x / sqrt(mean(x^2) + eps) * w, row by row.  x, y [M, H] (fp32 or bf16); w [H]."""
+    _rows(x, "x")
+    if y is None:
+        y = torch.empty_like(x, memory_format=torch.contiguous_format)
+    _rows(y, "y")
+    if w.dim() != 1 or not w.is_contiguous() or not w.is_cuda:
+        raise ValueError("w must be a contiguous 1-D CUDA tensor")
+    if y.dtype != x.dtype or tuple(y.shape) != tuple(x.shape):
+        raise ValueError("y must match x in shape and dtype")
+    M, H = x.shape
+    st = library().bi_rmsnorm(_ptr(x), _ptr(w), _ptr(y), M, H, max(x.stride(0), H), max(y.stride(0), H),
+                              float(eps), _dtype_code(x), _dtype_code(w), _stream(stream))
+    _check("bi_rmsnorm", st)
+    return y
+
+
+def bi_get_device_error(stream=None) -> int:
+    code = ctypes.c_uint32(0)
+    st = library().bi_get_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (0, 6):
+        raise BIError("bi_get_device_error", st)
+    return int(code.value)
+
+
+def bi_clear_device_error(stream=None) -> None:
+    _check("bi_clear_device_error", library().bi_clear_device_error(_stream(stream)))

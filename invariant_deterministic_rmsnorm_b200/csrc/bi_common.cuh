@@ -1,0 +1,66 @@
+// bi_common.cuh -- shared host/device helpers for the libbi.so kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "bi.h"
+
+#define BI_API extern "C" __attribute__((visibility("default")))
+
+namespace bi {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+// Device address of the library's error word on the current device (bi_abi.cu).
+uint32_t* device_error_word();
+
+inline int elem_size(int dtype) { return dtype == BI_F32 ? 4 : (dtype == BI_BF16 ? 2 : 0); }
+
+// Device error word bits (OR-ed by kernels whose bounded waits ran out).
+enum : uint32_t {
+    DEVERR_WAIT_TMA = 1u << 0,      // producer waited too long for a free stage
+    DEVERR_WAIT_FULL = 1u << 1,     // MMA issuer waited too long for a loaded stage
+    DEVERR_WAIT_ACCUM = 1u << 2,    // epilogue waited too long for the accumulator
+    DEVERR_WAIT_CLUSTER = 1u << 3,  // cluster barrier / DSMEM handshake ran out
+};
+
+// ------------------------------------------------------------------ device helpers
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint4 ld_cached_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// bf16 pair <-> two floats.  The unpack is exact: a bf16 is the top half of a binary32.
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Two floats -> packed bf16x2, each rounded to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+}  // namespace bi

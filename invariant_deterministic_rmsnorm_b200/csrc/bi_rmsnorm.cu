@@ -1,0 +1,195 @@
+// bi_rmsnorm.cu -- batch-invariant RMSNorm: one CTA per row, reduction tree fixed by H.
+//
+// Source: "Defeating Nondeterminism in LLM Inference" (Spanish summary), section
+// "Diseño de kernels invariantes al batch", RMSNorm.  That section asks for a
+// data-parallel strategy in which one core handles each batch element.  The
+// strategy must not change with batch size.  The small-batch split-reduction
+// variant the section mentions gives up invariance and is not used here.
+//
+// Launch plan, a function of (H, dtypes) only:
+//   vec     = 16 bytes / element size (8 bf16 or 4 fp32 elements per 128-bit load)
+//   nvec    = H / vec
+//   threads = min(256, nvec rounded up to a warp)
+//   vpt     = ceil(nvec / threads) vectors per thread (compile-time 1, 2, 4, 8 or 16)
+// Thread t owns vectors t, t + threads, t + 2*threads, ...  It keeps them in
+// registers (one HBM read of x), sums their squares sequentially with fused
+// multiply-adds, then joins a butterfly shuffle tree within its warp and a second
+// fixed tree over the warps.  Because the plan depends on H alone, every row is
+// reduced in exactly the same order at every M and every row position.
+#include "bi_common.cuh"
+
+namespace {
+
+constexpr int kMaxThreads = 256;
+
+template <typename TIO>
+struct IoTraits;
+template <>
+struct IoTraits<float> {
+    static constexpr int kVec = 4;
+    static __device__ __forceinline__ void unpack(const uint4& u, float (&f)[4]) {
+        f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+    }
+    static __device__ __forceinline__ uint4 pack(const float (&f)[4]) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                          __float_as_uint(f[3]));
+    }
+};
+template <>
+struct IoTraits<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    static __device__ __forceinline__ void unpack(const uint4& u, float (&f)[8]) {
+        f[0] = bi::bf16_lo(u.x); f[1] = bi::bf16_hi(u.x); f[2] = bi::bf16_lo(u.y); f[3] = bi::bf16_hi(u.y);
+        f[4] = bi::bf16_lo(u.z); f[5] = bi::bf16_hi(u.z); f[6] = bi::bf16_lo(u.w); f[7] = bi::bf16_hi(u.w);
+    }
+    static __device__ __forceinline__ uint4 pack(const float (&f)[8]) {
+        return make_uint4(bi::pack_bf16x2(f[0], f[1]), bi::pack_bf16x2(f[2], f[3]),
+                          bi::pack_bf16x2(f[4], f[5]), bi::pack_bf16x2(f[6], f[7]));
+    }
+};
+
+// Load kVec weights of type TW starting at element index e0 and widen to fp32.
+template <typename TW, int V>
+__device__ __forceinline__ void load_w(const TW* w, int64_t e0, float (&f)[V]) {
+    if constexpr (sizeof(TW) == 4) {
+#pragma unroll
+        for (int i = 0; i < V; i += 4) {
+            uint4 u = bi::ld_cached_v4(reinterpret_cast<const float*>(w) + e0 + i);
+            f[i] = __uint_as_float(u.x); f[i + 1] = __uint_as_float(u.y);
+            f[i + 2] = __uint_as_float(u.z); f[i + 3] = __uint_as_float(u.w);
+        }
+    } else if constexpr (V == 4) {  // fp32 rows with bf16 weights: 4 weights = 8 bytes
+        uint2 u;
+        asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(u.x), "=r"(u.y)
+                     : "l"(reinterpret_cast<const __nv_bfloat16*>(w) + e0));
+        f[0] = bi::bf16_lo(u.x); f[1] = bi::bf16_hi(u.x); f[2] = bi::bf16_lo(u.y); f[3] = bi::bf16_hi(u.y);
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; i += 8) {
+            uint4 u = bi::ld_cached_v4(reinterpret_cast<const __nv_bfloat16*>(w) + e0 + i);
+            f[i] = bi::bf16_lo(u.x); f[i + 1] = bi::bf16_hi(u.x); f[i + 2] = bi::bf16_lo(u.y);
+            f[i + 3] = bi::bf16_hi(u.y); f[i + 4] = bi::bf16_lo(u.z); f[i + 5] = bi::bf16_hi(u.z);
+            f[i + 6] = bi::bf16_lo(u.w); f[i + 7] = bi::bf16_hi(u.w);
+        }
+    }
+}
+
+template <typename TIO, typename TW, int VPT>
+__global__ void __launch_bounds__(kMaxThreads)
+rmsnorm_rows_kernel(const TIO* __restrict__ x, const TW* __restrict__ w, TIO* __restrict__ y, int nvec,
+                    int64_t ldx, int64_t ldy, float h_float, float eps) {
+    constexpr int V = IoTraits<TIO>::kVec;
+    __shared__ float warp_sums[kMaxThreads / 32];
+    __shared__ float row_total;
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int nthreads = blockDim.x;
+    const int64_t row = blockIdx.x;
+    const TIO* xr = x + row * ldx;
+    TIO* yr = y + row * ldy;
+
+    // 1. Stream this thread's vectors of the row into registers (all loads issued first).
+    uint4 xv[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = tid + i * nthreads;
+        xv[i] = (v < nvec) ? bi::ld_stream_v4(xr + (int64_t)v * V) : make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    // 2. Per-thread sum of squares, vectors in order, elements in order.
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        float f[V];
+        IoTraits<TIO>::unpack(xv[i], f);
+#pragma unroll
+        for (int e = 0; e < V; ++e) ss = __fmaf_rn(f[e], f[e], ss);
+    }
+
+    // 3. Warp butterfly.  Partners add the same two values, so every lane ends with the same bits.
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
+    if (lane == 0) warp_sums[warp] = ss;
+    __syncthreads();
+
+    // 4. Fixed tree over the warps (missing warps contribute +0, which is exact).
+    if (warp == 0) {
+        const int nwarps = nthreads >> 5;
+        float t = (lane < nwarps) ? warp_sums[lane] : 0.0f;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
+        if (lane == 0) row_total = t;
+    }
+    __syncthreads();
+
+    const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(row_total, h_float), eps));
+
+    // 5. y = (x * inv) * w, one rounding to the output type.
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = tid + i * nthreads;
+        if (v < nvec) {
+            float f[V], wf[V];
+            IoTraits<TIO>::unpack(xv[i], f);
+            load_w<TW, V>(w, (int64_t)v * V, wf);
+#pragma unroll
+            for (int e = 0; e < V; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], inv), wf[e]);
+            bi::st_stream_v4(yr + (int64_t)v * V, IoTraits<TIO>::pack(f));
+        }
+    }
+}
+
+template <typename TIO, typename TW>
+int launch_typed(const void* x, const void* w, void* y, int64_t M, int64_t H, int64_t ldx, int64_t ldy, float eps,
+                 cudaStream_t s) {
+    constexpr int V = IoTraits<TIO>::kVec;
+    const int nvec = (int)(H / V);
+    int threads = ((nvec + 31) / 32) * 32;
+    if (threads > kMaxThreads) threads = kMaxThreads;
+    const int vpt = (nvec + threads - 1) / threads;
+    dim3 grid((unsigned)M), block(threads);
+    const TIO* xp = static_cast<const TIO*>(x);
+    const TW* wp = static_cast<const TW*>(w);
+    TIO* yp = static_cast<TIO*>(y);
+    const float hf = (float)H;
+    switch (vpt) {
+        case 1: rmsnorm_rows_kernel<TIO, TW, 1><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
+        case 2: rmsnorm_rows_kernel<TIO, TW, 2><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
+        case 3: case 4:
+            rmsnorm_rows_kernel<TIO, TW, 4><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
+        case 5: case 6: case 7: case 8:
+            rmsnorm_rows_kernel<TIO, TW, 8><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
+        default:
+            rmsnorm_rows_kernel<TIO, TW, 16><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
+    }
+    return bi::launch_status();
+}
+
+}  // namespace
+
+BI_API int bi_rmsnorm(const void* x, const void* w, void* y, int64_t M, int64_t H, int64_t ldx, int64_t ldy,
+                      float eps, int io_dtype, int w_dtype, void* stream) {
+    const int es = bi::elem_size(io_dtype);
+    const int ws = bi::elem_size(w_dtype);
+    if (es == 0 || ws == 0) return BI_ERR_INVALID_ARG;
+    if (M < 0 || H <= 0 || ldx < H || ldy < H || !(eps >= 0.0f)) return BI_ERR_INVALID_ARG;
+    if (M == 0) return BI_OK;
+    if (!x || !w || !y) return BI_ERR_INVALID_ARG;
+    if (M > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
+    const int vec = 16 / es;
+    if (H % vec != 0 || H % (16 / ws) != 0) return BI_ERR_MISALIGNED;
+    if ((ldx * es) % 16 != 0 || (ldy * es) % 16 != 0) return BI_ERR_MISALIGNED;
+    if (!bi::aligned16(x) || !bi::aligned16(w) || !bi::aligned16(y)) return BI_ERR_MISALIGNED;
+    if (H / vec > (int64_t)kMaxThreads * 16) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (y == x && ldy != ldx) return BI_ERR_INVALID_ARG;
+    cudaStream_t s = bi::as_stream(stream);
+    if (io_dtype == BI_F32 && w_dtype == BI_F32) return launch_typed<float, float>(x, w, y, M, H, ldx, ldy, eps, s);
+    if (io_dtype == BI_F32 && w_dtype == BI_BF16)
+        return launch_typed<float, __nv_bfloat16>(x, w, y, M, H, ldx, ldy, eps, s);
+    if (io_dtype == BI_BF16 && w_dtype == BI_BF16)
+        return launch_typed<__nv_bfloat16, __nv_bfloat16>(x, w, y, M, H, ldx, ldy, eps, s);
+    return launch_typed<__nv_bfloat16, float>(x, w, y, M, H, ldx, ldy, eps, s);
+}

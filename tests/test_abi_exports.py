@@ -1,0 +1,71 @@
+"""libbi.so loads on a machine without a GPU and exports every entry point include/*.h declares.
+
+Only host-side paths run here: status strings, the ABI version and argument
+checks that return before any CUDA call (null pointers, negative sizes, bad
+dtypes, misaligned addresses, empty batches).
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from invariant_deterministic_rmsnorm_b200 import build as bi_build
+from invariant_deterministic_rmsnorm_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+char\s*\*|int|size_t|void)\s+(bi_\w+)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    bi_build.build()
+    return binding.library()
+
+
+def test_headers_declare_entry_points():
+    names = _declared()
+    for required in ("bi_rmsnorm", "bi_status_str", "bi_get_device_error"):
+        assert required in names
+
+
+@pytest.mark.parametrize("name", _declared())
+def test_symbol_exported(lib, name):
+    assert hasattr(lib, name), f"{name} declared in include/ but not exported by libbi.so"
+
+
+def test_status_strings(lib):
+    assert lib.bi_abi_version() == 1
+    for code, name in binding.STATUS.items():
+        assert lib.bi_status_str(code).decode() == name
+    assert lib.bi_status_str(99).decode() == "BI_ERR_UNKNOWN"
+
+
+def _rms(lib, x, w, y, M, H, ldx=None, ldy=None, eps=1e-6, io=0, wd=0):
+    P = ctypes.c_void_p
+    return lib.bi_rmsnorm(P(x), P(w), P(y), M, H, ldx if ldx is not None else H, ldy if ldy is not None else H,
+                          eps, io, wd, None)
+
+
+def test_rmsnorm_host_checks(lib):
+    a = 1 << 20  # a 16-byte aligned fake address; never dereferenced on these paths
+    assert _rms(lib, a, a, a, 0, 256) == 0                 # empty batch: no-op
+    assert _rms(lib, None, a, a, 4, 256) == 1              # null x
+    assert _rms(lib, a, a, a, -1, 256) == 1                # negative M
+    assert _rms(lib, a, a, a, 4, 0) == 1                   # H = 0
+    assert _rms(lib, a, a, a, 4, 256, io=7) == 1           # unknown dtype
+    assert _rms(lib, a, a, a, 4, 256, eps=-1.0) == 1       # negative eps
+    assert _rms(lib, a, a, a, 4, 256, ldx=100) == 1        # ldx < H
+    assert _rms(lib, a + 4, a, a, 4, 256) == 3             # misaligned x
+    assert _rms(lib, a, a, a, 4, 258) == 3                 # H not a multiple of 4 fp32
+    assert _rms(lib, a, a, a, 4, 256, ldx=258) == 3        # row stride not 16-byte aligned
+    assert _rms(lib, a, a, a, 4, 1 << 16) == 2             # H beyond the in-register plan
+    assert _rms(lib, a, a, a, 4, 256, ldy=260) == 1        # in place with a different row stride
