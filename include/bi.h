@@ -94,6 +94,33 @@ int bi_clear_device_error(void* stream);
 int bi_rmsnorm(const void* x, const void* w, void* y, int64_t M, int64_t H, int64_t ldx, int64_t ldy,
                float eps, int io_dtype, int w_dtype, void* stream);
 
+/*
+ * bi_gemm -- C[M, N] = A[M, K] . W[K, N]
+ *
+ * Source: "Defeating Nondeterminism in LLM Inference" (Spanish summary), section
+ * "Multiplicación de matrices".  The matmul is tile-parallel over 2-D tiles on
+ * tensor cores.  A split-K chosen for small batches breaks batch invariance.  The
+ * remedy is to force the same kernel configuration for every batch size.
+ *
+ *   A    device, bf16 [M, K] row-major (K contiguous)
+ *   W    device, bf16 [K, N] row-major (N contiguous), the weight
+ *   C    device, [M, N] row-major, dtype c_dtype (BI_F32: the fp32 accumulator as is;
+ *        BI_BF16: the accumulator rounded to nearest even)
+ *   M    >= 0 rows.  N, K > 0, multiples of 8 (16-byte rows for the TMA unit).
+ *        M <= 65535*128.
+ *   ws, ws_bytes  workspace, at least bi_gemm_workspace_size(M, N, K) bytes.  That
+ *        size is 0 for every shape this version supports, so ws may be NULL.
+ *
+ * Arithmetic: tcgen05.mma 128x256x16, bf16 x bf16 -> fp32 in tensor memory.  The tile
+ * is 128 rows x 256 columns and K is walked in ascending 64-wide blocks.  The plan
+ * (tile, MMA shape, K order, split count) is a function of (N, K) only.  Rows past M
+ * and columns past N or K are zero-filled on load and never stored.  C may not
+ * alias A or W.
+ */
+size_t bi_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype, void* ws,
+            size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,6 +52,8 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_get_device_error": ([P, P], C),
         "bi_clear_device_error": ([P], C),
         "bi_rmsnorm": ([P, P, P, I64, I64, I64, I64, F, C, C, P], C),
+        "bi_gemm_workspace_size": ([I64, I64, I64], Z),
+        "bi_gemm": ([P, P, P, I64, I64, I64, C, P, Z, P], C),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -106,6 +108,32 @@ def bi_rmsnorm(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, 
                               float(eps), _dtype_code(x), _dtype_code(w), _stream(stream))
     _check("bi_rmsnorm", st)
     return y
+
+
+def bi_gemm(A: torch.Tensor, W: torch.Tensor, C: torch.Tensor | None = None, out_dtype=torch.float32,
+            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """C = A @ W with A [M, K] bf16, W [K, N] bf16 (both row-major contiguous); C fp32 or bf16 [M, N]."""
+    for t, n in ((A, "A"), (W, "W")):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 2 or not t.is_cuda:
+            raise ValueError(f"{n} must be a contiguous 2-D bf16 CUDA tensor")
+    M, K = A.shape
+    K2, N = W.shape
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    if C is None:
+        C = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    if tuple(C.shape) != (M, N) or not C.is_contiguous():
+        raise ValueError("C must be a contiguous [M, N] tensor")
+    lib = library()
+    need = lib.bi_gemm_workspace_size(M, N, K)
+    ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
+    if need:
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=A.device)
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    st = lib.bi_gemm(_ptr(A), _ptr(W), _ptr(C), M, N, K, _dtype_code(C), ws_ptr, ws_bytes, _stream(stream))
+    _check("bi_gemm", st)
+    return C
 
 
 def bi_get_device_error(stream=None) -> int:

@@ -1,0 +1,272 @@
+// bi_gemm.cu -- batch-invariant dense GEMM on tcgen05 tensor cores (sm_100a).
+//
+// C[M, N] = A[M, K] . W[K, N], bf16 operands, fp32 accumulation in TMEM, fp32 or bf16 output.
+//
+// Source: "Defeating Nondeterminism in LLM Inference" (Spanish summary), section
+// "Multiplicación de matrices".  The matmul is tile-parallel over 2-D output tiles.
+// Small batches tempt implementations into split-K, and a split chosen by batch size
+// breaks batch invariance.  The fix the section gives is to force one kernel
+// configuration for every batch size.  Here the configuration is fixed by (N, K)
+// alone: the tile (128 x 256), the MMA shape (128 x 256 x 16), the K-block order
+// (ascending, 64 at a time) and the split count (1).  A row's tile position and
+// the batch size M change which CTA computes the row.  They never change the
+// instructions that produce its bits.  Rows past M are zero-filled by the TMA unit
+// and are never stored.
+//
+// CTA structure (192 threads):
+//   warp 0      TMA producer: A tile [128 x 64] and W tile [64 x 256] per stage, 4-stage ring
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (4 MMAs of K = 16 per stage)
+//   warps 2..5  epilogue: tcgen05.ld of the 128 x 256 fp32 accumulator, convert, store
+// Shared-memory operand layouts are the 128-byte-swizzled canonical forms that the TMA
+// unit writes.  A is K-major (one 128-byte row per M row).  W is N-major: four boxes
+// of 64 N-columns x 64 K-rows, the leading-dimension offset is the box stride (8 KB),
+// and the stride offset is 8 K-rows (1 KB).
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "bi_common.cuh"
+#include "bi_sm100.cuh"
+
+using namespace bi::sm100;
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int UMMA_K = 16;
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK * 2;  // 16 KB
+constexpr int B_BOX = 64 * BK * 2;    // 8 KB: 64 N-columns x 64 K-rows
+constexpr int B_STAGE = BN * BK * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
+constexpr int TMEM_COLS = 256;
+constexpr int THREADS = 192;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+
+struct Bars {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t accum;
+    uint32_t tmem_addr;
+    int abort;
+};
+
+__device__ __forceinline__ void fail(uint32_t* err, volatile int* abort, uint32_t bit) {
+    atomicOr(err, bit);
+    *abort = 1;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                       void* __restrict__ C, int M, int N, int K, int c_bf16, uint32_t* err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * A_STAGE;
+    Bars* bars = reinterpret_cast<Bars*>(sB + STAGES * B_STAGE);
+    volatile int* abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN;
+    const int m0 = blockIdx.y * BM;
+    const int num_kb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&bars->full[s]), 1);
+            mbar_init(smem_u32(&bars->empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bars->accum), 1);
+        bars->abort = 0;
+        fence_barrier_init();
+        fence_proxy_async_shared();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&bars->tmem_addr), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = bars->tmem_addr;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t round = (uint32_t)(kb / STAGES);
+                if (!mbar_wait(smem_u32(&bars->empty[s]), (round & 1u) ^ 1u, abort)) {
+                    fail(err, abort, bi::DEVERR_WAIT_TMA);
+                    break;
+                }
+                const uint32_t fb = smem_u32(&bars->full[s]);
+                mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                tma_load_2d(smem_u32(sA + s * A_STAGE), &tmA, kb * BK, m0, fb);
+#pragma unroll
+                for (int j = 0; j < BN / 64; ++j)
+                    tma_load_2d(smem_u32(sB + s * B_STAGE + j * B_BOX), &tmW, n0 + 64 * j, kb * BK, fb);
+                ++issued;
+            }
+            if (*abort) {  // let loads already in flight land before the CTA's shared memory is released
+                for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
+                    (void)mbar_wait(smem_u32(&bars->full[kb % STAGES]), (uint32_t)(kb / STAGES) & 1u, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc_bf16_f32(BM, BN, 0, 1);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t round = (uint32_t)(kb / STAGES);
+                if (!mbar_wait(smem_u32(&bars->full[s]), round & 1u, abort)) {
+                    fail(err, abort, bi::DEVERR_WAIT_FULL);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(sA + s * A_STAGE);
+                const uint32_t b_base = smem_u32(sB + s * B_STAGE);
+#pragma unroll
+                for (int k = 0; k < BK / UMMA_K; ++k) {
+                    // A: K-major, 128B swizzle; the k-th 16-element slice starts 32 bytes further along the row.
+                    const uint64_t adesc = make_smem_desc(a_base + k * UMMA_K * 2, 16, 1024, 2);
+                    // W: N-major, 128B swizzle; 16 K-rows of 128 bytes each per step.
+                    const uint64_t bdesc = make_smem_desc(b_base + k * UMMA_K * 128, B_BOX, 1024, 2);
+                    mma_bf16_ss(tmem_base, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+                }
+                mma_commit(smem_u32(&bars->empty[s]));  // stage free once these MMAs have read it
+            }
+            mma_commit(smem_u32(&bars->accum));  // accumulator complete
+        }
+    } else {
+        const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter .. +31
+        const bool ok = mbar_wait(smem_u32(&bars->accum), 0u, abort);
+        if (!ok) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+        // tcgen05.ld is warp-collective: the whole warp takes the same branch
+        if (__all_sync(0xffffffffu, ok && !*abort)) {
+            tc_fence_after();
+            const int row = m0 + quarter * 32 + lane;
+            const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(lane_addr + (uint32_t)c, r);
+                tmem_wait_ld();
+                const int col = n0 + c;
+                if (row < M && col < N) {
+                    if (!c_bf16) {
+                        float* dst = static_cast<float*>(C) + (int64_t)row * N + col;
+                        if (col + 32 <= N) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<uint4*>(dst + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < N - col) dst[i] = __uint_as_float(r[i]);
+                        }
+                    } else {
+                        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(C) + (int64_t)row * N + col;
+                        uint32_t p[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            p[i] = bi::pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        if (col + 32 <= N) {
+#pragma unroll
+                            for (int i = 0; i < 16; i += 4)
+                                *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(p[i], p[i + 1], p[i + 2], p[i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < N - col) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// bf16 row-major [outer, inner] matrix, box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool ensure_smem_attr() {
+    static std::once_flag once[64];
+    static bool ok[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::call_once(once[dev], [&] {
+        ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES) == cudaSuccess;
+    });
+    return ok[dev];
+}
+
+}  // namespace
+
+BI_API size_t bi_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+    (void)M; (void)N; (void)K;
+    return 0;
+}
+
+BI_API int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype, void* ws,
+                   size_t ws_bytes, void* stream) {
+    (void)ws; (void)ws_bytes;
+    if (c_dtype != BI_F32 && c_dtype != BI_BF16) return BI_ERR_INVALID_ARG;
+    if (M < 0 || N <= 0 || K <= 0) return BI_ERR_INVALID_ARG;
+    if (M == 0) return BI_OK;
+    if (!A || !W || !C) return BI_ERR_INVALID_ARG;
+    if (!bi::aligned16(A) || !bi::aligned16(W) || !bi::aligned16(C)) return BI_ERR_MISALIGNED;
+    if (K % 8 != 0 || N % 8 != 0) return BI_ERR_MISALIGNED;  // 16-byte row strides for the TMA unit
+    if (M > (int64_t)65535 * BM || N > (int64_t)65535 * BN || K > (1LL << 30)) return BI_ERR_UNSUPPORTED_SHAPE;
+    uint32_t* err = bi::device_error_word();
+    if (!err || !ensure_smem_attr()) return BI_ERR_CUDA;
+    CUtensorMap tmA, tmW;
+    if (!make_tmap_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM)) return BI_ERR_CUDA;
+    if (!make_tmap_bf16(&tmW, W, (uint64_t)N, (uint64_t)K, (uint64_t)N * 2, 64, BK)) return BI_ERR_CUDA;
+    dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+    bi_gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, bi::as_stream(stream)>>>(
+        tmA, tmW, C, (int)M, (int)N, (int)K, c_dtype == BI_BF16 ? 1 : 0, err);
+    return bi::launch_status();
+}

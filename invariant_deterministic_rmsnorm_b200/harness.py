@@ -131,3 +131,53 @@ def pin_tuple(extra: dict | None = None) -> dict:
     if extra:
         d.update(extra)
     return d
+
+
+def bi_check_rows(op: str, run, probes, filler, m_list: Sequence[int], trials: int = 3,
+                  seed_positions: int = inputs.SEED_POSITIONS, report: BIReport | None = None) -> BIReport:
+    """Row-batch form of ``bi_check`` on torch tensors, batches assembled where the tensors live.
+
+    run(batch [M, ...]) -> out [M, ...]; probes [P, ...]; filler(trial) -> tensor [>= max(m_list), ...].
+    Outputs are compared as raw bits (viewed as integers of the same width).
+    """
+    import torch
+
+    def bits(t):
+        return t.contiguous().view({1: torch.uint8, 2: torch.int16, 4: torch.int32, 8: torch.int64}[t.element_size()])
+
+    rep = report or BIReport(op)
+    P = probes.shape[0]
+    solo = [bits(run(probes[p:p + 1].clone())[0]).clone() for p in range(P)]
+    for M in m_list:
+        bad = 0
+        for trial in range(trials):
+            rng = np.random.default_rng([seed_positions, int(M), trial])
+            pos = rng.choice(M, size=min(M, P), replace=False)
+            batch = filler(trial)[:M].clone()
+            for p_idx, where in enumerate(pos):
+                batch[int(where)] = probes[p_idx]
+            out = run(batch)
+            for p_idx, where in enumerate(pos):
+                rep.comparisons += 1
+                if not torch.equal(bits(out[int(where)]), solo[p_idx]):
+                    bad += 1
+                    if rep.first_failure is None:
+                        diff = int((bits(out[int(where)]) != solo[p_idx]).sum())
+                        rep.first_failure = {"M": int(M), "trial": trial, "position": int(where), "probe": p_idx,
+                                             "differing_elements": diff}
+        rep.per_m[int(M)] = bad
+        rep.violations += bad
+    return rep
+
+
+def rerun_check_rows(run, batch, n: int = 10, report: BIReport | None = None, op: str = "") -> BIReport:
+    """Tensor form of ``rerun_check``: one fixed batch run n times, bitwise against the first run."""
+    import torch
+    rep = report or BIReport(op)
+    ref = run(batch).clone()
+    for _ in range(n - 1):
+        out = run(batch)
+        rep.reruns += 1
+        if not torch.equal(out.contiguous().view(torch.uint8), ref.contiguous().view(torch.uint8)):
+            rep.rerun_violations += 1
+    return rep

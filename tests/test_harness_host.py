@@ -66,3 +66,26 @@ def test_pin_tuple_has_fields():
     d = harness.pin_tuple({"config": "x"})
     for k in ("torch", "git", "utc", "config"):
         assert k in d
+
+
+def test_bi_check_rows_on_cpu_tensors():
+    import torch
+    g = torch.Generator().manual_seed(0)
+    probes = torch.randn(4, 16, generator=g)
+    fill = {t: torch.randn(64, 16, generator=torch.Generator().manual_seed(100 + t)) for t in range(3)}
+    rowwise = lambda b: torch.tanh(b) * 0.5
+    rep = harness.bi_check_rows("rowwise", rowwise, probes, lambda t: fill[t], [1, 5, 64])
+    assert rep.violations == 0 and rep.comparisons == 3 + 4 * 3 + 4 * 3
+    dep = lambda b: b * (1.0 + 1e-6 * b.shape[0])
+    assert harness.bi_check_rows("dep", dep, probes, lambda t: fill[t], [1, 5]).violations > 0
+    # a reduction whose order depends on M: the sum over a row split into M-dependent chunks
+    def split_sum(b):
+        chunks = 2 if b.shape[0] > 3 else 1
+        parts = torch.tensor_split(b, chunks, dim=1)
+        s = parts[0].sum(1, keepdim=True)
+        for p in parts[1:]:
+            s = s + p.sum(1, keepdim=True)
+        return s.expand_as(b).contiguous()
+    assert harness.bi_check_rows("split", split_sum, probes, lambda t: fill[t], [1, 8]).violations > 0
+    rep = harness.rerun_check_rows(rowwise, fill[0], n=5)
+    assert rep.reruns == 4 and rep.rerun_violations == 0
