@@ -84,10 +84,11 @@ def test_bf16_output():
     assert rel_frobenius(bf16_to_f64(Cb[rows]), ref) <= 2e-3
     # the bf16 output is the nearest-even rounding of the kernel's own fp32 accumulator
     assert np.array_equal(Cb, inputs.f32_to_bf16_bits(C32))
-    # elementwise: within one bf16 step of the exact value, relative to max(|r|, 1e-3 * rms(row))
+    # elementwise: bf16 rounding (at most 2^-8 relative to |r|) plus fp32 accumulation error,
+    # which scales with the row (bounded here by 2e-4 * rms(row))
     g = bf16_to_f64(Cb[rows])
-    den = np.maximum(np.abs(ref), 1e-3 * np.sqrt((ref ** 2).mean(axis=1, keepdims=True)))
-    assert np.max(np.abs(g - ref) / den) <= 2.0 ** -8 + 1e-4
+    rms = np.sqrt((ref ** 2).mean(axis=1, keepdims=True))
+    assert np.all(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-4 * rms)
 
 
 def test_full_size_sampled_rows():
