@@ -121,6 +121,50 @@ size_t bi_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype, void* ws,
             size_t ws_bytes, void* stream);
 
+/*
+ * bi_lora_shrink -- t[M, r] = x[M, K] . A[K, r], deterministic split-K
+ *
+ * Source: "Reproducible LoRA Inference Through Deterministic Split-K Reduction"
+ * (abstract).  A Split-K = 8 shrink keeps its parallelism but combines the per-slice
+ * FP32 partials in a fixed order instead of with floating-point atomic additions.  Its
+ * FP32 output is then identical under replay.
+ *
+ *   x     device, bf16 [M, K] row-major
+ *   A     device, bf16 [K, r] row-major (the LoRA down-projection)
+ *   t     device, fp32 [M, r] row-major, overwritten
+ *   r     8, 16, 32 or 64.  split_k: 1, 2, 4 or 8 (the workloads use 8).
+ *         K must be a multiple of 64 * split_k.
+ *   ws, ws_bytes  workspace of bi_lora_shrink_workspace_size() bytes.  That size is
+ *         always 0, because the partials never leave the chip.  ws may be NULL.
+ *
+ * Arithmetic: one cluster of split_k CTAs per 64-row tile.  CTA s accumulates its
+ * contiguous K slice with mma.sync (bf16 in, fp32 accumulate, K ascending).  CTA 0
+ * then adds the partials over distributed shared memory, s = 0, 1, ..., split_k-1 in
+ * order, each add rounded to nearest.  No atomics.  The plan depends on (K, r,
+ * split_k) only.
+ */
+size_t bi_lora_shrink_workspace_size(int64_t M, int64_t K, int32_t r, int32_t split_k);
+int bi_lora_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r, int32_t split_k,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * bi_lora_expand -- y[M, N] += scale * bf16(t)[M, r] . B[r, N], in place
+ *
+ * Source: the same abstract ("low-rank LoRA multiplications").  The low-rank product
+ * is added to the base layer's output.
+ *
+ *   t     device, fp32 [M, r] row-major (the shrink output).  It enters the product
+ *         rounded to bf16, nearest even.
+ *   B     device, bf16 [r, N] row-major (the LoRA up-projection)
+ *   y     device, [M, N] with row stride ldy elements, dtype y_dtype, read and written
+ *   r     8, 16, 32 or 64.  N: a multiple of 8.  scale: the LoRA scaling (alpha / r).
+ *
+ * Arithmetic: mma.sync, bf16 in, fp32 accumulate over r.  Then
+ * y = round_to_y_dtype(fma(scale, delta, y)), elementwise.
+ */
+int bi_lora_expand(const float* t, const void* B, void* y, int64_t M, int32_t r, int64_t N, int64_t ldy,
+                   float scale, int y_dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

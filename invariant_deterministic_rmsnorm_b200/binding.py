@@ -54,6 +54,10 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_rmsnorm": ([P, P, P, I64, I64, I64, I64, F, C, C, P], C),
         "bi_gemm_workspace_size": ([I64, I64, I64], Z),
         "bi_gemm": ([P, P, P, I64, I64, I64, C, P, Z, P], C),
+        "bi_lora_shrink_workspace_size": ([I64, I64, I32, I32], Z),
+        "bi_lora_shrink": ([P, P, P, I64, I64, I32, I32, P, Z, P], C),
+        "bi_lora_expand": ([P, P, P, I64, I32, I64, I64, F, C, P], C),
+        "bi_ctrl_lora_shrink_atomic": ([P, P, P, I64, I64, I32, I32, P], C),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -134,6 +138,61 @@ def bi_gemm(A: torch.Tensor, W: torch.Tensor, C: torch.Tensor | None = None, out
     st = lib.bi_gemm(_ptr(A), _ptr(W), _ptr(C), M, N, K, _dtype_code(C), ws_ptr, ws_bytes, _stream(stream))
     _check("bi_gemm", st)
     return C
+
+
+def _bf16_2d(t: torch.Tensor, name: str) -> None:
+    if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 2 or not t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous 2-D bf16 CUDA tensor")
+
+
+def bi_lora_shrink(x: torch.Tensor, A: torch.Tensor, t: torch.Tensor | None = None, split_k: int = 8,
+                   stream=None) -> torch.Tensor:
+    """t = x @ A (fp32 [M, r]), K cut into split_k slices whose partials are added in slice order."""
+    _bf16_2d(x, "x")
+    _bf16_2d(A, "A")
+    M, K = x.shape
+    K2, r = A.shape
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    if t is None:
+        t = torch.empty((M, r), dtype=torch.float32, device=x.device)
+    if t.dtype != torch.float32 or tuple(t.shape) != (M, r) or not t.is_contiguous():
+        raise ValueError("t must be a contiguous fp32 [M, r] tensor")
+    st = library().bi_lora_shrink(_ptr(x), _ptr(A), _ptr(t), M, K, r, split_k, ctypes.c_void_p(0), 0,
+                                  _stream(stream))
+    _check("bi_lora_shrink", st)
+    return t
+
+
+def bi_lora_expand(t: torch.Tensor, B: torch.Tensor, y: torch.Tensor, scale: float = 1.0,
+                   stream=None) -> torch.Tensor:
+    """y += scale * bf16(t) @ B in place; t fp32 [M, r], B bf16 [r, N], y [M, N] (row stride may exceed N)."""
+    if t.dtype != torch.float32 or not t.is_contiguous() or t.dim() != 2 or not t.is_cuda:
+        raise ValueError("t must be a contiguous fp32 2-D CUDA tensor")
+    _bf16_2d(B, "B")
+    _rows(y, "y")
+    M, r = t.shape
+    r2, N = B.shape
+    if r != r2 or tuple(y.shape) != (M, N):
+        raise ValueError("shape mismatch")
+    st = library().bi_lora_expand(_ptr(t), _ptr(B), _ptr(y), M, r, N, max(y.stride(0), N), float(scale),
+                                  _dtype_code(y), _stream(stream))
+    _check("bi_lora_expand", st)
+    return y
+
+
+def bi_ctrl_lora_shrink_atomic(x: torch.Tensor, A: torch.Tensor, t: torch.Tensor | None = None, split_k: int = 8,
+                               stream=None) -> torch.Tensor:
+    """Comparator: the same shrink with the partials combined by fp32 atomics (nondeterministic order)."""
+    _bf16_2d(x, "x")
+    _bf16_2d(A, "A")
+    M, K = x.shape
+    r = A.shape[1]
+    if t is None:
+        t = torch.empty((M, r), dtype=torch.float32, device=x.device)
+    st = library().bi_ctrl_lora_shrink_atomic(_ptr(x), _ptr(A), _ptr(t), M, K, r, split_k, _stream(stream))
+    _check("bi_ctrl_lora_shrink_atomic", st)
+    return t
 
 
 def bi_get_device_error(stream=None) -> int:

@@ -21,12 +21,11 @@
 // unit writes.  A is K-major (one 128-byte row per M row).  W is N-major: four boxes
 // of 64 N-columns x 64 K-rows, the leading-dimension offset is the box stride (8 KB),
 // and the stride offset is 8 K-rows (1 KB).
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
 #include "bi_common.cuh"
 #include "bi_sm100.cuh"
+#include "bi_tma_host.cuh"
 
 using namespace bi::sm100;
 
@@ -202,35 +201,6 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaDriverEntryPointQueryResult q;
-        void* p = nullptr;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// bf16 row-major [outer, inner] matrix, box [box_outer, box_inner], 128-byte swizzle, zero fill out of bounds.
-bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                    uint32_t box_inner, uint32_t box_outer) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 bool ensure_smem_attr() {
     static std::once_flag once[64];
     static bool ok[64];
@@ -263,8 +233,12 @@ BI_API int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, 
     uint32_t* err = bi::device_error_word();
     if (!err || !ensure_smem_attr()) return BI_ERR_CUDA;
     CUtensorMap tmA, tmW;
-    if (!make_tmap_bf16(&tmA, A, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM)) return BI_ERR_CUDA;
-    if (!make_tmap_bf16(&tmW, W, (uint64_t)N, (uint64_t)K, (uint64_t)N * 2, 64, BK)) return BI_ERR_CUDA;
+    if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK,
+                          BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    if (!bi::make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)N, (uint64_t)K, (uint64_t)N * 2, 64,
+                          BK, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
     dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
     bi_gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, bi::as_stream(stream)>>>(
         tmA, tmW, C, (int)M, (int)N, (int)K, c_dtype == BI_BF16 ? 1 : 0, err);
