@@ -165,6 +165,46 @@ int bi_lora_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K,
 int bi_lora_expand(const float* t, const void* B, void* y, int64_t M, int32_t r, int64_t N, int64_t ldy,
                    float scale, int y_dtype, void* stream);
 
+/*
+ * bi_decode_attn -- one decode step of grouped-query attention over a packed KV cache,
+ * split-KV with a FIXED split size.
+ *
+ * Source: "Defeating Nondeterminism in LLM Inference" (Spanish summary), section
+ * "Attention".  Split-KV (FlashDecoding) keeps the same reduction order if the split
+ * SIZE is fixed rather than the number of splits.  Cached and new keys/values share one
+ * consistent layout.
+ *
+ *   q          device, bf16 [B, Hq, head_dim], one query token per sequence
+ *   k, v       device, bf16 [total_tokens, Hkv, head_dim], the packed cache
+ *   kv_indptr  device, int32 [B + 1], non-decreasing.  Sequence b owns tokens
+ *              kv_indptr[b] .. kv_indptr[b] + kv_len[b] - 1.  Every kv_indptr[b] must be
+ *              a multiple of `chunk` and kv_indptr[B] <= total_tokens.  Tokens between
+ *              the end of a sequence and kv_indptr[b+1] are never read.
+ *   kv_len     device, int32 [B], 1 <= kv_len[b] <= kv_indptr[b+1] - kv_indptr[b]
+ *   Hq, Hkv    query / kv heads.  Hq / Hkv must be 1, 2, 4 or 8.  Query head h reads kv
+ *              head h / (Hq / Hkv).  head_dim must be 128.  chunk must be 256.
+ *   scale      score scale, usually 1/sqrt(head_dim)
+ *   out        device, [B, Hq, head_dim], dtype out_dtype
+ *   ws         device workspace of at least bi_decode_attn_workspace_size(total_tokens,
+ *              Hq, head_dim, chunk) bytes, 16-byte aligned.  It holds one fp32 partial
+ *              (head_dim values, the running max and the sum) per (256-token slot of the
+ *              cache, query head).  Its contents need no initialisation and are
+ *              overwritten.
+ *
+ * Arithmetic: chunk c of sequence b is its tokens [256c, min(256c + 256, L_b)).  Each
+ * chunk yields m_c = max s_j, l_c = sum exp(s_j - m_c) and o_c = sum exp(s_j - m_c) v_j,
+ * with s_j = scale * q . k_j (bf16 products, fp32 sums over fixed trees).  The chunks are
+ * merged in order c = 0, 1, ... with an fp32 log-sum-exp rescale, and out = o / l.
+ *
+ * Layout violations that only the device can see (kv_indptr not chunk-aligned, kv_len
+ * out of range) set bit 0x100 of the device error word.  The affected rows of out are
+ * then left unwritten.
+ */
+size_t bi_decode_attn_workspace_size(int64_t total_tokens, int32_t Hq, int32_t head_dim, int32_t chunk);
+int bi_decode_attn(const void* q, const void* k, const void* v, const int32_t* kv_indptr, const int32_t* kv_len,
+                   int32_t B, int64_t total_tokens, int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
+                   int32_t chunk, void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

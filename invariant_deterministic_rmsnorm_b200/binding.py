@@ -58,6 +58,8 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_lora_shrink": ([P, P, P, I64, I64, I32, I32, P, Z, P], C),
         "bi_lora_expand": ([P, P, P, I64, I32, I64, I64, F, C, P], C),
         "bi_ctrl_lora_shrink_atomic": ([P, P, P, I64, I64, I32, I32, P], C),
+        "bi_decode_attn_workspace_size": ([I64, I32, I32, I32], Z),
+        "bi_decode_attn": ([P, P, P, P, P, I32, I64, I32, I32, I32, F, I32, P, C, P, Z, P], C),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -193,6 +195,43 @@ def bi_ctrl_lora_shrink_atomic(x: torch.Tensor, A: torch.Tensor, t: torch.Tensor
     st = library().bi_ctrl_lora_shrink_atomic(_ptr(x), _ptr(A), _ptr(t), M, K, r, split_k, _stream(stream))
     _check("bi_ctrl_lora_shrink_atomic", st)
     return t
+
+
+def bi_decode_attn_workspace_size(total_tokens: int, Hq: int, head_dim: int = 128, chunk: int = 256) -> int:
+    return int(library().bi_decode_attn_workspace_size(total_tokens, Hq, head_dim, chunk))
+
+
+def bi_decode_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_indptr: torch.Tensor,
+                   kv_len: torch.Tensor, out: torch.Tensor | None = None, scale: float | None = None,
+                   chunk: int = 256, out_dtype=torch.bfloat16, workspace: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """Decode attention: q [B, Hq, D] against the packed cache k, v [T, Hkv, D] (bf16).
+
+    kv_indptr int32 [B + 1] (chunk-aligned sequence starts), kv_len int32 [B].  A workspace of
+    bi_decode_attn_workspace_size(T, Hq) bytes is allocated here when none is passed."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3 or not t.is_cuda:
+            raise ValueError(f"{n} must be a contiguous 3-D bf16 CUDA tensor")
+    for t, n in ((kv_indptr, "kv_indptr"), (kv_len, "kv_len")):
+        if t.dtype != torch.int32 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{n} must be a contiguous int32 CUDA tensor")
+    B, Hq, D = q.shape
+    T, Hkv, D2 = k.shape
+    if tuple(v.shape) != tuple(k.shape) or D2 != D or kv_indptr.numel() != B + 1 or kv_len.numel() != B:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=out_dtype, device=q.device)
+    lib = library()
+    need = lib.bi_decode_attn_workspace_size(T, Hq, D, chunk)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib.bi_decode_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_indptr), _ptr(kv_len), B, T, Hq, Hkv, D,
+                            float(scale), chunk, _ptr(out), _dtype_code(out), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("bi_decode_attn", st)
+    return out
 
 
 def bi_get_device_error(stream=None) -> int:
