@@ -189,6 +189,20 @@ def build_ops(device, stream):
     return ops, io
 
 
+def reduce_over_ranks(times_ms, violations, world, device):
+    """Replicas: every timing becomes its max over ranks, the violation counts are summed.
+    The only collectives in the benchmark; none touches the data path."""
+    if world <= 1:
+        return list(times_ms), int(violations)
+    import torch
+    import torch.distributed as dist
+    vals = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    vsum = torch.tensor([float(violations)], dtype=torch.float64, device=device)
+    dist.all_reduce(vsum, op=dist.ReduceOp.SUM)
+    return vals.tolist(), int(vsum.item())
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -274,13 +288,7 @@ def run_ours(args, rank, world, local_rank):
     viol = bi_spot_check(device, stream)
 
     clocks = clk.summary()
-    vals = torch.tensor([total_ms, e2e_ms] + op_ms, dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-        vsum = torch.tensor([float(viol)], dtype=torch.float64, device=device)
-        dist.all_reduce(vsum, op=dist.ReduceOp.SUM)
-        viol = int(vsum.item())
-    total_ms, e2e_ms, *op_ms = vals.tolist()
+    (total_ms, e2e_ms, *op_ms), viol = reduce_over_ranks([total_ms, e2e_ms] + op_ms, viol, world, device)
     if rank != 0:
         return None
 
