@@ -205,6 +205,36 @@ int bi_decode_attn(const void* q, const void* k, const void* v, const int32_t* k
                    int32_t B, int64_t total_tokens, int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
                    int32_t chunk, void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * bi_decode_attn_noalloc -- bi_decode_attn without a caller-provided workspace.
+ *
+ * The pages have no counterpart for this entry point.  It exists for callers that
+ * cannot allocate device memory.  Examples: a plugin interface that hands the kernel
+ * only its input and output buffers and offers no allocator; a serving process whose
+ * memory pool already owns all of the GPU's free memory; a latency-critical loop where
+ * cudaMalloc's implicit device synchronisation is not acceptable.
+ *
+ * Arguments, layout, arithmetic and results are those of bi_decode_attn, minus ws and
+ * ws_bytes.  The per-chunk partials live in one fixed array of
+ * BI_DECODE_ATTN_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory inside libbi.so.  Every
+ * GPU that loads the library holds that array until the process exits.  The call
+ * allocates and frees nothing.
+ *
+ *   - Limit: the partials need bi_decode_attn_workspace_size(total_tokens, Hq, 128, 256)
+ *     bytes.  Beyond 16 MiB the call returns BI_ERR_WORKSPACE and launches nothing.
+ *     At Hq = 32 that is about 258,000 cache tokens; use bi_decode_attn for larger caches.
+ *   - The first call on each device looks up the array's device address with that
+ *     device current, then caches it.  Make that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps whatever the last call
+ *     left there.  Nothing in it needs to start at zero.  Calls whose work overlaps on
+ *     the GPU (on different streams, or from different host threads without ordering)
+ *     race on the array and corrupt each other's results: serialise them.
+ */
+#define BI_DECODE_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int bi_decode_attn_noalloc(const void* q, const void* k, const void* v, const int32_t* kv_indptr,
+                           const int32_t* kv_len, int32_t B, int64_t total_tokens, int32_t Hq, int32_t Hkv,
+                           int32_t head_dim, float scale, int32_t chunk, void* out, int out_dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

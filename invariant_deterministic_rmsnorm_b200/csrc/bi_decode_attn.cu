@@ -394,3 +394,80 @@ BI_API int bi_decode_attn(const void* q, const void* k, const void* v, const int
         decode_attn_merge_kernel<false><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
     return bi::launch_status();
 }
+
+// ------------------------------------------------------------------ no-allocation variant
+//
+// Some callers cannot allocate device memory at all.  Examples: a plugin interface
+// that hands a kernel only its input and output buffers and offers no allocator; a
+// serving process whose memory pool already owns all of the GPU's free memory; a
+// latency-critical loop where cudaMalloc's implicit device synchronisation is not
+// acceptable.  bi_decode_attn_noalloc serves them.  It runs the same two kernels as
+// bi_decode_attn.  Its per-chunk partials live in the fixed array below, which every
+// GPU that loads this library holds until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;  // 16 MiB; mirrored in bi.h
+
+// In host code this name is only a host-side stand-in for the symbol, not a device
+// address.  Host code must use the address from cudaGetSymbolAddress (below).
+static __device__ __align__(256) unsigned char g_decode_attn_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::once_flag g_scratch_once[kNoAllocMaxDevices];
+void* g_scratch_ptr[kNoAllocMaxDevices];
+
+// Device address of the scratch array on the current device.  It is looked up on the
+// first call made with that device current, then cached.  Returns nullptr if the
+// lookup fails.
+void* noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+    std::call_once(g_scratch_once[dev], [dev] {
+        void* p = nullptr;
+        g_scratch_ptr[dev] = (cudaGetSymbolAddress(&p, g_decode_attn_scratch) == cudaSuccess) ? p : nullptr;
+    });
+    return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+BI_API int bi_decode_attn_noalloc(const void* q, const void* k, const void* v, const int32_t* kv_indptr,
+                                  const int32_t* kv_len, int32_t B, int64_t total_tokens, int32_t Hq, int32_t Hkv,
+                                  int32_t head_dim, float scale, int32_t chunk, void* out, int out_dtype,
+                                  void* stream) {
+    if (out_dtype != BI_F32 && out_dtype != BI_BF16) return BI_ERR_INVALID_ARG;
+    if (B < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0 || !(scale == scale)) return BI_ERR_INVALID_ARG;
+    if (head_dim != D || chunk != CHUNK || Hq % Hkv != 0) return BI_ERR_UNSUPPORTED_SHAPE;
+    const int G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0) return BI_OK;
+    if (total_tokens == 0) return BI_ERR_INVALID_ARG;
+    if (total_tokens > 0x7fffffffLL || B > 65535 || Hq > 4096) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (!q || !k || !v || !kv_indptr || !kv_len || !out) return BI_ERR_INVALID_ARG;
+    if (!bi::aligned16(q) || !bi::aligned16(k) || !bi::aligned16(v) || !bi::aligned16(out)) return BI_ERR_MISALIGNED;
+    // The partials must fit in the fixed scratch array; larger caches are refused, not truncated.
+    if (partial_bytes(total_tokens, Hq) > kNoAllocScratchBytes) return BI_ERR_WORKSPACE;
+    void* scratch = noalloc_scratch();
+    if (!scratch) return BI_ERR_CUDA;
+    // Nothing in the scratch needs to start at zero: phase 1 writes every partial that
+    // phase 2 reads, and slots no sequence covers are never read.
+    float* o_part = static_cast<float*>(scratch);
+    const int64_t slots = (total_tokens + CHUNK - 1) / CHUNK;
+    float* ml_part = o_part + (size_t)slots * Hq * D;
+    cudaStream_t s = bi::as_stream(stream);
+    int st;
+    switch (G) {
+        case 1: st = launch_chunks<1>(q, k, v, kv_indptr, kv_len, B, total_tokens, Hq, Hkv, scale, o_part, ml_part, s); break;
+        case 2: st = launch_chunks<2>(q, k, v, kv_indptr, kv_len, B, total_tokens, Hq, Hkv, scale, o_part, ml_part, s); break;
+        case 4: st = launch_chunks<4>(q, k, v, kv_indptr, kv_len, B, total_tokens, Hq, Hkv, scale, o_part, ml_part, s); break;
+        default: st = launch_chunks<8>(q, k, v, kv_indptr, kv_len, B, total_tokens, Hq, Hkv, scale, o_part, ml_part, s); break;
+    }
+    if (st != BI_OK) return st;
+    uint32_t* err = bi::device_error_word();
+    dim3 grid((unsigned)((Hq + 3) / 4), (unsigned)B);
+    if (out_dtype == BI_BF16)
+        decode_attn_merge_kernel<true><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+    else
+        decode_attn_merge_kernel<false><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+    return bi::launch_status();
+}
