@@ -40,14 +40,17 @@ constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 constexpr int B_BOX = 64 * BK * 2;    // 8 KB: 64 N-columns x 64 K-rows
 constexpr int B_STAGE = BN * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
-constexpr int TMEM_COLS = 256;
+constexpr int ACC_COLS = BN;          // one fp32 accumulator = 256 TMEM columns
+constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 4;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
 
 struct Bars {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    uint64_t accum;
+    uint64_t tfull[2];   // accumulator b holds a finished tile
+    uint64_t tempty[2];  // accumulator b has been read out
     uint32_t tmem_addr;
     int abort;
 };
@@ -57,9 +60,22 @@ __device__ __forceinline__ void fail(uint32_t* err, volatile int* abort, uint32_
     *abort = 1;
 }
 
+// Tile order: groups of `gm` row tiles, walked column by column inside a group, so that the
+// tiles in flight at any moment share a few W column blocks and a few A row blocks in L2.
+// The order decides only which CTA computes a tile, never how.
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int gm, int& m_tile, int& n_tile) {
+    const int per_group = gm * tiles_n;
+    const int group = t / per_group;
+    const int first_m = group * gm;
+    const int gsm = min(tiles_m - first_m, gm);
+    const int r = t - group * per_group;
+    m_tile = first_m + r % gsm;
+    n_tile = r / gsm;
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
-                       void* __restrict__ C, int M, int N, int K, int c_bf16, uint32_t* err) {
+                       void* __restrict__ C, int M, int N, int K, int c_bf16, int gm, uint32_t* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -69,8 +85,9 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN;
-    const int m0 = blockIdx.y * BM;
+    const int tiles_m = (M + BM - 1) / BM;
+    const int tiles_n = (N + BN - 1) / BN;
+    const int num_tiles = tiles_m * tiles_n;
     const int num_kb = (K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
@@ -78,7 +95,10 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             mbar_init(smem_u32(&bars->full[s]), 1);
             mbar_init(smem_u32(&bars->empty[s]), 1);
         }
-        mbar_init(smem_u32(&bars->accum), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&bars->tfull[b]), 1);
+            mbar_init(smem_u32(&bars->tempty[b]), EPI_WARPS);
+        }
         bars->abort = 0;
         fence_barrier_init();
         fence_proxy_async_shared();
@@ -98,67 +118,91 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
     if (warp == 0) {
         if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t round = (uint32_t)(kb / STAGES);
-                if (!mbar_wait(smem_u32(&bars->empty[s]), (round & 1u) ^ 1u, abort)) {
-                    fail(err, abort, bi::DEVERR_WAIT_TMA);
-                    break;
-                }
-                const uint32_t fb = smem_u32(&bars->full[s]);
-                mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                tma_load_2d(smem_u32(sA + s * A_STAGE), &tmA, kb * BK, m0, fb);
+            uint32_t it = 0;  // k-blocks issued by this CTA so far (the ring runs across tiles)
+            for (int t = blockIdx.x; t < num_tiles && !*abort; t += gridDim.x) {
+                int mt, nt;
+                tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
+                const int m0 = mt * BM, n0 = nt * BN;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t round = it / STAGES;
+                    if (!mbar_wait(smem_u32(&bars->empty[s]), (round & 1u) ^ 1u, abort)) {
+                        fail(err, abort, bi::DEVERR_WAIT_TMA);
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&bars->full[s]);
+                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+                    tma_load_2d(smem_u32(sA + s * A_STAGE), &tmA, kb * BK, m0, fb);
 #pragma unroll
-                for (int j = 0; j < BN / 64; ++j)
-                    tma_load_2d(smem_u32(sB + s * B_STAGE + j * B_BOX), &tmW, n0 + 64 * j, kb * BK, fb);
-                ++issued;
+                    for (int j = 0; j < BN / 64; ++j)
+                        tma_load_2d(smem_u32(sB + s * B_STAGE + j * B_BOX), &tmW, n0 + 64 * j, kb * BK, fb);
+                }
             }
             if (*abort) {  // let loads already in flight land before the CTA's shared memory is released
-                for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
-                    (void)mbar_wait(smem_u32(&bars->full[kb % STAGES]), (uint32_t)(kb / STAGES) & 1u, nullptr);
+                for (uint32_t i = it > (uint32_t)STAGES ? it - STAGES : 0u; i < it; ++i)
+                    (void)mbar_wait(smem_u32(&bars->full[i % STAGES]), (i / STAGES) & 1u, nullptr);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc_bf16_f32(BM, BN, 0, 1);
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t round = (uint32_t)(kb / STAGES);
-                if (!mbar_wait(smem_u32(&bars->full[s]), round & 1u, abort)) {
-                    fail(err, abort, bi::DEVERR_WAIT_FULL);
+            uint32_t it = 0, local = 0;
+            for (int t = blockIdx.x; t < num_tiles && !*abort; t += gridDim.x, ++local) {
+                const uint32_t acc = local & 1u, use = local >> 1;
+                if (!mbar_wait(smem_u32(&bars->tempty[acc]), (use & 1u) ^ 1u, abort)) {
+                    fail(err, abort, bi::DEVERR_WAIT_ACCUM);
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(sA + s * A_STAGE);
-                const uint32_t b_base = smem_u32(sB + s * B_STAGE);
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t round = it / STAGES;
+                    if (!mbar_wait(smem_u32(&bars->full[s]), round & 1u, abort)) {
+                        fail(err, abort, bi::DEVERR_WAIT_FULL);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA + s * A_STAGE);
+                    const uint32_t b_base = smem_u32(sB + s * B_STAGE);
 #pragma unroll
-                for (int k = 0; k < BK / UMMA_K; ++k) {
-                    // A: K-major, 128B swizzle; the k-th 16-element slice starts 32 bytes further along the row.
-                    const uint64_t adesc = make_smem_desc(a_base + k * UMMA_K * 2, 16, 1024, 2);
-                    // W: N-major, 128B swizzle; 16 K-rows of 128 bytes each per step.
-                    const uint64_t bdesc = make_smem_desc(b_base + k * UMMA_K * 128, B_BOX, 1024, 2);
-                    mma_bf16_ss(tmem_base, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        // A: K-major, 128B swizzle; the k-th 16-element slice starts 32 bytes along the row.
+                        const uint64_t adesc = make_smem_desc(a_base + k * UMMA_K * 2, 16, 1024, 2);
+                        // W: N-major, 128B swizzle; 16 K-rows of 128 bytes each per step.
+                        const uint64_t bdesc = make_smem_desc(b_base + k * UMMA_K * 128, B_BOX, 1024, 2);
+                        mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(smem_u32(&bars->empty[s]));  // stage free once these MMAs have read it
                 }
-                mma_commit(smem_u32(&bars->empty[s]));  // stage free once these MMAs have read it
+                mma_commit(smem_u32(&bars->tfull[acc]));  // accumulator complete
             }
-            mma_commit(smem_u32(&bars->accum));  // accumulator complete
         }
     } else {
         const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter .. +31
-        const bool ok = mbar_wait(smem_u32(&bars->accum), 0u, abort);
-        if (!ok) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
-        // tcgen05.ld is warp-collective: the whole warp takes the same branch
-        if (__all_sync(0xffffffffu, ok && !*abort)) {
+        uint32_t local = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+            const uint32_t acc = local & 1u, use = local >> 1;
+            const bool ok = mbar_wait(smem_u32(&bars->tfull[acc]), use & 1u, abort);
+            if (!ok) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+            // tcgen05.ld is warp-collective: the whole warp takes the same branch
+            if (!__all_sync(0xffffffffu, ok && !*abort)) break;
             tc_fence_after();
-            const int row = m0 + quarter * 32 + lane;
-            const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+            int mt, nt;
+            tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
+            const int row = mt * BM + quarter * 32 + lane;
+            const uint32_t lane_addr = tmem_base + acc * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(lane_addr + (uint32_t)c, r);
                 tmem_wait_ld();
-                const int col = n0 + c;
+                if (c == BN - 32) {  // every column of this accumulator is in registers: hand it back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&bars->tempty[acc]));
+                }
+                const int col = nt * BN + c;
                 if (row < M && col < N) {
                     if (!c_bf16) {
                         float* dst = static_cast<float*>(C) + (int64_t)row * N + col;
@@ -201,6 +245,18 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 }
 
 // ------------------------------------------------------------------ host side
+int num_sms() {
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 bool ensure_smem_attr() {
     static std::once_flag once[64];
     static bool ok[64];
@@ -229,7 +285,8 @@ BI_API int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, 
     if (!A || !W || !C) return BI_ERR_INVALID_ARG;
     if (!bi::aligned16(A) || !bi::aligned16(W) || !bi::aligned16(C)) return BI_ERR_MISALIGNED;
     if (K % 8 != 0 || N % 8 != 0) return BI_ERR_MISALIGNED;  // 16-byte row strides for the TMA unit
-    if (M > (int64_t)65535 * BM || N > (int64_t)65535 * BN || K > (1LL << 30)) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (((M + BM - 1) / BM) * ((N + BN - 1) / BN) > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
     uint32_t* err = bi::device_error_word();
     if (!err || !ensure_smem_attr()) return BI_ERR_CUDA;
     CUtensorMap tmA, tmW;
@@ -239,8 +296,12 @@ BI_API int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, 
     if (!bi::make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)N, (uint64_t)K, (uint64_t)N * 2, 64,
                           BK, CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
-    dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int sms = num_sms();
+    if (sms <= 0) return BI_ERR_CUDA;
+    const int gm = K >= 8192 ? 8 : 16;
+    dim3 grid((unsigned)(tiles < sms ? tiles : sms));
     bi_gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, bi::as_stream(stream)>>>(
-        tmA, tmW, C, (int)M, (int)N, (int)K, c_dtype == BI_BF16 ? 1 : 0, err);
+        tmA, tmW, C, (int)M, (int)N, (int)K, c_dtype == BI_BF16 ? 1 : 0, gm, err);
     return bi::launch_status();
 }
