@@ -36,228 +36,352 @@ namespace {
 
 constexpr int D = 128;
 constexpr int CHUNK = 256;
-constexpr int THREADS = 256;   // 8 warps
-constexpr int BOX_TOK = 64;    // tokens per TMA box
+constexpr int CWARPS = 8;                    // compute warps
+constexpr int CTHREADS = CWARPS * 32;        // 256
+constexpr int THREADS = CTHREADS + 32;       // + one producer warp
+constexpr int SUB = 128;                     // tokens per pipeline stage
+constexpr int BOX_TOK = 64;                  // tokens per TMA box
 constexpr int BOX_BYTES = BOX_TOK * 64 * 2;  // 64 tokens x 64 dims (one 128-byte half row) = 8 KB
-constexpr int KV_BYTES = CHUNK * D * 2;      // 64 KB
+constexpr int STAGE_BYTES = SUB * D * 2;     // 32 KB
+constexpr int NSTAGES = 3;
 
 constexpr uint32_t DEVERR_BAD_LAYOUT = 1u << 8;  // kv_indptr / kv_len violate the documented layout
 
+constexpr int P_PITCH = CHUNK + 8;  // bf16 per head row of the split probabilities (+8: no bank conflicts)
+
 template <int G>
 struct AttnLayout {
-    static constexpr int S_OFF = KV_BYTES;                      // scores / probabilities [CHUNK][G] fp32
-    static constexpr int RED_OFF = S_OFF + CHUNK * G * 4;       // [8 warps][G][D] fp32
-    static constexpr int STAT_OFF = RED_OFF + 8 * G * D * 4;    // per-warp partial max / sum [8][G] x 2
-    static constexpr int BAR_OFF = STAT_OFF + 2 * 8 * G * 4;
-    static constexpr size_t BYTES = 1024 + BAR_OFF + 64;
+    static constexpr int S_OFF = NSTAGES * STAGE_BYTES;         // scores [CHUNK][G] fp32
+    static constexpr int P_OFF = S_OFF + CHUNK * G * 4;         // p_hi, p_lo: bf16 [8 heads][P_PITCH] each
+    static constexpr int P_BYTES = 8 * P_PITCH * 2;
+    static constexpr int STAT_OFF = P_OFF + 2 * P_BYTES;        // per-warp partial max / sum [8][G] x 2
+    static constexpr int Q_OFF = STAT_OFF + 2 * CWARPS * G * 4;       // per stage: the item's queries, bf16 [G][D]
+    static constexpr int Q_BYTES = G * D * 2;
+    static constexpr int BAR_OFF = Q_OFF + NSTAGES * Q_BYTES;
+    static constexpr size_t BYTES = 1024 + BAR_OFF + 2 * NSTAGES * 8 + 16;
 };
 
-// smem address of (token j, dim pair starting at d) in the swizzled K/V buffer
-__device__ __forceinline__ uint32_t kv_addr(uint32_t base, int j, int d) {
+// smem address of (token j of a stage, dim d) in a 128B-swizzled stage
+__device__ __forceinline__ uint32_t kv_addr(uint32_t stage, int j, int d) {
     const uint32_t box = (uint32_t)((j >> 6) * 2 + (d >> 6));
-    return swz(base + box * BOX_BYTES + (uint32_t)(j & 63) * 128 + (uint32_t)(d & 63) * 2, 7u);
+    return swz(stage + box * BOX_BYTES + (uint32_t)(j & 63) * 128 + (uint32_t)(d & 63) * 2, 7u);
 }
 
+__device__ __forceinline__ void compute_barrier() { asm volatile("bar.sync 1, %0;" :: "n"(CTHREADS) : "memory"); }
+
+struct Item {
+    int b;       // sequence
+    int c;       // chunk of that sequence
+    int n_tok;   // live tokens in the chunk (0: nothing to do)
+    int64_t tok0;
+};
+
+// Remembers the sequence found for the previous slot; slots of one CTA increase, so the
+// next slot usually belongs to the same sequence and needs no memory access at all.
+struct SeqCache {
+    int b = -1;
+    int64_t lo_tok = 0, hi_tok = 0;  // the sequence's tokens [lo_tok, hi_tok) of the packed buffer
+    int len = 0;
+};
+
+// The (sequence, chunk) that owns 256-token slot `slot` of the packed cache.
+__device__ __forceinline__ Item item_of(int slot, const int32_t* __restrict__ kv_indptr,
+                                        const int32_t* __restrict__ kv_len, int B, bool& bad, SeqCache& sc) {
+    Item it{0, 0, 0, (int64_t)slot * CHUNK};
+    bad = false;
+    int lo;
+    if (sc.b >= 0 && it.tok0 >= sc.lo_tok && it.tok0 < sc.hi_tok) {
+        lo = sc.b;
+    } else {
+        if (it.tok0 < kv_indptr[0] || it.tok0 >= kv_indptr[B]) return it;
+        lo = 0;
+        int hi = B;  // the last b with kv_indptr[b] <= tok0
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (kv_indptr[mid] <= it.tok0) lo = mid; else hi = mid;
+        }
+        sc.b = lo;
+        sc.lo_tok = kv_indptr[lo];
+        sc.hi_tok = kv_indptr[lo + 1];
+        sc.len = kv_len[lo];
+    }
+    const int64_t sbase = sc.lo_tok;
+    const int len = sc.len;
+    const int64_t cap = sc.hi_tok - sbase;
+    if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap) {
+        bad = (it.tok0 - sbase) < CHUNK;  // report once per sequence
+        return it;
+    }
+    it.b = lo;
+    it.c = (int)((it.tok0 - sbase) / CHUNK);
+    it.n_tok = max(0, min(CHUNK, len - it.c * CHUNK));
+    return it;
+}
+
+// Phase 1, persistent: CTA i handles a contiguous range of work items; item w = (slot w / Hkv,
+// kv head w % Hkv), so consecutive items share a slot and usually a sequence.
+// A producer warp streams each item's K sub-blocks, then its V sub-blocks, through an NSTAGES ring;
+// eight compute warps consume them in the same order.
 template <int G>
 __global__ void __launch_bounds__(THREADS, 2)
 decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ kv_indptr,
-                         const int32_t* __restrict__ kv_len, int B, int Hq, int Hkv, float scale,
+                         const int32_t* __restrict__ kv_len, int B, int Hq, int Hkv, int n_items, float scale,
                          float* __restrict__ o_part, float* __restrict__ ml_part, uint32_t* err) {
     using L = AttnLayout<G>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* sS = reinterpret_cast<float*>(base + L::S_OFF);
-    float* sRed = reinterpret_cast<float*>(base + L::RED_OFF);
+    __nv_bfloat16* sPh = reinterpret_cast<__nv_bfloat16*>(base + L::P_OFF);
+    __nv_bfloat16* sPl = reinterpret_cast<__nv_bfloat16*>(base + L::P_OFF + L::P_BYTES);
     float* sMax = reinterpret_cast<float*>(base + L::STAT_OFF);
-    float* sSum = sMax + 8 * G;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(base + L::BAR_OFF);
+    float* sSum = sMax + CWARPS * G;
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::BAR_OFF);
+    uint64_t* empty = full + NSTAGES;
+    volatile int* abort = reinterpret_cast<volatile int*>(empty + NSTAGES);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int slot = blockIdx.x;
-    const int g = blockIdx.y;
-    const int64_t tok0 = (int64_t)slot * CHUNK;
+    const uint32_t stage0 = smem_u32(base);
+    const int per_cta = (n_items + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int w_begin = (int)blockIdx.x * per_cta;
+    const int w_end = min(n_items, w_begin + per_cta);
 
-    // Which sequence owns this slot: the last b with kv_indptr[b] <= tok0 (binary search).
-    int lo = 0, hi = B;  // invariant: kv_indptr[lo] <= tok0 < kv_indptr[hi] when tok0 < kv_indptr[B]
-    if (tok0 < kv_indptr[0] || tok0 >= kv_indptr[B]) return;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (kv_indptr[mid] <= tok0) lo = mid; else hi = mid;
-    }
-    const int b = lo;
-    const int64_t sbase = kv_indptr[b];
-    const int len = kv_len[b];
-    const int64_t cap = (int64_t)kv_indptr[b + 1] - sbase;
-    if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap) {
-        if (tid == 0 && g == 0 && tok0 - sbase < CHUNK) atomicOr(err, DEVERR_BAD_LAYOUT);
-        return;
-    }
-    const int c = (int)((tok0 - sbase) / CHUNK);
-    const int n_tok = min(CHUNK, len - c * CHUNK);
-    if (n_tok <= 0) return;  // capacity padding beyond the sequence
-    const int n_box_tok = (n_tok + BOX_TOK - 1) / BOX_TOK;  // 64-token groups holding live tokens
-
-    const uint32_t kv_base = smem_u32(base);
-    const uint32_t bar_a = smem_u32(bar);
     if (tid == 0) {
-        mbar_init(bar_a, 1);
+        for (int i = 0; i < NSTAGES; ++i) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), CWARPS);
+        }
+        *abort = 0;
         fence_barrier_init();
         fence_proxy_async_shared();
     }
     __syncthreads();
-    if (tid == 0) {
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
-        mbar_arrive_expect_tx(bar_a, (uint32_t)(n_box_tok * 2 * BOX_BYTES));
-        for (int tg = 0; tg < n_box_tok; ++tg)
-            for (int hf = 0; hf < 2; ++hf)
-                tma_load_2d(kv_base + (tg * 2 + hf) * BOX_BYTES, &tmK, g * D + hf * 64, (int)(tok0 + tg * BOX_TOK),
-                            bar_a);
-    }
 
-    // Query fragments (B operand, [16 dims x 8 heads] per k-step; heads >= G are zero).
-    uint32_t qf[8][2];
-    {
-        const int hh = lane >> 2, dq = (lane & 3) * 2;
-        const __nv_bfloat16* qh = q + ((int64_t)b * Hq + (int64_t)g * G + (hh < G ? hh : 0)) * D;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            uint32_t v0 = 0u, v1 = 0u;
-            if (hh < G) {
-                v0 = *reinterpret_cast<const uint32_t*>(qh + kk * 16 + dq);
-                v1 = *reinterpret_cast<const uint32_t*>(qh + kk * 16 + dq + 8);
+    if (warp == CWARPS) {
+        // ------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            uint32_t it = 0;
+            SeqCache sc;
+            for (int w = w_begin; w < w_end && !*abort; ++w) {
+                const int slot = w / Hkv, g = w % Hkv;
+                bool bad;
+                const Item itm = item_of(slot, kv_indptr, kv_len, B, bad, sc);
+                if (bad && g == 0) atomicOr(err, DEVERR_BAD_LAYOUT);
+                if (itm.n_tok == 0) continue;
+                const int nsub = (itm.n_tok + SUB - 1) / SUB;
+                for (int pass = 0; pass < 2 && !*abort; ++pass) {
+                    const CUtensorMap* tm = pass == 0 ? &tmK : &tmV;
+                    for (int sb = 0; sb < nsub; ++sb, ++it) {
+                        const int st = it % NSTAGES;
+                        if (!mbar_wait(smem_u32(&empty[st]), ((it / NSTAGES) & 1u) ^ 1u, abort)) {
+                            atomicOr(err, bi::DEVERR_WAIT_TMA);
+                            *abort = 1;
+                            break;
+                        }
+                        const int live = min(SUB, itm.n_tok - sb * SUB);
+                        const int ngrp = (live + BOX_TOK - 1) / BOX_TOK;
+                        const uint32_t fb = smem_u32(&full[st]);
+                        const bool with_q = pass == 0 && sb == 0;  // the item's queries ride on its first stage
+                        mbar_arrive_expect_tx(fb, (uint32_t)(ngrp * 2 * BOX_BYTES + (with_q ? L::Q_BYTES : 0)));
+                        if (with_q)
+                            bulk_load(smem_u32(base + L::Q_OFF + st * L::Q_BYTES),
+                                      q + ((int64_t)itm.b * Hq + (int64_t)g * G) * D, L::Q_BYTES, fb);
+                        const uint32_t dst = stage0 + st * STAGE_BYTES;
+                        for (int tg = 0; tg < ngrp; ++tg)
+                            for (int hf = 0; hf < 2; ++hf)
+                                tma_load_2d(dst + (tg * 2 + hf) * BOX_BYTES, tm, g * D + hf * 64,
+                                            (int)(itm.tok0 + sb * SUB + tg * BOX_TOK), fb);
+                    }
+                }
             }
-            qf[kk][0] = v0;
-            qf[kk][1] = v1;
-        }
-    }
-
-    const bool k_ok = __all_sync(0xffffffffu, mbar_wait(bar_a, 0u, nullptr));
-    if (!k_ok && lane == 0) atomicOr(err, bi::DEVERR_WAIT_FULL);
-
-    // ---- scores: warp w owns tokens [32w, 32w + 32) as two 16-row MMA tiles
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-        const int t0 = warp * 32 + mt * 16;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (k_ok && t0 < n_tok) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                uint32_t a[4];
-                ldmatrix_x4(kv_addr(kv_base, t0 + (lane & 15), kk * 16 + (lane >> 4) * 8), a);
-                mma_m16n8k16_bf16(acc, a, qf[kk]);
+            if (*abort) {
+                for (uint32_t i = it > (uint32_t)NSTAGES ? it - NSTAGES : 0u; i < it; ++i)
+                    (void)mbar_wait(smem_u32(&full[i % NSTAGES]), (i / NSTAGES) & 1u, nullptr);
             }
         }
-        const int gg = lane >> 2, hq = (lane & 3) * 2;
+        return;
+    }
+
+    // ---------------------------------------------------- compute warps
+    uint32_t it = 0;
+    SeqCache sc;
+    for (int w = w_begin; w < w_end; ++w) {
+        const int slot = w / Hkv, g = w % Hkv;
+        bool bad;
+        const Item itm = item_of(slot, kv_indptr, kv_len, B, bad, sc);
+        if (itm.n_tok == 0) continue;
+        const int n_tok = itm.n_tok;
+        const int nsub = (n_tok + SUB - 1) / SUB;
+
+        // ---- scores: in stage sb, warp w owns the 16 tokens [16 w, 16 w + 16)
+        bool ok = true;
+        uint32_t qf[8][2];
+        for (int sb = 0; sb < 2; ++sb) {
+            const int t0 = sb * SUB + warp * 16;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (sb < nsub) {
+                const int st = it % NSTAGES;
+                const bool w_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), (it / NSTAGES) & 1u, abort));
+                if (!w_ok) {
+                    ok = false;
+                    if (lane == 0) {
+                        atomicOr(err, bi::DEVERR_WAIT_FULL);
+                        *abort = 1;
+                    }
+                }
+                if (sb == 0) {
+                    // query fragments from the first stage's query slot (B operand, [16 dims x 8 heads]
+                    // per k-step; heads >= G are zero)
+                    const int hh = lane >> 2, dq = (lane & 3) * 2;
+                    const uint32_t qs = smem_u32(base + L::Q_OFF + st * L::Q_BYTES) + (uint32_t)(hh < G ? hh : 0) * D * 2;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int j = t0 + gg + (e >> 1) * 8;
-            const int h = hq + (e & 1);
-            if (h < G) sS[j * G + h] = (j < n_tok) ? __fmul_rn(acc[e], scale) : -INFINITY;
+                    for (int kk = 0; kk < 8; ++kk) {
+                        uint32_t v0 = 0u, v1 = 0u;
+                        if (hh < G && w_ok) {
+                            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v0) : "r"(qs + (kk * 16 + dq) * 2));
+                            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v1) : "r"(qs + (kk * 16 + dq + 8) * 2));
+                        }
+                        qf[kk][0] = v0;
+                        qf[kk][1] = v1;
+                    }
+                }
+                if (w_ok && t0 < n_tok) {
+                    const uint32_t sbase = stage0 + st * STAGE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        uint32_t a[4];
+                        ldmatrix_x4(kv_addr(sbase, warp * 16 + (lane & 15), kk * 16 + (lane >> 4) * 8), a);
+                        mma_m16n8k16_bf16(acc, a, qf[kk]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+                ++it;
+            }
+            const int gg = lane >> 2, hq = (lane & 3) * 2;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = t0 + gg + (e >> 1) * 8;
+                const int h = hq + (e & 1);
+                if (h < G) sS[j * G + h] = (j < n_tok) ? __fmul_rn(acc[e], scale) : -INFINITY;
+            }
         }
-    }
-    __syncthreads();  // K no longer needed; scores complete
+        // A failed wait never changes the control flow: every compute warp keeps meeting the same
+        // named barriers, the abort flag makes the remaining waits return at once, and the
+        // kernel runs to its end with the error recorded.
+        (void)ok;
+        compute_barrier();
 
-    if (tid == 0) {  // V into the same buffer (its previous contents are dead: every ldmatrix has completed)
-        fence_proxy_async_shared();
-        mbar_arrive_expect_tx(bar_a, (uint32_t)(n_box_tok * 2 * BOX_BYTES));
-        for (int tg = 0; tg < n_box_tok; ++tg)
-            for (int hf = 0; hf < 2; ++hf)
-                tma_load_2d(kv_base + (tg * 2 + hf) * BOX_BYTES, &tmV, g * D + hf * 64, (int)(tok0 + tg * BOX_TOK),
-                            bar_a);
-    }
-
-    // ---- softmax statistics over the chunk (thread tid owns token tid)
-    float s[G], p[G];
+        // ---- softmax statistics over the chunk (thread tid owns token tid)
+        float sv[G], p[G], mc[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) s[h] = sS[tid * G + h];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        float m = s[h];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (lane == 0) sMax[warp * G + h] = m;
-    }
-    __syncthreads();
-    float mc[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        float m = sMax[h];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) m = fmaxf(m, sMax[w * G + h]);
-        mc[h] = m;
-        p[h] = (tid < n_tok) ? expf(__fsub_rn(s[h], m)) : 0.0f;
-        sS[tid * G + h] = p[h];
-        float sum = p[h];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
-        if (lane == 0) sSum[warp * G + h] = sum;
-    }
-    __syncthreads();
-
-    // ---- o_c = sum_j p_j v_j: thread owns dims [8*dg, 8*dg + 8) and tokens j = tg + 16 i
-    const bool v_ok = __all_sync(0xffffffffu, mbar_wait(bar_a, 1u, nullptr));
-    if (!v_ok && lane == 0) atomicOr(err, bi::DEVERR_WAIT_FULL);
-    const int dg = tid & 15, tg = tid >> 4;
-    float acc[G][8];
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[h][e] = 0.0f;
-    if (v_ok) {
-#pragma unroll 4
-        for (int i = 0; i < CHUNK / 16; ++i) {
-            const int j = tg + 16 * i;
-            if (j >= n_tok) break;
-            uint4 u;
-            const uint32_t a = kv_addr(kv_base, j, dg * 8);
-            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(a));
-            const float vf[8] = {bi::bf16_lo(u.x), bi::bf16_hi(u.x), bi::bf16_lo(u.y), bi::bf16_hi(u.y),
-                                 bi::bf16_lo(u.z), bi::bf16_hi(u.z), bi::bf16_lo(u.w), bi::bf16_hi(u.w)};
-            float pj[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) pj[h] = sS[j * G + h];
-#pragma unroll
-            for (int h = 0; h < G; ++h)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[h][e] = __fmaf_rn(pj[h], vf[e], acc[h][e]);
-        }
-    }
-    // pair the two token groups of this warp (lanes l and l ^ 16 share dg), then warps in order
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[h][e] = __fadd_rn(acc[h][e], __shfl_xor_sync(0xffffffffu, acc[h][e], 16));
-    if (lane < 16) {
+        for (int h = 0; h < G; ++h) sv[h] = sS[tid * G + h];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            float4* dst = reinterpret_cast<float4*>(sRed + (warp * G + h) * D + dg * 8);
-            dst[0] = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-            dst[1] = make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
+            float m = sv[h];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            if (lane == 0) sMax[warp * G + h] = m;
         }
-    }
-    __syncthreads();
+        compute_barrier();
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            if (h < G) {
+                float m = sMax[h];
+#pragma unroll
+                for (int ww = 1; ww < CWARPS; ++ww) m = fmaxf(m, sMax[ww * G + h]);
+                mc[h] = m;
+                p[h] = (tid < n_tok) ? expf(__fsub_rn(sv[h], m)) : 0.0f;
+                // p = hi + lo + r with hi, lo bf16 and |r| <= 2^-18 |p|: the tensor-core PV below
+                // multiplies the exact bf16 values of V by hi and by lo and adds both in fp32
+                const __nv_bfloat16 hi = __float2bfloat16_rn(p[h]);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(p[h], __bfloat162float(hi)));
+                sPh[h * P_PITCH + tid] = hi;
+                sPl[h * P_PITCH + tid] = lo;
+                float sum = p[h];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, off));
+                if (lane == 0) sSum[warp * G + h] = sum;
+            } else {  // heads past the group: zero columns of the MMA's B operand
+                sPh[h * P_PITCH + tid] = __float2bfloat16_rn(0.0f);
+                sPl[h * P_PITCH + tid] = __float2bfloat16_rn(0.0f);
+            }
+        }
+        compute_barrier();
 
-    const int hq0 = g * G;
-    for (int o = tid; o < G * D; o += THREADS) {
-        const int h = o / D, d = o % D;
-        float v = sRed[h * D + d];
+        // ---- o_c = sum_j p_j v_j on tensor cores: warp w owns dims [16 w, 16 w + 16) for all 8
+        // (padded) heads: O^T[dims x heads] += V^T[dims x 16 tokens] . P[16 tokens x heads], tokens in
+        // ascending 16-token steps, the hi then the lo part of P at each step.
+        // two independent chains (the hi and the lo part of P), added once at the end
+        float oacc[4] = {0.f, 0.f, 0.f, 0.f}, oacc_lo[4] = {0.f, 0.f, 0.f, 0.f};
+        const int gq = lane >> 2, cq = lane & 3;
+        const uint32_t ph = smem_u32(sPh) + (uint32_t)(gq * P_PITCH + 2 * cq) * 2;
+        const uint32_t pl = smem_u32(sPl) + (uint32_t)(gq * P_PITCH + 2 * cq) * 2;
+        for (int sb = 0; sb < nsub; ++sb) {
+            const int st = it % NSTAGES;
+            const bool w_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), (it / NSTAGES) & 1u, abort));
+            if (!w_ok && lane == 0) {
+                atomicOr(err, bi::DEVERR_WAIT_FULL);
+                *abort = 1;
+            }
+            if (w_ok) {
+                const uint32_t sbase = stage0 + st * STAGE_BYTES;
+                const int live = min(SUB, n_tok - sb * SUB);
+                for (int ks = 0; ks * 16 < live; ++ks) {
+                    uint32_t a[4];
+                    // matrix i = lane / 8: tokens +8 * (i >> 1), dims +8 * (i & 1)
+                    const int mi = lane >> 3;
+                    ldmatrix_x4_trans(kv_addr(sbase, ks * 16 + (lane & 7) + 8 * (mi >> 1), warp * 16 + 8 * (mi & 1)), a);
+                    if (ks * 16 + 16 > live) {  // last, partial step: tokens past the end may hold anything
+                        const int t_lo = ks * 16 + 2 * cq;  // tokens of a0/a1 (and +8 for a2/a3)
 #pragma unroll
-        for (int w = 1; w < 8; ++w) v = __fadd_rn(v, sRed[(w * G + h) * D + d]);
-        o_part[((int64_t)slot * Hq + hq0 + h) * D + d] = v;
-    }
-    if (tid < G) {
-        float l = sSum[tid];
+                        for (int r = 0; r < 4; ++r) {
+                            const int t = t_lo + (r >> 1) * 8;
+                            uint32_t m = 0u;
+                            if (t < live) m |= 0x0000FFFFu;
+                            if (t + 1 < live) m |= 0xFFFF0000u;
+                            a[r] &= m;
+                        }
+                    }
+                    const int j0 = sb * SUB + ks * 16;  // token of the chunk at the start of this step
+                    uint32_t bh[2], bl[2];
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bh[0]) : "r"(ph + j0 * 2));
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bh[1]) : "r"(ph + (j0 + 8) * 2));
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bl[0]) : "r"(pl + j0 * 2));
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bl[1]) : "r"(pl + (j0 + 8) * 2));
+                    mma_m16n8k16_bf16(oacc, a, bh);
+                    mma_m16n8k16_bf16(oacc_lo, a, bl);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+            ++it;
+        }
+
+        // oacc: (dim 16w + gq, heads 2cq, 2cq+1) and (dim 16w + gq + 8, same heads)
+        const int hq0 = g * G;
 #pragma unroll
-        for (int w = 1; w < 8; ++w) l = __fadd_rn(l, sSum[w * G + tid]);
-        float2* ml = reinterpret_cast<float2*>(ml_part + ((int64_t)slot * Hq + hq0 + tid) * 2);
-        // mc[] is uniform across threads; select this head's value without dynamic register indexing
-        float m_sel = mc[0];
+        for (int e = 0; e < 4; ++e) oacc[e] = __fadd_rn(oacc[e], oacc_lo[e]);
 #pragma unroll
-        for (int h = 1; h < G; ++h)
-            if (tid == h) m_sel = mc[h];
-        *ml = make_float2(m_sel, l);
+        for (int e = 0; e < 4; ++e) {
+            const int h = 2 * cq + (e & 1);
+            const int d = warp * 16 + gq + (e >> 1) * 8;
+            if (h < G) o_part[((int64_t)slot * Hq + hq0 + h) * D + d] = oacc[e];
+        }
+        if (tid < G) {
+            float l = sSum[tid];
+#pragma unroll
+            for (int ww = 1; ww < CWARPS; ++ww) l = __fadd_rn(l, sSum[ww * G + tid]);
+            // mc[] is uniform across threads; select this head's value without dynamic register indexing
+            float m_sel = mc[0];
+#pragma unroll
+            for (int h = 1; h < G; ++h)
+                if (tid == h) m_sel = mc[h];
+            *reinterpret_cast<float2*>(ml_part + ((int64_t)slot * Hq + hq0 + tid) * 2) = make_float2(m_sel, l);
+        }
+        compute_barrier();  // scores, probabilities and statistics are reused by the next item
     }
 }
 
@@ -327,6 +451,18 @@ bool set_smem_once(F kernel, size_t bytes) {
     return true;
 }
 
+int num_sms() {
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 size_t partial_bytes(int64_t total_tokens, int32_t Hq) {
     const int64_t slots = (total_tokens + CHUNK - 1) / CHUNK;
     return (size_t)slots * Hq * (D + 2) * sizeof(float);
@@ -346,9 +482,14 @@ int launch_chunks(const void* q, const void* k, const void* v, const int32_t* kv
         !bi::make_tmap_2d(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, row, (uint64_t)T, row * 2, 64, BOX_TOK,
                           CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
-    dim3 grid((unsigned)((T + CHUNK - 1) / CHUNK), (unsigned)Hkv);
+    const int64_t items = ((T + CHUNK - 1) / CHUNK) * Hkv;
+    if (items > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
+    const int sms = num_sms();
+    if (sms <= 0) return BI_ERR_CUDA;
+    const int64_t ctas = 2LL * sms;  // two persistent CTAs per SM: one computes while the other waits
+    dim3 grid((unsigned)(items < ctas ? items : ctas));
     kern<<<grid, THREADS, L::BYTES, s>>>(tmK, tmV, static_cast<const __nv_bfloat16*>(q), kv_indptr, kv_len, B, Hq,
-                                         Hkv, scale, o_part, ml_part, err);
+                                         Hkv, (int)items, scale, o_part, ml_part, err);
     return bi::launch_status();
 }
 
