@@ -154,7 +154,7 @@ def _to_dev(a, device):
     return torch.from_numpy(a).to(device)
 
 
-def build_ops(device, stream):
+def build_ops(device, stream, attn_batch=None):
     """Allocate the synthetic workload on the device and return the list of ops of one step.
 
     Each op: dict(name, kind 'hbm'|'tensor', work (bytes or flops per launch), launch(k), src, desc).
@@ -164,6 +164,7 @@ def build_ops(device, stream):
     import torch
     from invariant_deterministic_rmsnorm_b200 import binding as B
 
+    attn_batch = attn_batch or ATTN_BATCH
     ops = []
     M, H = M_TOKENS, HIDDEN
     x_np, w_np = inputs.rmsnorm_case(M, H, "bf16")
@@ -203,22 +204,22 @@ def build_ops(device, stream):
     down = gemm_op("gemm_down", lambda k: up, 14336, H, inputs.SEED_WEIGHTS + 12)
 
     # decode attention over a batch of requests with ragged cache lengths
-    kv_len = inputs.kv_lengths(ATTN_BATCH)
+    kv_len = inputs.kv_lengths(attn_batch)
     indptr, T = inputs.kv_layout(kv_len, 256)
     g = torch.Generator(device=device).manual_seed(inputs.SEED_X + 30)
     kc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
     vc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
-    q_np = inputs.normal_bf16(inputs.SEED_X + 31, (ATTN_BATCH, 32, 128))
+    q_np = inputs.normal_bf16(inputs.SEED_X + 31, (attn_batch, 32, 128))
     qa = _to_dev(q_np, device)
     ip_d = torch.tensor(indptr, dtype=torch.int32, device=device)
     ln_d = torch.tensor(kv_len, dtype=torch.int32, device=device)
     ws = torch.empty(B.bi_decode_attn_workspace_size(T, 32), dtype=torch.uint8, device=device)
-    attn_out = torch.empty((ATTN_BATCH, 32, 128), dtype=torch.bfloat16, device=device)
+    attn_out = torch.empty((attn_batch, 32, 128), dtype=torch.bfloat16, device=device)
     kv_bytes = int(kv_len.sum()) * 8 * 128 * 2 * 2
-    ops.append(dict(name="decode_attn", kind="hbm", work=kv_bytes + ATTN_BATCH * 32 * 128 * 4, src="bi_decode_attn.cu",
+    ops.append(dict(name="decode_attn", kind="hbm", work=kv_bytes + attn_batch * 32 * 128 * 4, src="bi_decode_attn.cu",
                     launch=lambda k: B.bi_decode_attn(qa, kc, vc, ip_d, ln_d, out=attn_out, workspace=ws,
                                                       stream=stream),
-                    desc=f"B={ATTN_BATCH} requests, kv lengths U[512,32768] (sum {int(kv_len.sum())}), 32 q / 8 kv "
+                    desc=f"B={attn_batch} requests, kv lengths U[512,32768] (sum {int(kv_len.sum())}), 32 q / 8 kv "
                          f"heads, D=128, 256-token chunks", launches=2))
     io = dict(h2d=[(xs[0], x_np), (qa, q_np)], d2h=[down, attn_out])
     return ops, io
@@ -248,7 +249,7 @@ def run_ours(args, rank, world, local_rank):
     B.library()
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
-        ops, io = build_ops(device, stream)
+        ops, io = build_ops(device, stream, args.attn_batch)
     torch.cuda.synchronize()
 
     def step(k, evs=None):
@@ -383,7 +384,7 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) activations, "
         "N(0,0.02) weights; no trained weights)",
         "config": {"workload": f"Llama-3-8B-shaped dense ops at M={M_TOKENS} tokens, hidden {HIDDEN}; LoRA r="
-                               f"{LORA_RANK} split-K 8 on q; GQA decode attention over {ATTN_BATCH} requests",
+                               f"{LORA_RANK} split-K 8 on q; GQA decode attention over {args.attn_batch} requests",
                    "ops": [op["name"] for op in ops], "parallelism": f"replicas x{world} (no collective)",
                    "l2": "inputs larger than L2: the step's working set exceeds the 126 MB L2"},
         "ops": per_op, "roofline": roofline,
@@ -517,6 +518,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--attn-batch", type=int, default=ATTN_BATCH,
+                    help="decode requests in the step (smaller for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -299,7 +299,7 @@ BI_API int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, 
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int sms = num_sms();
     if (sms <= 0) return BI_ERR_CUDA;
-    const int gm = K >= 8192 ? 8 : 16;
+    const int gm = 16;  // ~16 row tiles x ~9 column tiles in flight: A and W blocks balanced within L2
     dim3 grid((unsigned)(tiles < sms ? tiles : sms));
     bi_gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, bi::as_stream(stream)>>>(
         tmA, tmW, C, (int)M, (int)N, (int)K, c_dtype == BI_BF16 ? 1 : 0, gm, err);

@@ -33,19 +33,22 @@ using namespace bi::sm100;
 namespace {
 
 // ------------------------------------------------------------------ shrink
-constexpr int SH_TM = 64;           // rows per CTA (4 warps x 16)
+constexpr int SH_TM = 128;          // rows per CTA (8 warps x 16)
 constexpr int SH_KC = 64;           // K per pipeline stage
-constexpr int SH_STAGES = 6;
-constexpr int SH_CWARPS = 4;        // compute warps
+constexpr int SH_CWARPS = 8;        // compute warps
 constexpr int SH_THREADS = (SH_CWARPS + 1) * 32;
+constexpr int SH_MAX_STAGES = 6;
 
 template <int R>
 struct ShrinkLayout {
-    static constexpr int X_STAGE = SH_TM * SH_KC * 2;  // 8 KB, 128B-swizzled rows of 64 K
+    static constexpr int X_STAGE = SH_TM * SH_KC * 2;  // 16 KB, 128B-swizzled rows of 64 K
     static constexpr int A_STAGE = SH_KC * R * 2;      // 64 K-rows of R
     static constexpr int STAGE = X_STAGE + A_STAGE;    // multiple of 1024
-    static constexpr int PART = SH_TM * R * 4;
-    static constexpr size_t BYTES = 1024 + (size_t)SH_STAGES * STAGE + PART + 2 * SH_STAGES * 8 + 16;
+    // as many stages as leave room for two CTAs per SM (about 113 KB each)
+    static constexpr int STAGES = (110 * 1024) / STAGE < SH_MAX_STAGES ? (110 * 1024) / STAGE : SH_MAX_STAGES;
+    static constexpr int PART = SH_TM * R * 4;         // the partial reuses the stage memory
+    static_assert(PART <= STAGES * STAGE, "partial must fit in the stage memory");
+    static constexpr size_t BYTES = 1024 + (size_t)STAGES * STAGE + 2 * SH_MAX_STAGES * 8 + 16;
     // swizzle of the A stage: inner extent 2R bytes
     static constexpr uint32_t A_MASK = R == 64 ? 7u : (R == 32 ? 3u : (R == 16 ? 1u : 0u));
 };
@@ -56,9 +59,10 @@ lora_shrink_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                    float* __restrict__ t, int M, int KS, int split, uint32_t* err) {
     using L = ShrinkLayout<R>;
     extern __shared__ uint8_t smem_raw[];
+    constexpr int SH_STAGES = L::STAGES;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* part = reinterpret_cast<float*>(base + SH_STAGES * L::STAGE);
-    uint64_t* full = reinterpret_cast<uint64_t*>(part + SH_TM * R);
+    float* part = reinterpret_cast<float*>(base);  // written only after every stage has been consumed
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + SH_STAGES * L::STAGE);
     uint64_t* empty = full + SH_STAGES;
     volatile int* abort = reinterpret_cast<volatile int*>(empty + SH_STAGES);
 
@@ -139,6 +143,8 @@ lora_shrink_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
         }
+        // every warp is done reading the stages before any partial overwrites them
+        asm volatile("bar.sync 1, %0;" :: "n"(SH_CWARPS * 32) : "memory");
         const int g = lane >> 2, q = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < R / 8; ++nt) {
@@ -191,7 +197,7 @@ struct ExpandLayout {
     static constexpr int RP = R < 16 ? 16 : R;       // K of the MMA, padded with zeros
     static constexpr int T_PITCH = RP * 2 + 16;       // bytes per row of bf16(t); +16 avoids bank conflicts
     static constexpr int B_PITCH = EX_TN * 2 + 16;    // bytes per K-row of the B tile
-    static constexpr int D_PITCH = EX_TN + 4;         // floats per row of the staged product
+    static constexpr int D_PITCH = EX_TN + 8;         // floats per row of the staged product (conflict-free)
     static constexpr int T_BYTES = EX_TM * T_PITCH;
     static constexpr int B_BYTES = RP * B_PITCH;
     static constexpr size_t BYTES = (size_t)T_BYTES + B_BYTES + EX_TM * D_PITCH * 4;
@@ -212,6 +218,30 @@ lora_expand_kernel(const float* __restrict__ t, const __nv_bfloat16* __restrict_
     const int lane = tid & 31;
     const int m0 = blockIdx.y * EX_TM;
     const int n0 = blockIdx.x * EX_TN;
+
+    // 0. Issue this thread's loads of the y tile first: their HBM latency overlaps steps 1-3.
+    //    A chunk is 4 consecutive elements of a row (8 bytes of bf16 or 16 of fp32), so that the
+    //    matching 16 bytes of the staged product are read without bank conflicts.
+    constexpr int CPR = EX_TN / 4;                              // chunks per tile row
+    constexpr int NCH = EX_TM * CPR / EX_THREADS;               // chunks per thread (8)
+    uint4 yv[NCH];
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+        const int i = tid + k * EX_THREADS;
+        const int row = i / CPR, cc = i % CPR;
+        const int col = n0 + cc * 4;
+        yv[k] = make_uint4(0u, 0u, 0u, 0u);
+        if (m0 + row < M && col < N) {
+            if constexpr (YBF16) {
+                const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(y) +
+                                                                 (size_t)(m0 + row) * ldy + col);
+                yv[k].x = u.x;
+                yv[k].y = u.y;
+            } else {
+                yv[k] = *reinterpret_cast<const uint4*>(static_cast<const float*>(y) + (size_t)(m0 + row) * ldy + col);
+            }
+        }
+    }
 
     // 1. bf16(t) rows into shared memory (rows past M and columns past R are zero).
     for (int i = tid; i < EX_TM * L::RP / 4; i += EX_THREADS) {
@@ -258,35 +288,28 @@ lora_expand_kernel(const float* __restrict__ t, const __nv_bfloat16* __restrict_
     __syncthreads();
 
     // 4. y = round(fma(scale, delta, y)) with coalesced 128-bit accesses.
-    if constexpr (YBF16) {
-        for (int i = tid; i < EX_TM * (EX_TN / 8); i += EX_THREADS) {
-            const int row = i / (EX_TN / 8), cc = i % (EX_TN / 8);
-            const int col = n0 + cc * 8;
-            if (m0 + row >= M || col >= N) continue;
-            __nv_bfloat16* p = static_cast<__nv_bfloat16*>(y) + (size_t)(m0 + row) * ldy + col;
-            uint4 u = *reinterpret_cast<const uint4*>(p);
-            const float* d = sD + row * L::D_PITCH + cc * 8;
-            uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float lo = __fmaf_rn(scale, d[2 * j], bi::bf16_lo(w[j]));
-                const float hi = __fmaf_rn(scale, d[2 * j + 1], bi::bf16_hi(w[j]));
-                w[j] = bi::pack_bf16x2(lo, hi);
-            }
-            *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-    } else {
-        for (int i = tid; i < EX_TM * (EX_TN / 4); i += EX_THREADS) {
-            const int row = i / (EX_TN / 4), cc = i % (EX_TN / 4);
-            const int col = n0 + cc * 4;
-            if (m0 + row >= M || col >= N) continue;
+    for (int k = 0; k < NCH; ++k) {
+        const int i = tid + k * EX_THREADS;
+        const int row = i / CPR, cc = i % CPR;
+        const int col = n0 + cc * 4;
+        if (m0 + row >= M || col >= N) continue;
+        const float4 d = *reinterpret_cast<const float4*>(sD + row * L::D_PITCH + cc * 4);
+        if constexpr (YBF16) {
+            const float a0 = __fmaf_rn(scale, d.x, bi::bf16_lo(yv[k].x));
+            const float a1 = __fmaf_rn(scale, d.y, bi::bf16_hi(yv[k].x));
+            const float a2 = __fmaf_rn(scale, d.z, bi::bf16_lo(yv[k].y));
+            const float a3 = __fmaf_rn(scale, d.w, bi::bf16_hi(yv[k].y));
+            __nv_bfloat16* p = static_cast<__nv_bfloat16*>(y) + (size_t)(m0 + row) * ldy + col;
+            *reinterpret_cast<uint2*>(p) = make_uint2(bi::pack_bf16x2(a0, a1), bi::pack_bf16x2(a2, a3));
+        } else {
+            float4 v = make_float4(__uint_as_float(yv[k].x), __uint_as_float(yv[k].y), __uint_as_float(yv[k].z),
+                                   __uint_as_float(yv[k].w));
+            v.x = __fmaf_rn(scale, d.x, v.x);
+            v.y = __fmaf_rn(scale, d.y, v.y);
+            v.z = __fmaf_rn(scale, d.z, v.z);
+            v.w = __fmaf_rn(scale, d.w, v.w);
             float* p = static_cast<float*>(y) + (size_t)(m0 + row) * ldy + col;
-            float4 v = *reinterpret_cast<const float4*>(p);
-            const float* d = sD + row * L::D_PITCH + cc * 4;
-            v.x = __fmaf_rn(scale, d[0], v.x);
-            v.y = __fmaf_rn(scale, d[1], v.y);
-            v.z = __fmaf_rn(scale, d[2], v.z);
-            v.w = __fmaf_rn(scale, d[3], v.w);
             *reinterpret_cast<float4*>(p) = v;
         }
     }

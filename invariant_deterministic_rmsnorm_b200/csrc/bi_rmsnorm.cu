@@ -9,7 +9,7 @@
 // Launch plan, a function of (H, dtypes) only:
 //   vec     = 16 bytes / element size (8 bf16 or 4 fp32 elements per 128-bit load)
 //   nvec    = H / vec
-//   threads = min(256, nvec rounded up to a warp)
+//   threads = nvec / 4 rounded up to a warp, clamped to [32, 256]
 //   vpt     = ceil(nvec / threads) vectors per thread (compile-time 1, 2, 4, 8 or 16)
 // Thread t owns vectors t, t + threads, t + 2*threads, ...  It keeps them in
 // registers (one HBM read of x), sums their squares sequentially with fused
@@ -75,71 +75,125 @@ __device__ __forceinline__ void load_w(const TW* w, int64_t e0, float (&f)[V]) {
     }
 }
 
+// Row r's arithmetic: thread t owns vectors t, t + threads, ... of the row; sequential FMAs
+// per thread, a warp butterfly, then a fixed tree over the warps.  The CTA walks rows
+// r = blockIdx.x, blockIdx.x + gridDim.x, ... and keeps the next row's loads in flight
+// while it reduces the current one.  Which CTA handles a row never changes its arithmetic.
 template <typename TIO, typename TW, int VPT>
 __global__ void __launch_bounds__(kMaxThreads)
-rmsnorm_rows_kernel(const TIO* __restrict__ x, const TW* __restrict__ w, TIO* __restrict__ y, int nvec,
+rmsnorm_rows_kernel(const TIO* __restrict__ x, const TW* __restrict__ w, TIO* __restrict__ y, int64_t M, int nvec,
                     int64_t ldx, int64_t ldy, float h_float, float eps) {
     constexpr int V = IoTraits<TIO>::kVec;
-    __shared__ float warp_sums[kMaxThreads / 32];
-    __shared__ float row_total;
+    __shared__ float warp_sums[2][kMaxThreads / 32];
+    __shared__ float row_total[2];
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int nthreads = blockDim.x;
-    const int64_t row = blockIdx.x;
-    const TIO* xr = x + row * ldx;
-    TIO* yr = y + row * ldy;
+    const int nwarps = nthreads >> 5;
 
-    // 1. Stream this thread's vectors of the row into registers (all loads issued first).
-    uint4 xv[VPT];
+    uint4 xv[VPT], xn[VPT];
+    int64_t row = blockIdx.x;
+    if (row >= M) return;
+    // the weights are the same for every row: when a thread's share is small, widen them to
+    // fp32 once per CTA and keep them in registers; otherwise re-read them (L1/L2) per row
+    constexpr bool kWInRegs = VPT * V <= 32;
+    float wr[kWInRegs ? VPT : 1][V];
+    if constexpr (kWInRegs) {
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        const int v = tid + i * nthreads;
-        xv[i] = (v < nvec) ? bi::ld_stream_v4(xr + (int64_t)v * V) : make_uint4(0u, 0u, 0u, 0u);
-    }
-
-    // 2. Per-thread sum of squares, vectors in order, elements in order.
-    float ss = 0.0f;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        float f[V];
-        IoTraits<TIO>::unpack(xv[i], f);
-#pragma unroll
-        for (int e = 0; e < V; ++e) ss = __fmaf_rn(f[e], f[e], ss);
-    }
-
-    // 3. Warp butterfly.  Partners add the same two values, so every lane ends with the same bits.
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
-    if (lane == 0) warp_sums[warp] = ss;
-    __syncthreads();
-
-    // 4. Fixed tree over the warps (missing warps contribute +0, which is exact).
-    if (warp == 0) {
-        const int nwarps = nthreads >> 5;
-        float t = (lane < nwarps) ? warp_sums[lane] : 0.0f;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
-        if (lane == 0) row_total = t;
-    }
-    __syncthreads();
-
-    const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(row_total, h_float), eps));
-
-    // 5. y = (x * inv) * w, one rounding to the output type.
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        const int v = tid + i * nthreads;
-        if (v < nvec) {
-            float f[V], wf[V];
-            IoTraits<TIO>::unpack(xv[i], f);
-            load_w<TW, V>(w, (int64_t)v * V, wf);
-#pragma unroll
-            for (int e = 0; e < V; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], inv), wf[e]);
-            bi::st_stream_v4(yr + (int64_t)v * V, IoTraits<TIO>::pack(f));
+        for (int i = 0; i < VPT; ++i) {
+            const int v = tid + i * nthreads;
+            if (v < nvec) load_w<TW, V>(w, (int64_t)v * V, wr[i]);
         }
     }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = tid + i * nthreads;
+        xv[i] = (v < nvec) ? bi::ld_stream_v4(x + row * ldx + (int64_t)v * V) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int buf = 0; row < M; row += gridDim.x, buf ^= 1) {
+        // 1. prefetch the next row of this CTA
+        const int64_t nrow = row + gridDim.x;
+        if (nrow < M) {
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = tid + i * nthreads;
+                xn[i] = (v < nvec) ? bi::ld_stream_v4(x + nrow * ldx + (int64_t)v * V) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+
+        // 2. per-thread sum of squares, vectors in order, elements in order
+        float ss = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            float f[V];
+            IoTraits<TIO>::unpack(xv[i], f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) ss = __fmaf_rn(f[e], f[e], ss);
+        }
+
+        // 3. warp butterfly: partners add the same two values, so every lane ends with the same bits
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
+        if (lane == 0) warp_sums[buf][warp] = ss;
+        __syncthreads();
+
+        // 4. fixed tree over the warps (missing warps contribute +0, which is exact)
+        if (warp == 0) {
+            float t = (lane < nwarps) ? warp_sums[buf][lane] : 0.0f;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, off));
+            if (lane == 0) row_total[buf] = t;
+        }
+        __syncthreads();
+        // (the buffers alternate between rows, so the next row's writes cannot race these reads)
+
+        const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(row_total[buf], h_float), eps));
+
+        // 5. y = (x * inv) * w, one rounding to the output type
+        TIO* yr = y + row * ldy;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = tid + i * nthreads;
+            if (v < nvec) {
+                float f[V], wf[V];
+                IoTraits<TIO>::unpack(xv[i], f);
+                if constexpr (kWInRegs) {
+#pragma unroll
+                    for (int e = 0; e < V; ++e) wf[e] = wr[i][e];
+                } else {
+                    load_w<TW, V>(w, (int64_t)v * V, wf);
+                }
+#pragma unroll
+                for (int e = 0; e < V; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], inv), wf[e]);
+                bi::st_stream_v4(yr + (int64_t)v * V, IoTraits<TIO>::pack(f));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) xv[i] = xn[i];
+    }
+}
+
+// Grid: as many CTAs as fit on the GPU at once (at most one per row); each loops over rows.
+template <typename TIO, typename TW, int VPT>
+int launch_rows(const TIO* x, const TW* w, TIO* y, int64_t M, int nvec, int threads, int64_t ldx, int64_t ldy,
+                float hf, float eps, cudaStream_t s) {
+    static int resident[64][kMaxThreads / 32 + 1];  // CTAs per SM, per device and block size
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BI_ERR_CUDA;
+    int& per_sm = resident[dev][threads / 32];
+    if (per_sm == 0) {
+        int n = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rmsnorm_rows_kernel<TIO, TW, VPT>, threads, 0) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return BI_ERR_CUDA;
+        per_sm = (n > 0 ? n : 1) * sms;
+    }
+    const int64_t grid = M < per_sm ? M : per_sm;
+    rmsnorm_rows_kernel<TIO, TW, VPT><<<(unsigned)grid, threads, 0, s>>>(x, w, y, M, nvec, ldx, ldy, hf, eps);
+    return bi::launch_status();
 }
 
 template <typename TIO, typename TW>
@@ -147,25 +201,21 @@ int launch_typed(const void* x, const void* w, void* y, int64_t M, int64_t H, in
                  cudaStream_t s) {
     constexpr int V = IoTraits<TIO>::kVec;
     const int nvec = (int)(H / V);
-    int threads = ((nvec + 31) / 32) * 32;
+    int threads = ((nvec / 4 + 31) / 32) * 32;  // about four 16-byte vectors per thread
+    if (threads < 32) threads = 32;
     if (threads > kMaxThreads) threads = kMaxThreads;
     const int vpt = (nvec + threads - 1) / threads;
-    dim3 grid((unsigned)M), block(threads);
     const TIO* xp = static_cast<const TIO*>(x);
     const TW* wp = static_cast<const TW*>(w);
     TIO* yp = static_cast<TIO*>(y);
     const float hf = (float)H;
     switch (vpt) {
-        case 1: rmsnorm_rows_kernel<TIO, TW, 1><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
-        case 2: rmsnorm_rows_kernel<TIO, TW, 2><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
-        case 3: case 4:
-            rmsnorm_rows_kernel<TIO, TW, 4><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
-        case 5: case 6: case 7: case 8:
-            rmsnorm_rows_kernel<TIO, TW, 8><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
-        default:
-            rmsnorm_rows_kernel<TIO, TW, 16><<<grid, block, 0, s>>>(xp, wp, yp, nvec, ldx, ldy, hf, eps); break;
+        case 1: return launch_rows<TIO, TW, 1>(xp, wp, yp, M, nvec, threads, ldx, ldy, hf, eps, s);
+        case 2: return launch_rows<TIO, TW, 2>(xp, wp, yp, M, nvec, threads, ldx, ldy, hf, eps, s);
+        case 3: case 4: return launch_rows<TIO, TW, 4>(xp, wp, yp, M, nvec, threads, ldx, ldy, hf, eps, s);
+        case 5: case 6: case 7: case 8: return launch_rows<TIO, TW, 8>(xp, wp, yp, M, nvec, threads, ldx, ldy, hf, eps, s);
+        default: return launch_rows<TIO, TW, 16>(xp, wp, yp, M, nvec, threads, ldx, ldy, hf, eps, s);
     }
-    return bi::launch_status();
 }
 
 }  // namespace
