@@ -26,6 +26,42 @@ extern "C" {
 int bi_ctrl_lora_shrink_atomic(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r,
                                int32_t split_k, void* stream);
 
+/*
+ * bi_ctrl_rmsnorm_split -- RMSNorm whose row reduction is cut across S CTAs of a
+ * thread-block cluster, S in {1, 2, 4, 8}, chosen from M (more pieces for smaller batches).
+ * It is the small-batch "split reduction" that "Defeating Nondeterminism in LLM
+ * Inference" (Spanish summary, section "Diseño de kernels invariantes al batch",
+ * RMSNorm) names as the strategy that sacrifices batch invariance.  Arguments as
+ * bi_rmsnorm.  The row length H must split into slices of at most 1024 16-byte vectors,
+ * and M <= 65535.
+ */
+int bi_ctrl_rmsnorm_split(const void* x, const void* w, void* y, int64_t M, int64_t H, int64_t ldx, int64_t ldy,
+                          float eps, int io_dtype, int w_dtype, void* stream);
+
+/*
+ * bi_ctrl_gemm_splitk -- bi_gemm with a split-K chosen from M, the batch-size-dependent
+ * strategy of the "Multiplicación de matrices" section of the same page.  When the batch
+ * alone yields too few output tiles to fill the GPU, K is cut into S in {2, 4, 8} slices.
+ * Each slice is a bi_gemm into fp32 partials in ws.  The partials are then added in slice
+ * order and rounded to c_dtype.  A row's accumulation order therefore depends on M.
+ * ws must hold bi_ctrl_gemm_splitk_workspace_size(M, N, K) bytes (0 when S = 1).
+ */
+size_t bi_ctrl_gemm_splitk_workspace_size(int64_t M, int64_t N, int64_t K);
+int bi_ctrl_gemm_splitk(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * bi_ctrl_decode_attn_adaptive -- bi_decode_attn with the split size chosen from the
+ * batch: 128-token chunks when B < 16, 256 otherwise.  That is the batch-dependent
+ * split-KV which the "Attention" section of the same page warns against.  Arguments as
+ * bi_decode_attn (head_dim 128).  ws must hold
+ * bi_ctrl_decode_attn_adaptive_workspace_size(total_tokens, Hq) bytes.
+ */
+size_t bi_ctrl_decode_attn_adaptive_workspace_size(int64_t total_tokens, int32_t Hq);
+int bi_ctrl_decode_attn_adaptive(const void* q, const void* k, const void* v, const int32_t* kv_indptr,
+                                 const int32_t* kv_len, int32_t B, int64_t total_tokens, int32_t Hq, int32_t Hkv,
+                                 float scale, void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -60,6 +60,11 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_ctrl_lora_shrink_atomic": ([P, P, P, I64, I64, I32, I32, P], C),
         "bi_decode_attn_workspace_size": ([I64, I32, I32, I32], Z),
         "bi_decode_attn": ([P, P, P, P, P, I32, I64, I32, I32, I32, F, I32, P, C, P, Z, P], C),
+        "bi_ctrl_rmsnorm_split": ([P, P, P, I64, I64, I64, I64, F, C, C, P], C),
+        "bi_ctrl_gemm_splitk_workspace_size": ([I64, I64, I64], Z),
+        "bi_ctrl_gemm_splitk": ([P, P, P, I64, I64, I64, C, P, Z, P], C),
+        "bi_ctrl_decode_attn_adaptive_workspace_size": ([I64, I32], Z),
+        "bi_ctrl_decode_attn_adaptive": ([P, P, P, P, P, I32, I64, I32, I32, F, P, C, P, Z, P], C),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -231,6 +236,60 @@ def bi_decode_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_indptr:
                             float(scale), chunk, _ptr(out), _dtype_code(out), _ptr(workspace),
                             workspace.numel() * workspace.element_size(), _stream(stream))
     _check("bi_decode_attn", st)
+    return out
+
+
+# ------------------------------------------------------------------ comparators (not batch-invariant)
+def bi_ctrl_rmsnorm_split(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, eps: float = 1e-6,
+                          stream=None) -> torch.Tensor:
+    """Comparator: RMSNorm with the row reduction split across a cluster, split count chosen from M."""
+    _rows(x, "x")
+    if y is None:
+        y = torch.empty_like(x, memory_format=torch.contiguous_format)
+    M, H = x.shape
+    st = library().bi_ctrl_rmsnorm_split(_ptr(x), _ptr(w), _ptr(y), M, H, max(x.stride(0), H),
+                                         max(y.stride(0), H), float(eps), _dtype_code(x), _dtype_code(w),
+                                         _stream(stream))
+    _check("bi_ctrl_rmsnorm_split", st)
+    return y
+
+
+def bi_ctrl_gemm_splitk(A: torch.Tensor, W: torch.Tensor, C: torch.Tensor | None = None, out_dtype=torch.float32,
+                        stream=None) -> torch.Tensor:
+    """Comparator: GEMM with a split-K chosen from M (fp32 partials, ordered sum)."""
+    _bf16_2d(A, "A")
+    _bf16_2d(W, "W")
+    M, K = A.shape
+    N = W.shape[1]
+    if C is None:
+        C = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    lib = library()
+    need = lib.bi_ctrl_gemm_splitk_workspace_size(M, N, K)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=A.device)
+    st = lib.bi_ctrl_gemm_splitk(_ptr(A), _ptr(W), _ptr(C), M, N, K, _dtype_code(C), _ptr(ws), ws.numel(),
+                                 _stream(stream))
+    _check("bi_ctrl_gemm_splitk", st)
+    return C
+
+
+def bi_ctrl_decode_attn_adaptive(q, k, v, kv_indptr, kv_len, out=None, scale=None, out_dtype=torch.bfloat16,
+                                 workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Comparator: decode attention with 128-token chunks for batches under 16, 256 otherwise."""
+    B, Hq, D = q.shape
+    T, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=out_dtype, device=q.device)
+    lib = library()
+    need = lib.bi_ctrl_decode_attn_adaptive_workspace_size(T, Hq)
+    ws = workspace
+    if ws is None or ws.numel() * ws.element_size() < need:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib.bi_ctrl_decode_attn_adaptive(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_indptr), _ptr(kv_len), B, T, Hq, Hkv,
+                                          float(scale), _ptr(out), _dtype_code(out), _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream))
+    _check("bi_ctrl_decode_attn_adaptive", st)
     return out
 
 

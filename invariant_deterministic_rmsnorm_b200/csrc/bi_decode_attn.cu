@@ -84,10 +84,11 @@ struct SeqCache {
     int len = 0;
 };
 
-// The (sequence, chunk) that owns 256-token slot `slot` of the packed cache.
+// The (sequence, chunk) that owns CH-token slot `slot` of the packed cache.
+template <int CH>
 __device__ __forceinline__ Item item_of(int slot, const int32_t* __restrict__ kv_indptr,
                                         const int32_t* __restrict__ kv_len, int B, bool& bad, SeqCache& sc) {
-    Item it{0, 0, 0, (int64_t)slot * CHUNK};
+    Item it{0, 0, 0, (int64_t)slot * CH};
     bad = false;
     int lo;
     if (sc.b >= 0 && it.tok0 >= sc.lo_tok && it.tok0 < sc.hi_tok) {
@@ -109,12 +110,12 @@ __device__ __forceinline__ Item item_of(int slot, const int32_t* __restrict__ kv
     const int len = sc.len;
     const int64_t cap = sc.hi_tok - sbase;
     if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap) {
-        bad = (it.tok0 - sbase) < CHUNK;  // report once per sequence
+        bad = (it.tok0 - sbase) < CH;  // report once per sequence
         return it;
     }
     it.b = lo;
-    it.c = (int)((it.tok0 - sbase) / CHUNK);
-    it.n_tok = max(0, min(CHUNK, len - it.c * CHUNK));
+    it.c = (int)((it.tok0 - sbase) / CH);
+    it.n_tok = max(0, min(CH, len - it.c * CH));
     return it;
 }
 
@@ -122,7 +123,7 @@ __device__ __forceinline__ Item item_of(int slot, const int32_t* __restrict__ kv
 // kv head w % Hkv), so consecutive items share a slot and usually a sequence.
 // A producer warp streams each item's K sub-blocks, then its V sub-blocks, through an NSTAGES ring;
 // eight compute warps consume them in the same order.
-template <int G>
+template <int G, int CH>
 __global__ void __launch_bounds__(THREADS, 2)
 decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ kv_indptr,
@@ -167,7 +168,7 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             for (int w = w_begin; w < w_end && !*abort; ++w) {
                 const int slot = w / Hkv, g = w % Hkv;
                 bool bad;
-                const Item itm = item_of(slot, kv_indptr, kv_len, B, bad, sc);
+                const Item itm = item_of<CH>(slot, kv_indptr, kv_len, B, bad, sc);
                 if (bad && g == 0) atomicOr(err, DEVERR_BAD_LAYOUT);
                 if (itm.n_tok == 0) continue;
                 const int nsub = (itm.n_tok + SUB - 1) / SUB;
@@ -210,7 +211,7 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     for (int w = w_begin; w < w_end; ++w) {
         const int slot = w / Hkv, g = w % Hkv;
         bool bad;
-        const Item itm = item_of(slot, kv_indptr, kv_len, B, bad, sc);
+        const Item itm = item_of<CH>(slot, kv_indptr, kv_len, B, bad, sc);
         if (itm.n_tok == 0) continue;
         const int n_tok = itm.n_tok;
         const int nsub = (n_tok + SUB - 1) / SUB;
@@ -386,7 +387,7 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 }
 
 // Phase 2: one warp per (sequence, query head); lane owns dims [4*lane, 4*lane + 4).
-template <bool OUT_BF16>
+template <bool OUT_BF16, int CH>
 __global__ void __launch_bounds__(128)
 decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restrict__ ml_part,
                          const int32_t* __restrict__ kv_indptr, const int32_t* __restrict__ kv_len, int Hq,
@@ -402,8 +403,8 @@ decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restri
         if (lane == 0) atomicOr(err, DEVERR_BAD_LAYOUT);  // out row left unwritten
         return;
     }
-    const int nch = (len + CHUNK - 1) / CHUNK;
-    const int64_t slot0 = sbase / CHUNK;
+    const int nch = (len + CH - 1) / CH;
+    const int64_t slot0 = sbase / CH;
     float m = -INFINITY, l = 0.0f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int c = 0; c < nch; ++c) {
@@ -463,17 +464,17 @@ int num_sms() {
     return cached[dev];
 }
 
-size_t partial_bytes(int64_t total_tokens, int32_t Hq) {
-    const int64_t slots = (total_tokens + CHUNK - 1) / CHUNK;
+size_t partial_bytes(int64_t total_tokens, int32_t Hq, int ch = CHUNK) {
+    const int64_t slots = (total_tokens + ch - 1) / ch;
     return (size_t)slots * Hq * (D + 2) * sizeof(float);
 }
 
-template <int G>
+template <int G, int CH = CHUNK>
 int launch_chunks(const void* q, const void* k, const void* v, const int32_t* kv_indptr, const int32_t* kv_len,
                   int B, int64_t T, int Hq, int Hkv, float scale, float* o_part, float* ml_part, cudaStream_t s) {
     using L = AttnLayout<G>;
     uint32_t* err = bi::device_error_word();
-    auto kern = decode_attn_chunk_kernel<G>;
+    auto kern = decode_attn_chunk_kernel<G, CH>;
     if (!err || !set_smem_once(kern, L::BYTES)) return BI_ERR_CUDA;
     CUtensorMap tmK, tmV;
     const uint64_t row = (uint64_t)Hkv * D;  // elements per packed token
@@ -482,7 +483,7 @@ int launch_chunks(const void* q, const void* k, const void* v, const int32_t* kv
         !bi::make_tmap_2d(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, row, (uint64_t)T, row * 2, 64, BOX_TOK,
                           CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
-    const int64_t items = ((T + CHUNK - 1) / CHUNK) * Hkv;
+    const int64_t items = ((T + CH - 1) / CH) * Hkv;
     if (items > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
     const int sms = num_sms();
     if (sms <= 0) return BI_ERR_CUDA;
@@ -530,9 +531,9 @@ BI_API int bi_decode_attn(const void* q, const void* k, const void* v, const int
     dim3 grid((unsigned)((Hq + 3) / 4), (unsigned)B);
     uint32_t* err = bi::device_error_word();
     if (out_dtype == BI_BF16)
-        decode_attn_merge_kernel<true><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        decode_attn_merge_kernel<true, CHUNK><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
     else
-        decode_attn_merge_kernel<false><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        decode_attn_merge_kernel<false, CHUNK><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
     return bi::launch_status();
 }
 
@@ -607,8 +608,68 @@ BI_API int bi_decode_attn_noalloc(const void* q, const void* k, const void* v, c
     uint32_t* err = bi::device_error_word();
     dim3 grid((unsigned)((Hq + 3) / 4), (unsigned)B);
     if (out_dtype == BI_BF16)
-        decode_attn_merge_kernel<true><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        decode_attn_merge_kernel<true, CHUNK><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
     else
-        decode_attn_merge_kernel<false><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        decode_attn_merge_kernel<false, CHUNK><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
     return bi::launch_status();
+}
+
+// ------------------------------------------------------------------ comparator: batch-adaptive split
+//
+// What a batch-size-adaptive split-KV kernel does: when the batch is small, cut the cache into
+// more, smaller chunks (128 tokens instead of 256) to fill the GPU.  A request's chunking, and
+// so its merge order, then depends on how many other requests share its batch: not batch-invariant.
+namespace {
+
+template <int CH>
+int run_adaptive(const void* q, const void* k, const void* v, const int32_t* kv_indptr, const int32_t* kv_len,
+                 int B, int64_t T, int Hq, int Hkv, float scale, void* out, int out_dtype, float* ws, cudaStream_t s) {
+    const int G = Hq / Hkv;
+    const int64_t slots = (T + CH - 1) / CH;
+    float* o_part = ws;
+    float* ml_part = o_part + (size_t)slots * Hq * D;
+    int st;
+    switch (G) {
+        case 1: st = launch_chunks<1, CH>(q, k, v, kv_indptr, kv_len, B, T, Hq, Hkv, scale, o_part, ml_part, s); break;
+        case 2: st = launch_chunks<2, CH>(q, k, v, kv_indptr, kv_len, B, T, Hq, Hkv, scale, o_part, ml_part, s); break;
+        case 4: st = launch_chunks<4, CH>(q, k, v, kv_indptr, kv_len, B, T, Hq, Hkv, scale, o_part, ml_part, s); break;
+        default: st = launch_chunks<8, CH>(q, k, v, kv_indptr, kv_len, B, T, Hq, Hkv, scale, o_part, ml_part, s); break;
+    }
+    if (st != BI_OK) return st;
+    uint32_t* err = bi::device_error_word();
+    dim3 grid((unsigned)((Hq + 3) / 4), (unsigned)B);
+    if (out_dtype == BI_BF16)
+        decode_attn_merge_kernel<true, CH><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+    else
+        decode_attn_merge_kernel<false, CH><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+    return bi::launch_status();
+}
+
+}  // namespace
+
+BI_API size_t bi_ctrl_decode_attn_adaptive_workspace_size(int64_t total_tokens, int32_t Hq) {
+    if (total_tokens <= 0 || Hq <= 0) return 0;
+    return partial_bytes(total_tokens, Hq, 128);
+}
+
+BI_API int bi_ctrl_decode_attn_adaptive(const void* q, const void* k, const void* v, const int32_t* kv_indptr,
+                                        const int32_t* kv_len, int32_t B, int64_t total_tokens, int32_t Hq,
+                                        int32_t Hkv, float scale, void* out, int out_dtype, void* ws, size_t ws_bytes,
+                                        void* stream) {
+    if (out_dtype != BI_F32 && out_dtype != BI_BF16) return BI_ERR_INVALID_ARG;
+    if (B < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return BI_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0) return BI_OK;
+    if (total_tokens == 0 || !q || !k || !v || !kv_indptr || !kv_len || !out) return BI_ERR_INVALID_ARG;
+    if (total_tokens > 0x7fffffffLL || B > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (!bi::aligned16(q) || !bi::aligned16(k) || !bi::aligned16(v) || !bi::aligned16(out)) return BI_ERR_MISALIGNED;
+    const int ch = B < 16 ? 128 : 256;
+    if (!ws || ws_bytes < partial_bytes(total_tokens, Hq, ch) || !bi::aligned16(ws)) return BI_ERR_WORKSPACE;
+    cudaStream_t s = bi::as_stream(stream);
+    if (ch == 128)
+        return run_adaptive<128>(q, k, v, kv_indptr, kv_len, B, total_tokens, Hq, Hkv, scale, out, out_dtype,
+                                 static_cast<float*>(ws), s);
+    return run_adaptive<256>(q, k, v, kv_indptr, kv_len, B, total_tokens, Hq, Hkv, scale, out, out_dtype,
+                             static_cast<float*>(ws), s);
 }

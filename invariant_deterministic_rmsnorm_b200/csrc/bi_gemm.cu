@@ -269,6 +269,74 @@ bool ensure_smem_attr() {
     return ok[dev];
 }
 
+
+// Launch the GEMM on operands with arbitrary (16-byte multiple) row strides: A [M, K] with
+// row stride lda, W [K, N] with row stride ldw, C [M, N] with row stride N.
+int launch_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N, int64_t K,
+                bool c_bf16, cudaStream_t stream) {
+    uint32_t* err = bi::device_error_word();
+    if (!err || !ensure_smem_attr()) return BI_ERR_CUDA;
+    CUtensorMap tmA, tmW;
+    if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK,
+                          BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    if (!bi::make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)N, (uint64_t)K, (uint64_t)ldw * 2, 64,
+                          BK, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int sms = num_sms();
+    if (sms <= 0) return BI_ERR_CUDA;
+    const int gm = 16;  // ~16 row tiles x ~9 column tiles in flight: A and W blocks balanced within L2
+    dim3 grid((unsigned)(tiles < sms ? tiles : sms));
+    bi_gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmW, C, (int)M, (int)N, (int)K,
+                                                                   c_bf16 ? 1 : 0, gm, err);
+    return bi::launch_status();
+}
+
+int gemm_shape_checks(const void* A, const void* W, const void* C, int64_t M, int64_t N, int64_t K, int c_dtype) {
+    if (c_dtype != BI_F32 && c_dtype != BI_BF16) return BI_ERR_INVALID_ARG;
+    if (M < 0 || N <= 0 || K <= 0) return BI_ERR_INVALID_ARG;
+    if (M == 0) return -1;  // no-op
+    if (!A || !W || !C) return BI_ERR_INVALID_ARG;
+    if (!bi::aligned16(A) || !bi::aligned16(W) || !bi::aligned16(C)) return BI_ERR_MISALIGNED;
+    if (K % 8 != 0 || N % 8 != 0) return BI_ERR_MISALIGNED;  // 16-byte row strides for the TMA unit
+    if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (((M + BM - 1) / BM) * ((N + BN - 1) / BN) > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
+    return BI_OK;
+}
+
+// ------------------------------------------------------------------ comparator: split-K chosen by M
+// Sum of S fp32 partials in order s = 0, 1, ..., S-1, then the output rounding.
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, void* __restrict__ C, int64_t MN, int S,
+                                     int c_bf16) {
+    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (i >= MN) return;
+    float4 acc = *reinterpret_cast<const float4*>(part + i);
+    for (int s = 1; s < S; ++s) {
+        const float4 p = *reinterpret_cast<const float4*>(part + (int64_t)s * MN + i);
+        acc.x = __fadd_rn(acc.x, p.x);
+        acc.y = __fadd_rn(acc.y, p.y);
+        acc.z = __fadd_rn(acc.z, p.z);
+        acc.w = __fadd_rn(acc.w, p.w);
+    }
+    if (c_bf16) {
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(C) + i) =
+            make_uint2(bi::pack_bf16x2(acc.x, acc.y), bi::pack_bf16x2(acc.z, acc.w));
+    } else {
+        *reinterpret_cast<float4*>(static_cast<float*>(C) + i) = acc;
+    }
+}
+
+// The split a batch-size-adaptive library would pick: enough K slices to fill the GPU when
+// the batch alone yields too few output tiles (1, 2, 4 or 8, with K / S a multiple of 64).
+int splitk_for(int64_t M, int64_t N, int64_t K) {
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    int S = 1;
+    while (S < 8 && tiles * S * 2 <= sms && K % ((int64_t)S * 2 * BK) == 0) S *= 2;
+    return S;
+}
+
 }  // namespace
 
 BI_API size_t bi_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
@@ -279,29 +347,38 @@ BI_API size_t bi_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 BI_API int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype, void* ws,
                    size_t ws_bytes, void* stream) {
     (void)ws; (void)ws_bytes;
-    if (c_dtype != BI_F32 && c_dtype != BI_BF16) return BI_ERR_INVALID_ARG;
-    if (M < 0 || N <= 0 || K <= 0) return BI_ERR_INVALID_ARG;
-    if (M == 0) return BI_OK;
-    if (!A || !W || !C) return BI_ERR_INVALID_ARG;
-    if (!bi::aligned16(A) || !bi::aligned16(W) || !bi::aligned16(C)) return BI_ERR_MISALIGNED;
-    if (K % 8 != 0 || N % 8 != 0) return BI_ERR_MISALIGNED;  // 16-byte row strides for the TMA unit
-    if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return BI_ERR_UNSUPPORTED_SHAPE;
-    if (((M + BM - 1) / BM) * ((N + BN - 1) / BN) > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
-    uint32_t* err = bi::device_error_word();
-    if (!err || !ensure_smem_attr()) return BI_ERR_CUDA;
-    CUtensorMap tmA, tmW;
-    if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK,
-                          BM, CU_TENSOR_MAP_SWIZZLE_128B))
-        return BI_ERR_CUDA;
-    if (!bi::make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)N, (uint64_t)K, (uint64_t)N * 2, 64,
-                          BK, CU_TENSOR_MAP_SWIZZLE_128B))
-        return BI_ERR_CUDA;
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int sms = num_sms();
-    if (sms <= 0) return BI_ERR_CUDA;
-    const int gm = 16;  // ~16 row tiles x ~9 column tiles in flight: A and W blocks balanced within L2
-    dim3 grid((unsigned)(tiles < sms ? tiles : sms));
-    bi_gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, bi::as_stream(stream)>>>(
-        tmA, tmW, C, (int)M, (int)N, (int)K, c_dtype == BI_BF16 ? 1 : 0, gm, err);
+    const int c = gemm_shape_checks(A, W, C, M, N, K, c_dtype);
+    if (c < 0) return BI_OK;
+    if (c != BI_OK) return c;
+    return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, bi::as_stream(stream));
+}
+
+BI_API size_t bi_ctrl_gemm_splitk_workspace_size(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    const int S = splitk_for(M, N, K);
+    return S > 1 ? (size_t)S * M * N * sizeof(float) : 0;
+}
+
+BI_API int bi_ctrl_gemm_splitk(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype,
+                               void* ws, size_t ws_bytes, void* stream) {
+    const int c = gemm_shape_checks(A, W, C, M, N, K, c_dtype);
+    if (c < 0) return BI_OK;
+    if (c != BI_OK) return c;
+    cudaStream_t s = bi::as_stream(stream);
+    const int S = splitk_for(M, N, K);
+    if (S == 1) return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, s);
+    const size_t need = (size_t)S * M * N * sizeof(float);
+    if (!ws || ws_bytes < need || !bi::aligned16(ws)) return BI_ERR_WORKSPACE;
+    const int64_t KS = K / S;
+    float* part = static_cast<float*>(ws);
+    for (int i = 0; i < S; ++i) {
+        const int st = launch_gemm(static_cast<const __nv_bfloat16*>(A) + i * KS, K,
+                                   static_cast<const __nv_bfloat16*>(W) + i * KS * N, N, part + (int64_t)i * M * N, M,
+                                   N, KS, false, s);
+        if (st != BI_OK) return st;
+    }
+    const int64_t MN = M * N;  // N % 8 == 0, so MN is a multiple of 4
+    const int64_t threads = (MN / 4 + 255) / 256;
+    splitk_reduce_kernel<<<(unsigned)threads, 256, 0, s>>>(part, C, MN, S, c_dtype == BI_BF16 ? 1 : 0);
     return bi::launch_status();
 }

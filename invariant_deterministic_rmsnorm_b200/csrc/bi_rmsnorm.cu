@@ -17,6 +17,7 @@
 // fixed tree over the warps.  Because the plan depends on H alone, every row is
 // reduced in exactly the same order at every M and every row position.
 #include "bi_common.cuh"
+#include "bi_sm100.cuh"
 
 namespace {
 
@@ -242,4 +243,119 @@ BI_API int bi_rmsnorm(const void* x, const void* w, void* y, int64_t M, int64_t 
     if (io_dtype == BI_BF16 && w_dtype == BI_BF16)
         return launch_typed<__nv_bfloat16, __nv_bfloat16>(x, w, y, M, H, ldx, ldy, eps, s);
     return launch_typed<__nv_bfloat16, float>(x, w, y, M, H, ldx, ldy, eps, s);
+}
+
+// ------------------------------------------------------------------ comparator: split reduction
+//
+// The small-batch alternative the RMSNorm section mentions: when the batch is small, cut each
+// row across S CTAs (a thread-block cluster), reduce the slices in parallel and exchange the
+// partial sums over distributed shared memory.  S is chosen from M, so a row's reduction tree
+// changes with the batch size: faster for small batches, and not batch-invariant.
+namespace {
+
+int split_for(int64_t M, int64_t nvec) {
+    int S = M <= 148 ? 8 : (M <= 296 ? 4 : (M <= 592 ? 2 : 1));
+    while (S > 1 && (nvec % S != 0 || nvec / S < 32)) S >>= 1;
+    return S;
+}
+
+template <typename TIO, typename TW>
+__global__ void __launch_bounds__(128)
+rmsnorm_split_kernel(const TIO* __restrict__ x, const TW* __restrict__ w, TIO* __restrict__ y, int nvec_slice,
+                     int64_t ldx, int64_t ldy, float h_float, float eps) {
+    constexpr int V = IoTraits<TIO>::kVec;
+    constexpr int MAXV = 8;
+    __shared__ float warp_sums[4];
+    __shared__ float slice_sum;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t rank = bi::sm100::cluster_ctarank();
+    const uint32_t S = gridDim.x;
+    const int64_t row = blockIdx.y;
+    const int64_t v0 = (int64_t)rank * nvec_slice;
+    uint4 xv[MAXV];
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int v = tid + i * 128;
+        xv[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (v < nvec_slice) {
+            xv[i] = bi::ld_stream_v4(x + row * ldx + (v0 + v) * V);
+            float f[V];
+            IoTraits<TIO>::unpack(xv[i], f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) ss = __fmaf_rn(f[e], f[e], ss);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
+    if (lane == 0) warp_sums[warp] = ss;
+    __syncthreads();
+    if (tid == 0) slice_sum = __fadd_rn(__fadd_rn(warp_sums[0], warp_sums[1]), __fadd_rn(warp_sums[2], warp_sums[3]));
+    bi::sm100::cluster_sync();
+    float total = 0.0f;
+    const uint32_t local = bi::sm100::smem_u32(&slice_sum);
+    for (uint32_t s = 0; s < S; ++s) {
+        float p;
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(p) : "r"(bi::sm100::mapa(local, s)) : "memory");
+        total = __fadd_rn(total, p);
+    }
+    const float inv = __frsqrt_rn(__fadd_rn(__fdiv_rn(total, h_float), eps));
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int v = tid + i * 128;
+        if (v < nvec_slice) {
+            float f[V], wf[V];
+            IoTraits<TIO>::unpack(xv[i], f);
+            load_w<TW, V>(w, (v0 + v) * V, wf);
+#pragma unroll
+            for (int e = 0; e < V; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], inv), wf[e]);
+            bi::st_stream_v4(y + row * ldy + (v0 + v) * V, IoTraits<TIO>::pack(f));
+        }
+    }
+    bi::sm100::cluster_sync();  // peers keep their partial sums until every CTA has read them
+}
+
+template <typename TIO, typename TW>
+int launch_split(const void* x, const void* w, void* y, int64_t M, int64_t H, int64_t ldx, int64_t ldy, float eps,
+                 cudaStream_t s) {
+    constexpr int V = IoTraits<TIO>::kVec;
+    const int64_t nvec = H / V;
+    const int S = split_for(M, nvec);
+    const int64_t nvs = nvec / S;
+    if (nvs > 128 * 8 || M > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)S, (unsigned)M, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, rmsnorm_split_kernel<TIO, TW>, static_cast<const TIO*>(x), static_cast<const TW*>(w),
+                           static_cast<TIO*>(y), (int)nvs, ldx, ldy, (float)H, eps) != cudaSuccess)
+        return BI_ERR_CUDA;
+    return bi::launch_status();
+}
+
+}  // namespace
+
+BI_API int bi_ctrl_rmsnorm_split(const void* x, const void* w, void* y, int64_t M, int64_t H, int64_t ldx,
+                                 int64_t ldy, float eps, int io_dtype, int w_dtype, void* stream) {
+    const int es = bi::elem_size(io_dtype);
+    const int ws = bi::elem_size(w_dtype);
+    if (es == 0 || ws == 0) return BI_ERR_INVALID_ARG;
+    if (M < 0 || H <= 0 || ldx < H || ldy < H || !(eps >= 0.0f)) return BI_ERR_INVALID_ARG;
+    if (M == 0) return BI_OK;
+    if (!x || !w || !y) return BI_ERR_INVALID_ARG;
+    if (H % (16 / es) != 0 || H % (16 / ws) != 0 || (ldx * es) % 16 != 0 || (ldy * es) % 16 != 0)
+        return BI_ERR_MISALIGNED;
+    if (!bi::aligned16(x) || !bi::aligned16(w) || !bi::aligned16(y)) return BI_ERR_MISALIGNED;
+    cudaStream_t s = bi::as_stream(stream);
+    if (io_dtype == BI_F32 && w_dtype == BI_F32) return launch_split<float, float>(x, w, y, M, H, ldx, ldy, eps, s);
+    if (io_dtype == BI_F32) return launch_split<float, __nv_bfloat16>(x, w, y, M, H, ldx, ldy, eps, s);
+    if (w_dtype == BI_BF16) return launch_split<__nv_bfloat16, __nv_bfloat16>(x, w, y, M, H, ldx, ldy, eps, s);
+    return launch_split<__nv_bfloat16, float>(x, w, y, M, H, ldx, ldy, eps, s);
 }
