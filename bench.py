@@ -331,6 +331,12 @@ def run_ours(args, rank, world, local_rank):
         return None
 
     peaks, peak_src = load_peaks()
+    # A kernel timed inside a long step (a timed region of half a second or more, long enough for
+    # the 1 kW power cap to engage) is compared with the sustained bf16 figure; a short region
+    # gets the burst figure.
+    long_step = total_ms >= 500.0
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) if long_step else peaks["bf16_tflops"]
+    tensor_peak_name = "bf16_tflops_sustained" if long_step else "bf16_tflops (burst)"
     per_op = {}
     for op, ms in zip(ops, op_ms):
         avg_s = ms / K / 1e3
@@ -340,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
             unit = "GB/s"
         else:
             ach = op["work"] / avg_s / 1e12
-            peak = peaks["bf16_tflops"]
+            peak = tensor_peak
             unit = "TFLOP/s"
         per_op[op["name"]] = {"us": round(avg_s * 1e6, 2), "achieved": round(ach, 1), "unit": unit,
                               "frac": round(ach / peak, 4), "desc": op["desc"]}
@@ -370,13 +376,15 @@ def run_ours(args, rank, world, local_rank):
         runit, bound = "GB/s", "hbm"
     else:
         ach = dop["work"] / d_avg_s / 1e12
-        peak = peaks["bf16_tflops"]
+        peak = tensor_peak
         runit, bound = "TFLOP/s", "tensor"
     tr = TRAFFIC.get(dop["name"])
     traffic = tr[1] if tr and tr[0] == _src_sha(dop["src"]) else None
     roofline = {"bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": runit,
                 "frac": round(ach / peak, 4), "traffic": traffic, "kernel": dop["name"],
-                "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+                "peak_source": (f"{peak_src} (MEASURED_PEAKS.json" + (f", {tensor_peak_name})" if bound == "tensor"
+                                                                       else ", hbm_gbs)"))
+                if peak_src == "measured" else "fallback",
                 "algorithmic_work_per_launch": dop["work"]}
 
     cpu = cpu_baseline(args.cpu_seconds)
@@ -646,6 +654,106 @@ def run_reference(args, rank, world):
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_sweep(args):
+    """Throughput of every op across batch sizes, next to its batch-dependent fast path (one GPU).
+    Prints one JSON object per (op, shape) with a row per batch size."""
+    import torch
+    from invariant_deterministic_rmsnorm_b200 import binding as B
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device)
+    lib = B.library()
+    peaks, _ = load_peaks()
+
+    def emit(d):
+        print(json.dumps(d), flush=True)
+
+    def rows_dev(seed, M, cols):
+        g = torch.Generator(device=device).manual_seed(seed)
+        return torch.randn((M, cols), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+    # GEMM
+    for i, (K, N) in enumerate(GEMM_SHAPES):
+        table = []
+        for M in (1, 16, 64, 128, 256, 512, 1024, 2048, 4096, 8192):
+            R = _copies(2 * (M * K + K * N + M * N))
+            Ws = [rows_dev(50 + j, K, N).mul_(0.02) for j in range(R)]
+            As = [rows_dev(60 + j, M, K) for j in range(R)]
+            Cs = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(R)]
+            fl = 2 * M * N * K / 1e12
+            t_bi = _time_graph([lambda j=j: B.bi_gemm(As[j], Ws[j], C=Cs[j], stream=stream) for j in range(R)], stream)
+            t_cb = _time_graph([lambda j=j: torch.matmul(As[j], Ws[j], out=Cs[j]) for j in range(R)], stream)
+            table.append({"M": M, "bi_tflops": round(fl / (t_bi / 1e3), 1), "cublas_tflops": round(fl / (t_cb / 1e3), 1),
+                          "bi_frac_burst": round(fl / (t_bi / 1e3) / peaks["bf16_tflops"], 3)})
+            del Ws, As, Cs
+        emit({"op": "gemm", "K": K, "N": N, "rows": table})
+    # RMSNorm
+    table = []
+    w = _to_dev(inputs.rmsnorm_case(1, HIDDEN, "bf16")[1], device)
+    for M in (1, 64, 256, 1024, 4096, 8192, 16384):
+        R = _copies(2 * 2 * HIDDEN * M)
+        xs = [rows_dev(70 + j, M, HIDDEN) for j in range(R)]
+        ys = [torch.empty_like(xs[0]) for _ in range(R)]
+        by = 2 * 2 * HIDDEN * M / 1e9
+        t_bi = _time_graph([lambda j=j: B.bi_rmsnorm(xs[j], w, y=ys[j], stream=stream) for j in range(R)], stream)
+        t_sp = _time_graph([lambda j=j: B.bi_ctrl_rmsnorm_split(xs[j], w, y=ys[j], stream=stream) for j in range(R)],
+                           stream)
+        table.append({"M": M, "bi_gbs": round(by / (t_bi / 1e3), 1), "split_gbs": round(by / (t_sp / 1e3), 1),
+                      "bi_frac": round(by / (t_bi / 1e3) / peaks["hbm_gbs"], 3)})
+        del xs, ys
+    emit({"op": "rmsnorm", "H": HIDDEN, "dtype": "bf16", "rows": table})
+    # LoRA shrink and expand
+    for r in (8, 16, 64):
+        A_l = rows_dev(80, HIDDEN, r).mul_(0.02)
+        B_l = rows_dev(81, r, HIDDEN).mul_(0.02)
+        table = []
+        for M in (1, 64, 256, 1024, 4096):
+            R = _copies(2 * HIDDEN * M)
+            xs = [rows_dev(90 + j, M, HIDDEN) for j in range(R)]
+            t = torch.empty((M, r), dtype=torch.float32, device=device)
+            ys = [rows_dev(100 + j, M, HIDDEN) for j in range(R)]
+            by_s = (2 * HIDDEN * M + 2 * HIDDEN * r + 4 * M * r) / 1e9
+            by_e = (4 * M * r + 2 * r * HIDDEN + 2 * 2 * HIDDEN * M) / 1e9
+            t_det = _time_graph([lambda j=j: B.bi_lora_shrink(xs[j], A_l, t=t, split_k=8, stream=stream)
+                                 for j in range(R)], stream)
+            t_atom = _time_graph([lambda j=j: B.bi_ctrl_lora_shrink_atomic(xs[j], A_l, t=t, split_k=8, stream=stream)
+                                  for j in range(R)], stream)
+            t_uns = _time_graph([lambda j=j: B.bi_lora_shrink(xs[j], A_l, t=t, split_k=1, stream=stream)
+                                 for j in range(R)], stream)
+            t_exp = _time_graph([lambda j=j: B.bi_lora_expand(t, B_l, ys[j], stream=stream) for j in range(R)], stream)
+            table.append({"M": M, "shrink_gbs": round(by_s / (t_det / 1e3), 1),
+                          "shrink_frac": round(by_s / (t_det / 1e3) / peaks["hbm_gbs"], 3),
+                          "shrink_us": round(t_det * 1e3, 2), "atomic_us": round(t_atom * 1e3, 2),
+                          "unsplit_us": round(t_uns * 1e3, 2), "expand_gbs": round(by_e / (t_exp / 1e3), 1),
+                          "expand_frac": round(by_e / (t_exp / 1e3) / peaks["hbm_gbs"], 3)})
+            del xs, ys
+        emit({"op": "lora", "r": r, "K": HIDDEN, "N": HIDDEN, "split_k": 8, "rows": table})
+    # decode attention: prefixes of one packed cache of 128 requests
+    kv_len = inputs.kv_lengths(128)
+    indptr, T = inputs.kv_layout(kv_len, 256)
+    g = torch.Generator(device=device).manual_seed(5)
+    kc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    qa = torch.randn((128, 32, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    ip_d = torch.tensor(indptr, dtype=torch.int32, device=device)
+    ln_d = torch.tensor(kv_len, dtype=torch.int32, device=device)
+    table = []
+    for Bn in (1, 2, 4, 8, 16, 32, 64, 128):
+        Tn = int(indptr[Bn])
+        o = torch.empty((Bn, 32, 128), dtype=torch.bfloat16, device=device)
+        ws_bi = torch.empty(B.bi_decode_attn_workspace_size(Tn, 32), dtype=torch.uint8, device=device)
+        ws_ad = torch.empty(lib.bi_ctrl_decode_attn_adaptive_workspace_size(Tn, 32), dtype=torch.uint8, device=device)
+        q = qa[:Bn].contiguous()
+        by = (int(kv_len[:Bn].sum()) * 8 * 128 * 2 * 2 + Bn * 32 * 128 * 4) / 1e9
+        t_bi = _time_graph([lambda: B.bi_decode_attn(q, kc[:Tn], vc[:Tn], ip_d[:Bn + 1], ln_d[:Bn], out=o,
+                                                     workspace=ws_bi, stream=stream)], stream)
+        t_ad = _time_graph([lambda: B.bi_ctrl_decode_attn_adaptive(q, kc[:Tn], vc[:Tn], ip_d[:Bn + 1], ln_d[:Bn],
+                                                                   out=o, workspace=ws_ad, stream=stream)], stream)
+        table.append({"B": Bn, "kv_gb": round(by, 3), "bi_gbs": round(by / (t_bi / 1e3), 1),
+                      "adaptive_gbs": round(by / (t_ad / 1e3), 1), "bi_frac": round(by / (t_bi / 1e3) / peaks["hbm_gbs"], 3)})
+    emit({"op": "decode_attn", "Hq": 32, "Hkv": 8, "D": 128, "chunk": 256, "kv_lengths": "U[512,32768]", "rows": table})
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -654,12 +762,17 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-tax", action="store_true", help="skip the invariance-tax comparison")
+    ap.add_argument("--sweep", action="store_true",
+                    help="print per-op throughput across batch sizes (one GPU) instead of the benchmark line")
     ap.add_argument("--attn-batch", type=int, default=ATTN_BATCH,
                     help="decode requests in the step (smaller for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
 
+    if args.sweep:
+        run_sweep(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

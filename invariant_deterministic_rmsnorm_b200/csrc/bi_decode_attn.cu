@@ -407,19 +407,33 @@ decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restri
     const int64_t slot0 = sbase / CH;
     float m = -INFINITY, l = 0.0f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < nch; ++c) {
-        const int64_t idx = (slot0 + c) * Hq + h;
-        const float2 mlc = *reinterpret_cast<const float2*>(ml_part + idx * 2);
-        const float4 oc = *reinterpret_cast<const float4*>(o_part + idx * D + lane * 4);
-        const float mn = fmaxf(m, mlc.x);
-        const float a = expf(__fsub_rn(m, mn));   // 0 on the first chunk (m = -inf)
-        const float bsc = expf(__fsub_rn(mlc.x, mn));
-        l = __fmaf_rn(l, a, __fmul_rn(mlc.y, bsc));
-        o.x = __fmaf_rn(o.x, a, __fmul_rn(oc.x, bsc));
-        o.y = __fmaf_rn(o.y, a, __fmul_rn(oc.y, bsc));
-        o.z = __fmaf_rn(o.z, a, __fmul_rn(oc.z, bsc));
-        o.w = __fmaf_rn(o.w, a, __fmul_rn(oc.w, bsc));
-        m = mn;
+    // The merge is sequential in c; the loads are not.  Fetch PF chunks ahead, merge them in order.
+    constexpr int PF = 8;
+    for (int c0 = 0; c0 < nch; c0 += PF) {
+        float2 mlc[PF];
+        float4 oc[PF];
+#pragma unroll
+        for (int i = 0; i < PF; ++i) {
+            if (c0 + i < nch) {
+                const int64_t idx = (slot0 + c0 + i) * Hq + h;
+                mlc[i] = *reinterpret_cast<const float2*>(ml_part + idx * 2);
+                oc[i] = *reinterpret_cast<const float4*>(o_part + idx * D + lane * 4);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < PF; ++i) {
+            if (c0 + i < nch) {
+                const float mn = fmaxf(m, mlc[i].x);
+                const float a = expf(__fsub_rn(m, mn));   // 0 on the first chunk (m = -inf)
+                const float bsc = expf(__fsub_rn(mlc[i].x, mn));
+                l = __fmaf_rn(l, a, __fmul_rn(mlc[i].y, bsc));
+                o.x = __fmaf_rn(o.x, a, __fmul_rn(oc[i].x, bsc));
+                o.y = __fmaf_rn(o.y, a, __fmul_rn(oc[i].y, bsc));
+                o.z = __fmaf_rn(o.z, a, __fmul_rn(oc[i].z, bsc));
+                o.w = __fmaf_rn(o.w, a, __fmul_rn(oc[i].w, bsc));
+                m = mn;
+            }
+        }
     }
     const float r0 = __fdiv_rn(o.x, l), r1 = __fdiv_rn(o.y, l), r2 = __fdiv_rn(o.z, l), r3 = __fdiv_rn(o.w, l);
     const int64_t off = ((int64_t)b * Hq + h) * D + lane * 4;

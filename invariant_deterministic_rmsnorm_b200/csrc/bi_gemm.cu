@@ -32,23 +32,28 @@ using namespace bi::sm100;
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK = 64;
 constexpr int UMMA_K = 16;
-constexpr int STAGES = 4;
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 constexpr int B_BOX = 64 * BK * 2;    // 8 KB: 64 N-columns x 64 K-rows
-constexpr int B_STAGE = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
-constexpr int ACC_COLS = BN;          // one fp32 accumulator = 256 TMEM columns
-constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int THREADS = 192;
 constexpr int EPI_WARPS = 4;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+constexpr int MAX_STAGES = 8;
+
+// Tile geometry for a tile width BN (64, 128 or 256 output columns).
+template <int BN>
+struct Tile {
+    static constexpr int B_STAGE = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
+    static constexpr int STAGES = (196 * 1024) / STAGE_BYTES < MAX_STAGES ? (196 * 1024) / STAGE_BYTES : MAX_STAGES;
+    static constexpr int ACC_COLS = BN;  // one fp32 accumulator = BN TMEM columns
+    static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulators, a power of two
+    static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+};
 
 struct Bars {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
     uint64_t tfull[2];   // accumulator b holds a finished tile
     uint64_t tempty[2];  // accumulator b has been read out
     uint32_t tmem_addr;
@@ -73,9 +78,15 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
     n_tile = r / gsm;
 }
 
+template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
 bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                        void* __restrict__ C, int M, int N, int K, int c_bf16, int gm, uint32_t* err) {
+    constexpr int STAGES = Tile<BN>::STAGES;
+    constexpr int B_STAGE = Tile<BN>::B_STAGE;
+    constexpr int STAGE_BYTES = Tile<BN>::STAGE_BYTES;
+    constexpr int ACC_COLS = Tile<BN>::ACC_COLS;
+    constexpr int TMEM_COLS = Tile<BN>::TMEM_COLS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
@@ -257,25 +268,33 @@ int num_sms() {
     return cached[dev];
 }
 
+template <int BN>
 bool ensure_smem_attr() {
     static std::once_flag once[64];
     static bool ok[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::call_once(once[dev], [&] {
-        ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES) == cudaSuccess;
+        ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Tile<BN>::SMEM_BYTES) == cudaSuccess;
     });
     return ok[dev];
 }
 
+// The tile width for a weight of shape [K, N].  A function of (N, K) only, never of M, so every
+// batch size runs the same MMA shape and K order on every row.
+int plan_bn(int64_t N, int64_t K) {
+    (void)N; (void)K;
+    return 256;
+}
 
 // Launch the GEMM on operands with arbitrary (16-byte multiple) row strides: A [M, K] with
 // row stride lda, W [K, N] with row stride ldw, C [M, N] with row stride N.
-int launch_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N, int64_t K,
-                bool c_bf16, cudaStream_t stream) {
+template <int BN>
+int launch_gemm_bn(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N, int64_t K,
+                   bool c_bf16, cudaStream_t stream) {
     uint32_t* err = bi::device_error_word();
-    if (!err || !ensure_smem_attr()) return BI_ERR_CUDA;
+    if (!err || !ensure_smem_attr<BN>()) return BI_ERR_CUDA;
     CUtensorMap tmA, tmW;
     if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK,
                           BM, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -288,9 +307,18 @@ int launch_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C,
     if (sms <= 0) return BI_ERR_CUDA;
     const int gm = 16;  // ~16 row tiles x ~9 column tiles in flight: A and W blocks balanced within L2
     dim3 grid((unsigned)(tiles < sms ? tiles : sms));
-    bi_gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmW, C, (int)M, (int)N, (int)K,
-                                                                   c_bf16 ? 1 : 0, gm, err);
+    bi_gemm_bf16_tc_kernel<BN><<<grid, THREADS, Tile<BN>::SMEM_BYTES, stream>>>(tmA, tmW, C, (int)M, (int)N, (int)K,
+                                                                                 c_bf16 ? 1 : 0, gm, err);
     return bi::launch_status();
+}
+
+int launch_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N, int64_t K,
+                bool c_bf16, cudaStream_t stream) {
+    switch (plan_bn(N, K)) {
+        case 64: return launch_gemm_bn<64>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
+        case 128: return launch_gemm_bn<128>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
+        default: return launch_gemm_bn<256>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
+    }
 }
 
 int gemm_shape_checks(const void* A, const void* W, const void* C, int64_t M, int64_t N, int64_t K, int c_dtype) {
@@ -301,7 +329,7 @@ int gemm_shape_checks(const void* A, const void* W, const void* C, int64_t M, in
     if (!bi::aligned16(A) || !bi::aligned16(W) || !bi::aligned16(C)) return BI_ERR_MISALIGNED;
     if (K % 8 != 0 || N % 8 != 0) return BI_ERR_MISALIGNED;  // 16-byte row strides for the TMA unit
     if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return BI_ERR_UNSUPPORTED_SHAPE;
-    if (((M + BM - 1) / BM) * ((N + BN - 1) / BN) > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (((M + BM - 1) / BM) * ((N + 63) / 64) > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
     return BI_OK;
 }
 
@@ -330,7 +358,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, void* __res
 // The split a batch-size-adaptive library would pick: enough K slices to fill the GPU when
 // the batch alone yields too few output tiles (1, 2, 4 or 8, with K / S a multiple of 64).
 int splitk_for(int64_t M, int64_t N, int64_t K) {
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int bn = plan_bn(N, K);
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + bn - 1) / bn);
     const int sms = num_sms() > 0 ? num_sms() : 148;
     int S = 1;
     while (S < 8 && tiles * S * 2 <= sms && K % ((int64_t)S * 2 * BK) == 0) S *= 2;

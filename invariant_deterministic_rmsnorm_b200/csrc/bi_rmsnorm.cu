@@ -97,15 +97,20 @@ rmsnorm_rows_kernel(const TIO* __restrict__ x, const TW* __restrict__ w, TIO* __
     uint4 xv[VPT], xn[VPT];
     int64_t row = blockIdx.x;
     if (row >= M) return;
-    // the weights are the same for every row: when a thread's share is small, widen them to
-    // fp32 once per CTA and keep them in registers; otherwise re-read them (L1/L2) per row
+    // the weights are the same for every row: when a thread's share is small, keep their raw
+    // bits in registers for the CTA's lifetime (widened per use); otherwise re-read them per row
     constexpr bool kWInRegs = VPT * V <= 32;
-    float wr[kWInRegs ? VPT : 1][V];
+    constexpr int WWORDS = V * (int)sizeof(TW) / 4;  // 32-bit words of weights per vector
+    uint32_t wr[kWInRegs ? VPT : 1][WWORDS];
     if constexpr (kWInRegs) {
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int v = tid + i * nthreads;
-            if (v < nvec) load_w<TW, V>(w, (int64_t)v * V, wr[i]);
+            if (v < nvec) {
+                const uint32_t* src = reinterpret_cast<const uint32_t*>(w + (int64_t)v * V);
+#pragma unroll
+                for (int k = 0; k < WWORDS; ++k) wr[i][k] = __ldg(src + k);
+            }
         }
     }
 #pragma unroll
@@ -161,8 +166,16 @@ rmsnorm_rows_kernel(const TIO* __restrict__ x, const TW* __restrict__ w, TIO* __
                 float f[V], wf[V];
                 IoTraits<TIO>::unpack(xv[i], f);
                 if constexpr (kWInRegs) {
+                    if constexpr (sizeof(TW) == 4) {
 #pragma unroll
-                    for (int e = 0; e < V; ++e) wf[e] = wr[i][e];
+                        for (int e = 0; e < V; ++e) wf[e] = __uint_as_float(wr[i][e]);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < WWORDS; ++k) {
+                            wf[2 * k] = bi::bf16_lo(wr[i][k]);
+                            wf[2 * k + 1] = bi::bf16_hi(wr[i][k]);
+                        }
+                    }
                 } else {
                     load_w<TW, V>(w, (int64_t)v * V, wf);
                 }
