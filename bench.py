@@ -404,8 +404,15 @@ def run_ours(args, rank, world, local_rank):
         "bi_violations": viol,
         "invariance_tax": tax,
         "clocks": clocks, "cpu_baseline": cpu,
+        # what the result was produced with (GPU, driver, CUDA, torch, commit)
+        "pin": harness_pin(),
     }
     return line
+
+
+def harness_pin():
+    from invariant_deterministic_rmsnorm_b200 import harness
+    return harness.pin_tuple()
 
 
 L2_FLUSH_BYTES = 256 << 20  # twice the B200's 126 MB L2
@@ -622,10 +629,13 @@ def cpu_baseline(seconds: float):
     if dt < seconds * 0.5:
         rows = max(rows, int(rows * seconds * 0.7 / max(dt, 1e-3)) // threads * threads)
         flops, dt = _oracle_gemm_sample(rows, threads)
+    f1, d1 = _oracle_gemm_sample(1, 1)  # the same oracle on one core, one row per projection
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": f"GEMM: {rows} of the {M_TOKENS} token rows through each of the three projections "
                       f"(K,N) = {GEMM_SHAPES}, fp64 oracle, row ranges split over {threads} threads",
-            "seconds": round(dt, 3)}
+            "seconds": round(dt, 3),
+            "single_core": {"value": round(f1 / d1 / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+                            "sample": "1 token row through each projection", "seconds": round(d1, 3)}}
 
 
 def run_reference(args, rank, world):

@@ -408,7 +408,7 @@ decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restri
     float m = -INFINITY, l = 0.0f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     // The merge is sequential in c; the loads are not.  Fetch PF chunks ahead, merge them in order.
-    constexpr int PF = 8;
+    constexpr int PF = 16;
     for (int c0 = 0; c0 < nch; c0 += PF) {
         float2 mlc[PF];
         float4 oc[PF];

@@ -9,7 +9,7 @@
 // Launch plan, a function of (H, dtypes) only:
 //   vec     = 16 bytes / element size (8 bf16 or 4 fp32 elements per 128-bit load)
 //   nvec    = H / vec
-//   threads = nvec / 4 rounded up to a warp, clamped to [32, 256]
+//   threads = nvec / 2 rounded up to a warp, clamped to [32, 256]
 //   vpt     = ceil(nvec / threads) vectors per thread (compile-time 1, 2, 4, 8 or 16)
 // Thread t owns vectors t, t + threads, t + 2*threads, ...  It keeps them in
 // registers (one HBM read of x), sums their squares sequentially with fused
@@ -215,7 +215,7 @@ int launch_typed(const void* x, const void* w, void* y, int64_t M, int64_t H, in
                  cudaStream_t s) {
     constexpr int V = IoTraits<TIO>::kVec;
     const int nvec = (int)(H / V);
-    int threads = ((nvec / 4 + 31) / 32) * 32;  // about four 16-byte vectors per thread
+    int threads = ((nvec / 2 + 31) / 32) * 32;  // about two 16-byte vectors per thread
     if (threads < 32) threads = 32;
     if (threads > kMaxThreads) threads = kMaxThreads;
     const int vpt = (nvec + threads - 1) / threads;

@@ -116,12 +116,21 @@ def pin_tuple(extra: dict | None = None) -> dict:
             d["sm"] = f"{cap[0]}{cap[1]}"
     except Exception:  # pragma: no cover
         pass
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     try:
-        root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
         d["git"] = subprocess.run(["git", "-C", root, "rev-parse", "--short", "HEAD"], capture_output=True,
                                   text=True, timeout=5).stdout.strip() or None
     except Exception:  # pragma: no cover
         d["git"] = None
+    # the kernel sources themselves, for copies of the tree without version control
+    import glob
+    import hashlib
+    hsh = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(root, "invariant_deterministic_rmsnorm_b200", "csrc", "*")) +
+                    glob.glob(os.path.join(root, "include", "*.h"))):
+        with open(f, "rb") as fh:
+            hsh.update(fh.read())
+    d["kernel_sources_sha256"] = hsh.hexdigest()[:16]
     try:
         out = subprocess.run(["nvidia-smi", "--query-gpu=driver_version", "--format=csv,noheader"],
                              capture_output=True, text=True, timeout=10).stdout.strip().splitlines()
