@@ -125,3 +125,72 @@ M_SWEEP_ODD = [3, 5, 7, 15, 17, 31, 33, 63, 65, 127, 129, 255, 257, 511, 513, 10
 
 def m_sweep(max_m: int = 8192):
     return sorted(m for m in set(M_SWEEP_POW2 + M_SWEEP_ODD) if m <= max_m)
+
+
+# ------------------------------------------------------------------ decoder
+# A Llama-shaped decoder: RMSNorm -> fused QKV projection -> RoPE -> attention -> output
+# projection -> residual; RMSNorm -> fused gate/up projection -> SwiGLU -> down projection ->
+# residual; a final RMSNorm and the vocabulary projection.  Matrices ~ N(0, 0.02) (random
+# init: no trained weights are used); norm weights ~ N(1, 0.02); prompts are uniform token
+# ids, prompt lengths uniform integers in [16, 2048].
+SEED_PROMPT_LEN = 4
+SEED_PROMPT_BASE = 5000
+
+
+class DecoderShape:
+    """Dimensions of the decoder (defaults: 4 layers of Llama-3-8B, vocabulary 32000)."""
+
+    def __init__(self, hidden=4096, layers=4, q_heads=32, kv_heads=8, head_dim=128, ffn=14336, vocab=32000,
+                 eps=1e-5, theta=500000.0):
+        self.hidden, self.layers, self.q_heads, self.kv_heads = hidden, layers, q_heads, kv_heads
+        self.head_dim, self.ffn, self.vocab, self.eps, self.theta = head_dim, ffn, vocab, eps, theta
+
+    @property
+    def qkv_cols(self) -> int:
+        return (self.q_heads + 2 * self.kv_heads) * self.head_dim
+
+    def matrices(self):
+        """(name, rows, cols, mean, std) of every weight, in generation order."""
+        H, F, V = self.hidden, self.ffn, self.vocab
+        out = [("embed", V, H, 0.0, 0.02)]
+        for l in range(self.layers):
+            out += [(f"l{l}.attn_norm", 1, H, 1.0, 0.02), (f"l{l}.wqkv", H, self.qkv_cols, 0.0, 0.02),
+                    (f"l{l}.wo", self.q_heads * self.head_dim, H, 0.0, 0.02), (f"l{l}.mlp_norm", 1, H, 1.0, 0.02),
+                    (f"l{l}.wgu", H, 2 * F, 0.0, 0.02), (f"l{l}.wdown", F, H, 0.0, 0.02)]
+        out += [("final_norm", 1, H, 1.0, 0.02), ("lm_head", H, V, 0.0, 0.02)]
+        return out
+
+
+LLAMA3_8B_4L = DecoderShape()
+TINY_DECODER = DecoderShape(hidden=512, layers=2, q_heads=4, kv_heads=2, ffn=768, vocab=1000)
+
+
+def decoder_weights_host(shape: DecoderShape, seed: int = SEED_WEIGHTS) -> dict:
+    """Every weight as bf16 bits (numpy uint16), norm weights 1-D.  For small shapes (host numpy draws)."""
+    out = {}
+    for i, (name, r, c, mean, std) in enumerate(shape.matrices()):
+        w = normal_bf16(seed * 1000 + i, (r, c), mean, std)
+        out[name] = w[0] if r == 1 else w
+    return out
+
+
+def decoder_weights_device(shape: DecoderShape, seed: int = SEED_WEIGHTS, device="cuda") -> dict:
+    """Every weight as a bf16 torch tensor drawn on the device (seeded torch generator): the fast
+    route for full-size shapes, whose 1.1e9 draws would take minutes with numpy."""
+    import torch
+
+    g = torch.Generator(device=device).manual_seed(seed)
+    out = {}
+    for name, r, c, mean, std in shape.matrices():
+        w = (torch.randn((r, c), generator=g, device=device, dtype=torch.float32) * std + mean).to(torch.bfloat16)
+        out[name] = w[0].contiguous() if r == 1 else w
+    return out
+
+
+def prompt_lengths(n: int, lo: int = 16, hi: int = 2048, seed: int = SEED_PROMPT_LEN) -> np.ndarray:
+    return np.random.default_rng(seed).integers(lo, hi + 1, size=n).astype(np.int32)
+
+
+def prompt(index: int, length: int, vocab: int) -> np.ndarray:
+    """Token ids of prompt number `index` (uniform in [0, vocab))."""
+    return np.random.default_rng(SEED_PROMPT_BASE + index).integers(0, vocab, size=length).astype(np.int32)
