@@ -764,6 +764,39 @@ def run_sweep(args):
     emit({"op": "decode_attn", "Hq": 32, "Hkv": 8, "D": 128, "chunk": 256, "kv_lengths": "U[512,32768]", "rows": table})
 
 
+def run_replay_study(args):
+    """Identical-input replay of the split-K=8 LoRA shrink: the share of replays whose fp32 output
+    differs in any bit from the first replay, and the share of output elements that differ, for
+    the atomic combine and for the ordered combine ("Reproducible LoRA Inference Through
+    Deterministic Split-K Reduction", abstract: 97.61 % of atomic comparisons differed, none of
+    the deterministic ones)."""
+    import torch
+    from invariant_deterministic_rmsnorm_b200 import binding as B
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    n = args.replays
+    for r in (8, 16, 64):
+        A_l = _to_dev(inputs.normal_bf16(inputs.SEED_WEIGHTS + 20, (HIDDEN, r), 0.0, 0.02), device)
+        rows = []
+        for M in (1, 64, 1024, 4096):
+            x = _to_dev(inputs.rows(inputs.SEED_X, M, HIDDEN, "bf16"), device)
+            res = {"M": M}
+            for name, fn in (("atomic", B.bi_ctrl_lora_shrink_atomic), ("ordered", B.bi_lora_shrink)):
+                first = fn(x, A_l, split_k=8).clone()
+                diff_runs, diff_elems = 0, 0
+                for _ in range(n - 1):
+                    t = fn(x, A_l, split_k=8)
+                    ne = int((t.view(torch.int32) != first.view(torch.int32)).sum())
+                    diff_runs += int(ne > 0)
+                    diff_elems += ne
+                torch.cuda.synchronize()
+                res[f"{name}_replays_differing_pct"] = round(100.0 * diff_runs / (n - 1), 2)
+                res[f"{name}_elements_differing_pct"] = round(100.0 * diff_elems / ((n - 1) * M * r), 3)
+            rows.append(res)
+        print(json.dumps({"study": "lora_shrink_replay", "r": r, "K": HIDDEN, "split_k": 8, "replays": n,
+                          "rows": rows}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -772,6 +805,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-tax", action="store_true", help="skip the invariance-tax comparison")
+    ap.add_argument("--replay-study", action="store_true",
+                    help="identical-input replay study of the atomic vs ordered split-K shrink (one GPU)")
+    ap.add_argument("--replays", type=int, default=200)
     ap.add_argument("--sweep", action="store_true",
                     help="print per-op throughput across batch sizes (one GPU) instead of the benchmark line")
     ap.add_argument("--attn-batch", type=int, default=ATTN_BATCH,
@@ -782,6 +818,9 @@ def main():
 
     if args.sweep:
         run_sweep(args)
+        return
+    if args.replay_study:
+        run_replay_study(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -1,4 +1,4 @@
-"""Thin ctypes binding over libbi.so, with the same names as the C ABI (include/bi.h).
+"""Thin ctypes binding over libbi.so, with the same names as the C ABI (include/bi.h, include/bi_model.h).
 
 Argument marshalling only: every step of every op runs in the library's CUDA
 kernels.  Tensors are torch CUDA tensors; PyTorch provides device memory and
@@ -65,6 +65,14 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_ctrl_gemm_splitk": ([P, P, P, I64, I64, I64, C, P, Z, P], C),
         "bi_ctrl_decode_attn_adaptive_workspace_size": ([I64, I32], Z),
         "bi_ctrl_decode_attn_adaptive": ([P, P, P, P, P, I32, I64, I32, I32, F, P, C, P, Z, P], C),
+        # include/bi_model.h
+        "bi_embed": ([P, P, P, I64, I64, I64, P], C),
+        "bi_rope": ([P, I64, I64, I32, I32, P, ctypes.c_double, P], C),
+        "bi_kv_append": ([P, I64, P, P, I64, I64, I64, P], C),
+        "bi_add": ([P, I64, P, I64, I64, I64, P], C),
+        "bi_swiglu": ([P, I64, P, I64, I64, I64, P], C),
+        "bi_argmax": ([P, I64, I64, I64, P, P], C),
+        "bi_prefill_attn": ([P, I64, I64, P, P, I64, P, P, I32, P, P, I32, I32, I32, I32, F, P, I64, P], C),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -236,6 +244,141 @@ def bi_decode_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kv_indptr:
                             float(scale), chunk, _ptr(out), _dtype_code(out), _ptr(workspace),
                             workspace.numel() * workspace.element_size(), _stream(stream))
     _check("bi_decode_attn", st)
+    return out
+
+
+# ------------------------------------------------------------------ decoder ops (include/bi_model.h)
+def _i32(t: torch.Tensor, name: str) -> None:
+    if t.dtype != torch.int32 or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+
+
+def _bf16_rows(t: torch.Tensor, name: str) -> None:
+    _rows(t, name)
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bf16")
+
+
+def bi_embed(tokens: torch.Tensor, table: torch.Tensor, out: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    """out[t] = table[tokens[t]] (bf16 rows)."""
+    _i32(tokens, "tokens")
+    _bf16_2d(table, "table")
+    vocab, H = table.shape
+    T = tokens.numel()
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=table.device)
+    if not out.is_contiguous() or tuple(out.shape) != (T, H):
+        raise ValueError("out must be a contiguous [T, H] tensor")
+    _check("bi_embed", library().bi_embed(_ptr(tokens), _ptr(table), _ptr(out), T, H, vocab, _stream(stream)))
+    return out
+
+
+def bi_rope(x: torch.Tensor, pos: torch.Tensor, heads: int, head_dim: int = 128, theta: float = 500000.0,
+            stream=None) -> torch.Tensor:
+    """Rotary embedding in place on the first heads*head_dim columns of each row of x (bf16)."""
+    _bf16_rows(x, "x")
+    _i32(pos, "pos")
+    T = x.shape[0]
+    if pos.numel() != T or x.shape[1] < heads * head_dim:
+        raise ValueError("shape mismatch")
+    _check("bi_rope", library().bi_rope(_ptr(x), T, x.stride(0), heads, head_dim, _ptr(pos), float(theta),
+                                        _stream(stream)))
+    return x
+
+
+def bi_kv_append(src: torch.Tensor, dst_row: torch.Tensor, dst: torch.Tensor, stream=None) -> torch.Tensor:
+    """dst[dst_row[t], :] = src[t, :dst.shape[1]] (bf16; dst is a contiguous [rows, E] cache view)."""
+    _bf16_rows(src, "src")
+    _i32(dst_row, "dst_row")
+    if dst.dtype != torch.bfloat16 or not dst.is_contiguous():
+        raise ValueError("dst must be a contiguous bf16 tensor")
+    d2 = dst.view(dst.shape[0], -1)
+    T, E = src.shape[0], d2.shape[1]
+    if dst_row.numel() != T or src.shape[1] < E:
+        raise ValueError("shape mismatch")
+    _check("bi_kv_append", library().bi_kv_append(_ptr(src), src.stride(0), _ptr(dst_row), _ptr(dst), T, E,
+                                                  d2.shape[0], _stream(stream)))
+    return dst
+
+
+def bi_add(h: torch.Tensor, d: torch.Tensor, stream=None) -> torch.Tensor:
+    """h += d in place (bf16 rows, one rounding per element)."""
+    _bf16_rows(h, "h")
+    _bf16_rows(d, "d")
+    if h.shape != d.shape:
+        raise ValueError("shape mismatch")
+    T, N = h.shape
+    _check("bi_add", library().bi_add(_ptr(h), h.stride(0), _ptr(d), d.stride(0), T, N, _stream(stream)))
+    return h
+
+
+def bi_swiglu(gu: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out = silu(gu[:, :N]) * gu[:, N:] with N = gu.shape[1] / 2 (bf16)."""
+    _bf16_rows(gu, "gu")
+    T, N2 = gu.shape
+    if N2 % 2:
+        raise ValueError("gu must have an even number of columns")
+    N = N2 // 2
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=gu.device)
+    _bf16_rows(out, "out")
+    _check("bi_swiglu", library().bi_swiglu(_ptr(gu), gu.stride(0), _ptr(out), out.stride(0), T, N,
+                                            _stream(stream)))
+    return out
+
+
+def bi_argmax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Row-wise argmax of fp32 x (smallest index on ties) -> int32 [T]."""
+    _rows(x, "x")
+    if x.dtype != torch.float32:
+        raise ValueError("x must be fp32")
+    T, N = x.shape
+    if out is None:
+        out = torch.empty((T,), dtype=torch.int32, device=x.device)
+    _i32(out, "out")
+    _check("bi_argmax", library().bi_argmax(_ptr(x), x.stride(0), T, N, _ptr(out), _stream(stream)))
+    return out
+
+
+def prefill_tiles(q_lens) -> list:
+    """q_tile_indptr for query lengths q_lens: prefix sums of ceil(len / 64)."""
+    out = [0]
+    for n in q_lens:
+        out.append(out[-1] + (int(n) + 63) // 64)
+    return out
+
+
+def bi_prefill_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, q_indptr: torch.Tensor,
+                    q_tile_indptr: torch.Tensor, n_tiles: int, kv_indptr: torch.Tensor, q_pos0: torch.Tensor,
+                    Hq: int, out: torch.Tensor | None = None, scale: float | None = None,
+                    stream=None) -> torch.Tensor:
+    """Causal prefill attention.  q: bf16 rows [q_rows, >= Hq*128] (any row stride); k_cache, v_cache:
+    bf16 [T, Hkv, 128] packed; int32 index arrays as include/bi_model.h describes; out: bf16
+    [q_rows, >= Hq*128] (allocated when None)."""
+    _bf16_rows(q, "q")
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{n} must be a contiguous 3-D bf16 tensor")
+    for t, n in ((q_indptr, "q_indptr"), (q_tile_indptr, "q_tile_indptr"), (kv_indptr, "kv_indptr"),
+                 (q_pos0, "q_pos0")):
+        _i32(t, n)
+    B = q_pos0.numel()
+    if q_indptr.numel() != B + 1 or q_tile_indptr.numel() != B + 1 or kv_indptr.numel() < B:
+        raise ValueError("index arrays do not match the number of sequences")
+    T, Hkv, D = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache and v_cache differ in shape")
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty((q.shape[0], Hq * D), dtype=torch.bfloat16, device=q.device)
+    _bf16_rows(out, "out")
+    st = library().bi_prefill_attn(_ptr(q), q.stride(0), q.shape[0], _ptr(k_cache), _ptr(v_cache), T,
+                                   _ptr(q_indptr), _ptr(q_tile_indptr), int(n_tiles), _ptr(kv_indptr),
+                                   _ptr(q_pos0), B, Hq, Hkv, D, float(scale), _ptr(out), out.stride(0),
+                                   _stream(stream))
+    _check("bi_prefill_attn", st)
     return out
 
 

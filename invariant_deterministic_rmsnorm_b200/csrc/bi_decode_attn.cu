@@ -45,7 +45,7 @@ constexpr int BOX_BYTES = BOX_TOK * 64 * 2;  // 64 tokens x 64 dims (one 128-byt
 constexpr int STAGE_BYTES = SUB * D * 2;     // 32 KB
 constexpr int NSTAGES = 3;
 
-constexpr uint32_t DEVERR_BAD_LAYOUT = 1u << 8;  // kv_indptr / kv_len violate the documented layout
+using bi::DEVERR_BAD_LAYOUT;
 
 constexpr int P_PITCH = CHUNK + 8;  // bf16 per head row of the split probabilities (+8: no bank conflicts)
 

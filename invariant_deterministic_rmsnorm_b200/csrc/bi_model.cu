@@ -1,0 +1,214 @@
+// bi_model.cu -- the row-wise model ops a decoder needs around the hot-path kernels:
+// embedding gather, rotary position embedding, KV-cache append, residual add, SwiGLU, argmax.
+//
+// Every op here works on one token row at a time, with no reduction across rows.  An
+// output row's bits therefore depend only on that row's inputs, and its position (for
+// RoPE), whatever the batch.  Source for why that matters: "Defeating Nondeterminism in
+// LLM Inference" (Spanish summary), "La verdadera causa clave".  The batch size changes
+// from request to request, so every kernel must give each row the same bits at any batch
+// size.
+#include <math.h>
+
+#include "bi_common.cuh"
+#include "bi_model.h"
+
+namespace {
+
+// ------------------------------------------------------------------ embedding gather
+__global__ void embed_kernel(const int32_t* __restrict__ tokens, const __nv_bfloat16* __restrict__ table,
+                             __nv_bfloat16* __restrict__ out, int64_t H, int64_t vocab, uint32_t* err) {
+    const int64_t t = blockIdx.x;
+    const int32_t id = tokens[t];
+    if (id < 0 || id >= vocab) {
+        if (threadIdx.x == 0) atomicOr(err, bi::DEVERR_BAD_TOKEN);  // token id out of range: row left unwritten
+        return;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(table + (int64_t)id * H);
+    uint4* dst = reinterpret_cast<uint4*>(out + t * H);
+    for (int64_t i = threadIdx.x; i < H / 8; i += blockDim.x) dst[i] = src[i];
+}
+
+// ------------------------------------------------------------------ rotary position embedding
+// For each head row of D dims and pair index i < D/2: angle = pos * theta^(-2i/D), computed in
+// double precision; (x_i, x_{i+D/2}) -> (x_i cos - x_{i+D/2} sin, x_{i+D/2} cos + x_i sin) in fp32,
+// rounded once to bf16 (the "rotate half" pairing of Llama).
+__global__ void rope_kernel(__nv_bfloat16* __restrict__ x, int64_t ld_row, int heads, int D,
+                            const int32_t* __restrict__ pos, double log_theta) {
+    const int64_t t = blockIdx.x;
+    const int half = D / 2;
+    const double p = (double)pos[t];
+    __nv_bfloat16* row = x + t * ld_row;
+    for (int i = threadIdx.x; i < half; i += blockDim.x) {
+        // the angle depends on (position, pair) only: one double-precision sincos, used by every head
+        const double ang = p * exp(-log_theta * (2.0 * i) / (double)D);
+        double sd, cd;
+        sincos(ang, &sd, &cd);
+        const float s = (float)sd, c = (float)cd;
+        for (int h = 0; h < heads; ++h) {
+            __nv_bfloat16* hp = row + (int64_t)h * D;
+            const float a = __bfloat162float(hp[i]);
+            const float b = __bfloat162float(hp[i + half]);
+            hp[i] = __float2bfloat16_rn(__fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s)));
+            hp[i + half] = __float2bfloat16_rn(__fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s)));
+        }
+    }
+}
+
+// ------------------------------------------------------------------ KV append
+// dst[dst_row[t], :] = src[t, :] for one packed row of `row_elems` bf16 (all kv heads of a token).
+__global__ void kv_append_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src,
+                                 const int32_t* __restrict__ dst_row, __nv_bfloat16* __restrict__ dst,
+                                 int64_t row_elems, int64_t dst_rows, uint32_t* err) {
+    const int64_t t = blockIdx.x;
+    const int64_t r = dst_row[t];
+    if (r < 0 || r >= dst_rows) {
+        if (threadIdx.x == 0) atomicOr(err, bi::DEVERR_BAD_DST_ROW);  // destination row out of range: skipped
+        return;
+    }
+    const uint4* s = reinterpret_cast<const uint4*>(src + t * ld_src);
+    uint4* d = reinterpret_cast<uint4*>(dst + r * row_elems);
+    for (int64_t i = threadIdx.x; i < row_elems / 8; i += blockDim.x) d[i] = s[i];
+}
+
+// ------------------------------------------------------------------ residual add (in place)
+__global__ void add_kernel(__nv_bfloat16* __restrict__ h, int64_t ldh, const __nv_bfloat16* __restrict__ d,
+                           int64_t ldd, int64_t N) {
+    const int64_t t = blockIdx.x;
+    for (int64_t i = threadIdx.x; i < N / 8; i += blockDim.x) {
+        uint4* hp = reinterpret_cast<uint4*>(h + t * ldh) + i;
+        const uint4 a = *hp;
+        const uint4 b = *(reinterpret_cast<const uint4*>(d + t * ldd) + i);
+        uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            av[j] = bi::pack_bf16x2(__fadd_rn(bi::bf16_lo(av[j]), bi::bf16_lo(bv[j])),
+                                    __fadd_rn(bi::bf16_hi(av[j]), bi::bf16_hi(bv[j])));
+        *hp = make_uint4(av[0], av[1], av[2], av[3]);
+    }
+}
+
+// ------------------------------------------------------------------ SwiGLU
+// out[t, j] = silu(gu[t, j]) * gu[t, N + j] with silu(g) = g / (1 + e^-g), fp32, rounded once.
+__global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ gu, int64_t ld_gu, __nv_bfloat16* __restrict__ out,
+                              int64_t ld_out, int64_t N) {
+    const int64_t t = blockIdx.x;
+    for (int64_t i = threadIdx.x; i < N / 8; i += blockDim.x) {
+        const uint4 g = *(reinterpret_cast<const uint4*>(gu + t * ld_gu) + i);
+        const uint4 u = *(reinterpret_cast<const uint4*>(gu + t * ld_gu + N) + i);
+        uint32_t gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w}, ov[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float g0 = bi::bf16_lo(gv[j]), g1 = bi::bf16_hi(gv[j]);
+            const float s0 = __fdiv_rn(g0, __fadd_rn(1.0f, expf(-g0)));
+            const float s1 = __fdiv_rn(g1, __fadd_rn(1.0f, expf(-g1)));
+            ov[j] = bi::pack_bf16x2(__fmul_rn(s0, bi::bf16_lo(uv[j])), __fmul_rn(s1, bi::bf16_hi(uv[j])));
+        }
+        *(reinterpret_cast<uint4*>(out + t * ld_out) + i) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+    }
+}
+
+// ------------------------------------------------------------------ argmax
+// The index of the largest fp32 value of each row; among equal values the smallest index.
+// NaN compares as smaller than everything.  One CTA per row, a fixed tree.
+__global__ void __launch_bounds__(256) argmax_kernel(const float* __restrict__ x, int64_t ld, int64_t N,
+                                                     int32_t* __restrict__ out) {
+    __shared__ float sv[256];
+    __shared__ int32_t si[256];
+    const int64_t t = blockIdx.x;
+    float best = -INFINITY;
+    int32_t bi_ = 0x7fffffff;
+    for (int64_t i = threadIdx.x; i < N; i += blockDim.x) {
+        const float v = x[t * ld + i];
+        if (v > best || (v == best && (int32_t)i < bi_)) {
+            best = v;
+            bi_ = (int32_t)i;
+        }
+    }
+    sv[threadIdx.x] = best;
+    si[threadIdx.x] = bi_;
+    __syncthreads();
+    for (int off = 128; off > 0; off >>= 1) {
+        if ((int)threadIdx.x < off) {
+            const float v = sv[threadIdx.x + off];
+            const int32_t j = si[threadIdx.x + off];
+            if (v > sv[threadIdx.x] || (v == sv[threadIdx.x] && j < si[threadIdx.x])) {
+                sv[threadIdx.x] = v;
+                si[threadIdx.x] = j;
+            }
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) out[t] = si[0] == 0x7fffffff ? 0 : si[0];
+}
+
+int rows_ok(int64_t rows) { return rows >= 0 && rows <= 0x7fffffffLL; }
+
+}  // namespace
+
+BI_API int bi_embed(const int32_t* tokens, const void* table, void* out, int64_t T, int64_t H, int64_t vocab,
+                    void* stream) {
+    if (T < 0 || H <= 0 || vocab <= 0 || !rows_ok(T)) return BI_ERR_INVALID_ARG;
+    if (T == 0) return BI_OK;
+    if (!tokens || !table || !out) return BI_ERR_INVALID_ARG;
+    if (H % 8 != 0 || !bi::aligned16(table) || !bi::aligned16(out)) return BI_ERR_MISALIGNED;
+    uint32_t* err = bi::device_error_word();
+    if (!err) return BI_ERR_CUDA;
+    embed_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(tokens, static_cast<const __nv_bfloat16*>(table),
+                                                                 static_cast<__nv_bfloat16*>(out), H, vocab, err);
+    return bi::launch_status();
+}
+
+BI_API int bi_rope(void* x, int64_t T, int64_t ld_row, int32_t heads, int32_t head_dim, const int32_t* pos,
+                   double theta, void* stream) {
+    if (T < 0 || heads <= 0 || head_dim <= 0 || head_dim % 2 != 0 || !(theta > 1.0) || !rows_ok(T))
+        return BI_ERR_INVALID_ARG;
+    if (ld_row < (int64_t)heads * head_dim) return BI_ERR_INVALID_ARG;
+    if (T == 0) return BI_OK;
+    if (!x || !pos) return BI_ERR_INVALID_ARG;
+    rope_kernel<<<(unsigned)T, 64, 0, bi::as_stream(stream)>>>(static_cast<__nv_bfloat16*>(x), ld_row, heads,
+                                                                head_dim, pos, log(theta));
+    return bi::launch_status();
+}
+
+BI_API int bi_kv_append(const void* src, int64_t ld_src, const int32_t* dst_row, void* dst, int64_t T,
+                        int64_t row_elems, int64_t dst_rows, void* stream) {
+    if (T < 0 || row_elems <= 0 || dst_rows < 0 || ld_src < row_elems || !rows_ok(T)) return BI_ERR_INVALID_ARG;
+    if (T == 0) return BI_OK;
+    if (!src || !dst_row || !dst) return BI_ERR_INVALID_ARG;
+    if (row_elems % 8 != 0 || ld_src % 8 != 0 || !bi::aligned16(src) || !bi::aligned16(dst)) return BI_ERR_MISALIGNED;
+    uint32_t* err = bi::device_error_word();
+    if (!err) return BI_ERR_CUDA;
+    kv_append_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(src), ld_src,
+                                                                     dst_row, static_cast<__nv_bfloat16*>(dst),
+                                                                     row_elems, dst_rows, err);
+    return bi::launch_status();
+}
+
+BI_API int bi_add(void* h, int64_t ldh, const void* d, int64_t ldd, int64_t T, int64_t N, void* stream) {
+    if (T < 0 || N <= 0 || ldh < N || ldd < N || !rows_ok(T)) return BI_ERR_INVALID_ARG;
+    if (T == 0) return BI_OK;
+    if (!h || !d) return BI_ERR_INVALID_ARG;
+    if (N % 8 != 0 || ldh % 8 != 0 || ldd % 8 != 0 || !bi::aligned16(h) || !bi::aligned16(d)) return BI_ERR_MISALIGNED;
+    add_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(static_cast<__nv_bfloat16*>(h), ldh,
+                                                                static_cast<const __nv_bfloat16*>(d), ldd, N);
+    return bi::launch_status();
+}
+
+BI_API int bi_swiglu(const void* gu, int64_t ld_gu, void* out, int64_t ld_out, int64_t T, int64_t N, void* stream) {
+    if (T < 0 || N <= 0 || ld_gu < 2 * N || ld_out < N || !rows_ok(T)) return BI_ERR_INVALID_ARG;
+    if (T == 0) return BI_OK;
+    if (!gu || !out) return BI_ERR_INVALID_ARG;
+    if (N % 8 != 0 || ld_gu % 8 != 0 || ld_out % 8 != 0 || !bi::aligned16(gu) || !bi::aligned16(out))
+        return BI_ERR_MISALIGNED;
+    swiglu_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(gu), ld_gu,
+                                                                   static_cast<__nv_bfloat16*>(out), ld_out, N);
+    return bi::launch_status();
+}
+
+BI_API int bi_argmax(const float* x, int64_t ld, int64_t T, int64_t N, int32_t* out, void* stream) {
+    if (T < 0 || N <= 0 || ld < N || !rows_ok(T) || N > 0x7fffffffLL) return BI_ERR_INVALID_ARG;
+    if (T == 0) return BI_OK;
+    if (!x || !out) return BI_ERR_INVALID_ARG;
+    argmax_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(x, ld, N, out);
+    return bi::launch_status();
+}

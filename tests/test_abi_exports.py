@@ -69,3 +69,36 @@ def test_rmsnorm_host_checks(lib):
     assert _rms(lib, a, a, a, 4, 256, ldx=258) == 3        # row stride not 16-byte aligned
     assert _rms(lib, a, a, a, 4, 1 << 16) == 2             # H beyond the in-register plan
     assert _rms(lib, a, a, a, 4, 256, ldy=260) == 1        # in place with a different row stride
+
+
+def test_model_ops_host_checks(lib):
+    P = ctypes.c_void_p
+    a = 1 << 20
+    s = None
+    # embed: empty, bad sizes, misaligned rows
+    assert lib.bi_embed(P(a), P(a), P(a), 0, 4096, 32000, s) == 0
+    assert lib.bi_embed(P(a), P(a), P(a), 4, 0, 32000, s) == 1
+    assert lib.bi_embed(P(a), P(a), P(a), 4, 4100, 32000, s) == 3
+    # rope: odd head_dim, theta <= 1
+    assert lib.bi_rope(P(a), 4, 4096, 32, 127, P(a), 500000.0, s) == 1
+    assert lib.bi_rope(P(a), 4, 4096, 32, 128, P(a), 1.0, s) == 1
+    assert lib.bi_rope(P(a), 0, 4096, 32, 128, P(a), 500000.0, s) == 0
+    # kv append: source stride shorter than a row, misaligned row
+    assert lib.bi_kv_append(P(a), 512, P(a), P(a), 4, 1024, 100, s) == 1
+    assert lib.bi_kv_append(P(a), 1028, P(a), P(a), 4, 1028, 100, s) == 3
+    # add / swiglu: strides
+    assert lib.bi_add(P(a), 8, P(a), 16, 4, 16, s) == 1
+    assert lib.bi_swiglu(P(a), 16, P(a), 16, 4, 16, s) == 1     # ld_gu < 2N
+    assert lib.bi_swiglu(P(a), 36, P(a), 18, 4, 18, s) == 3     # N not a multiple of 8
+    assert lib.bi_argmax(P(a), 10, 4, 20, P(a), s) == 1         # ld < N
+    # prefill attention: head_dim, grouping, empty batch, alignment, strides
+    args = lambda **kw: [P(kw.get("q", a)), kw.get("ldq", 4096), 64, P(a), P(a), 1024, P(a), P(a),
+                         kw.get("tiles", 1), P(a), P(a), kw.get("B", 1), kw.get("Hq", 32), kw.get("Hkv", 8),
+                         kw.get("D", 128), 0.088, P(a), kw.get("ldo", 4096), s]
+    assert lib.bi_prefill_attn(*args(D=64)) == 2
+    assert lib.bi_prefill_attn(*args(Hkv=5)) == 1
+    assert lib.bi_prefill_attn(*args(B=0)) == 0
+    assert lib.bi_prefill_attn(*args(tiles=0)) == 0
+    assert lib.bi_prefill_attn(*args(q=a + 2)) == 3
+    assert lib.bi_prefill_attn(*args(ldq=4100)) == 3
+    assert lib.bi_prefill_attn(*args(ldo=2048)) == 1
