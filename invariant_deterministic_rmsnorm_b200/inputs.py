@@ -165,10 +165,16 @@ LLAMA3_8B_4L = DecoderShape()
 TINY_DECODER = DecoderShape(hidden=512, layers=2, q_heads=4, kv_heads=2, ffn=768, vocab=1000)
 
 
-def decoder_weights_host(shape: DecoderShape, seed: int = SEED_WEIGHTS) -> dict:
-    """Every weight as bf16 bits (numpy uint16), norm weights 1-D.  For small shapes (host numpy draws)."""
+def decoder_weights_host(shape: DecoderShape, seed: int = SEED_WEIGHTS, matrix_std: float | None = None,
+                         norm_std: float | None = None) -> dict:
+    """Every weight as bf16 bits (numpy uint16), norm weights 1-D.  For small shapes (host numpy draws).
+    matrix_std / norm_std override the spreads of the matrices / the norm weights."""
     out = {}
     for i, (name, r, c, mean, std) in enumerate(shape.matrices()):
+        if mean == 0.0 and matrix_std is not None:
+            std = matrix_std
+        if mean != 0.0 and norm_std is not None:
+            std = norm_std
         w = normal_bf16(seed * 1000 + i, (r, c), mean, std)
         out[name] = w[0] if r == 1 else w
     return out

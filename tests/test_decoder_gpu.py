@@ -11,7 +11,8 @@ import pytest
 import torch
 
 from oracle import decoder as od
-from gpu_util import dev, rel_frobenius
+import decoder_case as case
+from gpu_util import dev
 from invariant_deterministic_rmsnorm_b200 import inputs
 from invariant_deterministic_rmsnorm_b200.decoder import Decoder
 
@@ -20,31 +21,24 @@ pytestmark = pytest.mark.gpu
 
 # ------------------------------------------------------------------ parity (small shape)
 @pytest.mark.parametrize("mode", ["split", "prefill"])
-def test_tiny_decoder_matches_the_oracle(mode):
-    shape = inputs.TINY_DECODER
-    wh = inputs.decoder_weights_host(shape)
+def test_small_decoder_matches_the_oracle(mode):
+    """tests/decoder_case.py gives the workload and the derivation of TOL."""
+    wh = case.weights()
     wd = {k: dev(v) for k, v in wh.items()}
-    lens = [1, 37, 64, 65, 130]
-    slots = [0, 2, 3, 4, 5]
-    prompts = [inputs.prompt(i, n, shape.vocab) for i, n in enumerate(lens)]
-    gpu = Decoder(shape, wd, max_seqs=6, max_len=140, decode_attention=mode)
-    orc = od.OracleDecoder(shape, wh, 6, gpu.cap)
-    # teacher-forced decode tokens (seeded), so that both sides see the same inputs
-    forced = np.random.default_rng(60).integers(0, shape.vocab, (3, len(lens))).astype(np.int32)
-    steps = [(prompts, "prefill")] + [([[int(t)] for t in row], "decode") for row in forced]
+    gpu = Decoder(case.SHAPE, wd, max_seqs=case.MAX_SEQS, max_len=case.CAP, decode_attention=mode)
+    orc = od.OracleDecoder(case.SHAPE, wh, case.MAX_SEQS, gpu.cap)
     worst = 0.0
-    for toks, phase in steps:
-        g = gpu.forward(slots, toks, phase).cpu().numpy().astype(np.float64)
-        r = orc.forward(slots, toks)
-        for b in range(len(slots)):
-            e = rel_frobenius(g[b], r[b])
-            worst = max(worst, e)
-            assert e <= 2e-3, (phase, b, e)
+    for toks, phase in case.steps():
+        g = gpu.forward(case.SLOTS, toks, phase).cpu().numpy()
+        r = orc.forward(case.SLOTS, toks)
+        errs = case.rel_errors(g, r)
+        worst = max(worst, max(errs))
+        assert max(errs) <= case.TOL, (phase, errs)
         # greedy choice: equal wherever the oracle's top two logits are clearly apart
         top2 = np.sort(r, axis=1)[:, -2:]
-        clear = (top2[:, 1] - top2[:, 0]) > 1e-3 * np.abs(r).max()
+        clear = (top2[:, 1] - top2[:, 0]) > 0.05 * np.abs(r).max()
         assert np.array_equal(np.argmax(g, 1)[clear], od.argmax(r)[clear])
-    print(f"tiny decoder ({mode}): worst per-sequence relative Frobenius error of the logits {worst:.2e}")
+    print(f"small decoder ({mode}): worst relative Frobenius error of the logits {worst:.2e}")
 
 
 # ------------------------------------------------------------------ the batch-invariance gate
