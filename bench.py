@@ -797,6 +797,83 @@ def run_replay_study(args):
                           "rows": rows}), flush=True)
 
 
+def _decoder_flops(shape, lens_new, lens_total):
+    """Model FLOPs of one step: 2 per weight per new token for every projection, plus causal
+    attention (QK^T and PV, 4 * head_dim per query head per visible key).  The prefill kernel
+    multiplies P by V twice (bf16 high and low parts); that doubling is not counted."""
+    H, F, V = shape.hidden, shape.ffn, shape.vocab
+    per_layer = H * shape.qkv_cols + shape.q_heads * shape.head_dim * H + H * 2 * F + F * H
+    T = int(np.sum(lens_new))
+    proj = 2.0 * T * per_layer * shape.layers + 2.0 * len(lens_new) * H * V
+    keys = 0.0
+    for n, L in zip(lens_new, lens_total):
+        keys += sum(range(int(L) - int(n) + 1, int(L) + 1))  # row i sees L - n + 1 + i keys
+    attn = 4.0 * shape.head_dim * shape.q_heads * shape.layers * keys
+    return proj, attn
+
+
+def run_decoder(args):
+    """The 4-layer Llama-3-8B-shaped decoder built from the batch-invariant kernels: prefill
+    throughput, and greedy decode steps replayed from a CUDA graph, at several batch sizes.
+    Prints one JSON object per phase (one GPU)."""
+    import torch
+    from invariant_deterministic_rmsnorm_b200.decoder import Decoder
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    peaks, _ = load_peaks()
+    shape = inputs.LLAMA3_8B_4L
+    w = inputs.decoder_weights_device(shape, device=device)
+    steps = max(1, args.steps)
+    n_max = max(args.decoder_batches)
+    dec = Decoder(shape, w, max_seqs=n_max, max_len=2048 + 2 * steps + 8 + args.warmup)
+    all_lens = inputs.prompt_lengths(n_max)
+    prompts = [inputs.prompt(i, int(n), shape.vocab) for i, n in enumerate(all_lens)]
+    weight_bytes = 2 * sum(r * c for name, r, c, _, _ in shape.matrices() if name != "embed")
+    kv_row_bytes = 2 * 2 * shape.kv_heads * shape.head_dim * shape.layers  # K and V, all layers
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for B in args.decoder_batches:
+        slots, lens = list(range(B)), all_lens[:B]
+        # prefill (the first pass also does the per-device set-up; time the second)
+        prefill_ms = []
+        for _ in range(2):
+            dec.reset()
+            torch.cuda.synchronize()
+            e0, e1 = ev(), ev()
+            e0.record()
+            dec.forward(slots, prompts[:B], "prefill")
+            e1.record()
+            torch.cuda.synchronize()
+            prefill_ms.append(e0.elapsed_time(e1))
+        T = int(lens.sum())
+        proj, attn = _decoder_flops(shape, lens, lens)
+        ms = prefill_ms[-1]
+        print(json.dumps({"phase": "prefill", "requests": B, "tokens": T, "ms": round(ms, 2),
+                          "tokens_per_s": round(T / ms * 1e3), "model_tflops": round((proj + attn) / ms / 1e9, 1),
+                          "frac_of_bf16_peak": round((proj + attn) / ms / 1e9 / peaks["bf16_tflops"], 3),
+                          "attn_share_of_flops": round(attn / (proj + attn), 3)}), flush=True)
+        # decode: greedy steps replayed from one graph; the timed replays follow `warmup` untimed ones
+        g = dec.decode_graph(slots)
+        for _ in range(args.warmup):
+            g.replay()
+        ctx = dec.length[slots].copy()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for _ in range(steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        kv_read = kv_row_bytes * float(np.sum(ctx + 0.5 * (steps + 1)))  # mean context over the timed steps
+        step_bytes = weight_bytes + B * 2 * shape.hidden + kv_read
+        print(json.dumps({"phase": "decode", "requests": B, "steps": steps, "ms_per_step": round(ms, 4),
+                          "tokens_per_s": round(B / ms * 1e3), "mean_context": round(float(np.mean(ctx)) + steps / 2, 1),
+                          "hbm_gbs": round(step_bytes / ms / 1e6, 1),
+                          "frac_of_hbm": round(step_bytes / ms / 1e6 / peaks["hbm_gbs"], 3),
+                          "bytes_per_step": int(step_bytes)}), flush=True)
+        del g
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -812,6 +889,9 @@ def main():
                     help="print per-op throughput across batch sizes (one GPU) instead of the benchmark line")
     ap.add_argument("--attn-batch", type=int, default=ATTN_BATCH,
                     help="decode requests in the step (smaller for profiler captures)")
+    ap.add_argument("--decoder", action="store_true",
+                    help="time the 4-layer Llama-3-8B-shaped decoder (prefill and graph-replayed decode, one GPU)")
+    ap.add_argument("--decoder-batches", type=int, nargs="+", default=[1, 8, 32, 128])
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -821,6 +901,9 @@ def main():
         return
     if args.replay_study:
         run_replay_study(args)
+        return
+    if args.decoder:
+        run_decoder(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -68,7 +68,8 @@ int bi_abi_version(void);
  * Bits: 0x1 a producer's wait for a free stage, 0x2 a wait for a loaded stage,
  * 0x4 a wait for the accumulator, 0x8 a cluster handshake; 0x100 decode-attention
  * layout, 0x200 embedding token id, 0x400 KV-append destination row, 0x800
- * prefill-attention layout (the last four are input checks made on the device).
+ * prefill-attention layout, 0x1000 RoPE position (the last five are input checks made on
+ * the device).
  */
 int bi_get_device_error(uint32_t* code, void* stream);
 int bi_clear_device_error(void* stream);

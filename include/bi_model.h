@@ -42,18 +42,29 @@ int bi_embed(const int32_t* tokens, const void* table, void* out, int64_t T, int
              void* stream);
 
 /*
+ * bi_rope_table -- the cos/sin table that bi_rope reads.
+ *
+ * table: fp32 pairs [positions, head_dim/2, 2], 16-byte aligned, owned by the caller.
+ * Entry (p, i) holds (cos a, sin a) for a = p * theta^(-2i/head_dim).  The angle and its
+ * cosine and sine are formed in double precision, then rounded once to fp32.  Build it once
+ * per (theta, head_dim) with as many positions as the longest sequence.  The pages give no
+ * position encoding; RoPE with theta = 500000 is the Llama-3 choice that the decoder's shapes
+ * follow.  head_dim must be a multiple of 4 and theta > 1.
+ */
+int bi_rope_table(void* table, int64_t positions, int32_t head_dim, double theta, void* stream);
+
+/*
  * bi_rope -- rotary position embedding, in place, rotate-half pairing (Llama form).
  *
- * x bf16: T rows of stride ld_row elements.  Each row holds `heads` heads of head_dim dims
- * at columns [h*head_dim, (h+1)*head_dim).  pos int32 [T] gives each row's position p.
- * For pair i < head_dim/2 the angle is p * theta^(-2i/head_dim), formed in double precision.
- * Then (a, b) = (x_i, x_{i+head_dim/2}) -> (a cos - b sin, b cos + a sin) in fp32, and each
- * result is rounded once to bf16.  The pages give no position encoding; RoPE with
- * theta = 500000 is the Llama-3 choice that the decoder's shapes follow.
- * head_dim must be even and theta > 1.
+ * x bf16: T rows of stride ld_row elements (ld_row even, x 4-byte aligned).  Each row holds
+ * `heads` heads of head_dim dims at columns [h*head_dim, (h+1)*head_dim).  pos int32 [T]
+ * gives each row's position p.  For pair i < head_dim/2, with (c, s) = table[p][i],
+ * (a, b) = (x_i, x_{i+head_dim/2}) becomes (a c - b s, b c + a s).  The math is fp32, and each
+ * result is rounded once to bf16.  table comes from bi_rope_table, with table_rows positions.
+ * A position outside [0, table_rows) leaves its row unchanged and sets bit 0x1000.
  */
 int bi_rope(void* x, int64_t T, int64_t ld_row, int32_t heads, int32_t head_dim, const int32_t* pos,
-            double theta, void* stream);
+            const void* table, int64_t table_rows, void* stream);
 
 /*
  * bi_kv_append -- dst[dst_row[t], :] = src[t, :] for t < T

@@ -67,7 +67,8 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_ctrl_decode_attn_adaptive": ([P, P, P, P, P, I32, I64, I32, I32, F, P, C, P, Z, P], C),
         # include/bi_model.h
         "bi_embed": ([P, P, P, I64, I64, I64, P], C),
-        "bi_rope": ([P, I64, I64, I32, I32, P, ctypes.c_double, P], C),
+        "bi_rope_table": ([P, I64, I32, ctypes.c_double, P], C),
+        "bi_rope": ([P, I64, I64, I32, I32, P, P, I64, P], C),
         "bi_kv_append": ([P, I64, P, P, I64, I64, I64, P], C),
         "bi_add": ([P, I64, P, I64, I64, I64, P], C),
         "bi_swiglu": ([P, I64, P, I64, I64, I64, P], C),
@@ -274,7 +275,15 @@ def bi_embed(tokens: torch.Tensor, table: torch.Tensor, out: torch.Tensor | None
     return out
 
 
-def bi_rope(x: torch.Tensor, pos: torch.Tensor, heads: int, head_dim: int = 128, theta: float = 500000.0,
+def bi_rope_table(positions: int, head_dim: int = 128, theta: float = 500000.0, device="cuda",
+                  stream=None) -> torch.Tensor:
+    """The (cos, sin) table bi_rope reads: fp32 [positions, head_dim / 2, 2]."""
+    table = torch.empty((positions, head_dim // 2, 2), dtype=torch.float32, device=device)
+    _check("bi_rope_table", library().bi_rope_table(_ptr(table), positions, head_dim, float(theta), _stream(stream)))
+    return table
+
+
+def bi_rope(x: torch.Tensor, pos: torch.Tensor, heads: int, table: torch.Tensor, head_dim: int = 128,
             stream=None) -> torch.Tensor:
     """Rotary embedding in place on the first heads*head_dim columns of each row of x (bf16)."""
     _bf16_rows(x, "x")
@@ -282,8 +291,10 @@ def bi_rope(x: torch.Tensor, pos: torch.Tensor, heads: int, head_dim: int = 128,
     T = x.shape[0]
     if pos.numel() != T or x.shape[1] < heads * head_dim:
         raise ValueError("shape mismatch")
-    _check("bi_rope", library().bi_rope(_ptr(x), T, x.stride(0), heads, head_dim, _ptr(pos), float(theta),
-                                        _stream(stream)))
+    if table.dtype != torch.float32 or not table.is_contiguous() or table.dim() != 3 or table.shape[1] * 2 != head_dim:
+        raise ValueError("table must be a contiguous fp32 [positions, head_dim / 2, 2] tensor from bi_rope_table")
+    _check("bi_rope", library().bi_rope(_ptr(x), T, x.stride(0), heads, head_dim, _ptr(pos), _ptr(table),
+                                        table.shape[0], _stream(stream)))
     return x
 
 

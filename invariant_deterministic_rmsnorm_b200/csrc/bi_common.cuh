@@ -35,6 +35,7 @@ enum : uint32_t {
     DEVERR_BAD_TOKEN = 1u << 9,     // embedding: token id outside [0, vocab)
     DEVERR_BAD_DST_ROW = 1u << 10,  // KV append: destination row outside the cache
     DEVERR_BAD_PREFILL = 1u << 11,  // prefill attention: indptr / positions outside the buffers
+    DEVERR_BAD_POSITION = 1u << 12, // RoPE: position outside the cos/sin table
 };
 
 // ------------------------------------------------------------------ device helpers

@@ -29,29 +29,43 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const __nv_bflo
 }
 
 // ------------------------------------------------------------------ rotary position embedding
-// For each head row of D dims and pair index i < D/2: angle = pos * theta^(-2i/D), computed in
-// double precision; (x_i, x_{i+D/2}) -> (x_i cos - x_{i+D/2} sin, x_{i+D/2} cos + x_i sin) in fp32,
-// rounded once to bf16 (the "rotate half" pairing of Llama).
+// table[p][i] = (cos, sin) of the angle p * theta^(-2i/D) for pair i < D/2, formed in double
+// precision and rounded once to fp32.  Built once per (theta, D, positions); every rotation reads it.
+__global__ void rope_table_kernel(float2* __restrict__ table, int64_t rows, int half, double log_theta, int D) {
+    const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= rows * half) return;
+    const int64_t p = k / half;
+    const int i = (int)(k % half);
+    const double ang = (double)p * exp(-log_theta * (2.0 * i) / (double)D);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    table[k] = make_float2((float)cd, (float)sd);
+}
+
+// (x_i, x_{i+D/2}) -> (x_i cos - x_{i+D/2} sin, x_{i+D/2} cos + x_i sin) in fp32, rounded once to
+// bf16 (the "rotate half" pairing of Llama).  One thread turns pairs i and i+1 of one head.
 __global__ void rope_kernel(__nv_bfloat16* __restrict__ x, int64_t ld_row, int heads, int D,
-                            const int32_t* __restrict__ pos, double log_theta) {
+                            const int32_t* __restrict__ pos, const float4* __restrict__ table, int64_t table_rows,
+                            uint32_t* err) {
     const int64_t t = blockIdx.x;
-    const int half = D / 2;
-    const double p = (double)pos[t];
-    __nv_bfloat16* row = x + t * ld_row;
-    for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        // the angle depends on (position, pair) only: one double-precision sincos, used by every head
-        const double ang = p * exp(-log_theta * (2.0 * i) / (double)D);
-        double sd, cd;
-        sincos(ang, &sd, &cd);
-        const float s = (float)sd, c = (float)cd;
-        for (int h = 0; h < heads; ++h) {
-            __nv_bfloat16* hp = row + (int64_t)h * D;
-            const float a = __bfloat162float(hp[i]);
-            const float b = __bfloat162float(hp[i + half]);
-            hp[i] = __float2bfloat16_rn(__fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s)));
-            hp[i + half] = __float2bfloat16_rn(__fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s)));
-        }
+    const int half = D / 2, quads = half / 2;  // pairs per head, two at a time
+    const int j = blockIdx.y * blockDim.x + threadIdx.x;
+    if (j >= heads * quads) return;
+    const int32_t p = pos[t];
+    if (p < 0 || p >= table_rows) {
+        if (j == 0) atomicOr(err, bi::DEVERR_BAD_POSITION);  // position outside the table: row left as is
+        return;
     }
+    const int h = j / quads, i = (j % quads) * 2;
+    const float4 cs = table[((int64_t)p * half + i) / 2];  // (cos_i, sin_i, cos_i+1, sin_i+1)
+    uint32_t* lo = reinterpret_cast<uint32_t*>(x + t * ld_row + (int64_t)h * D + i);
+    uint32_t* hi = reinterpret_cast<uint32_t*>(x + t * ld_row + (int64_t)h * D + half + i);
+    const uint32_t av = *lo, bv = *hi;
+    const float a0 = bi::bf16_lo(av), a1 = bi::bf16_hi(av), b0 = bi::bf16_lo(bv), b1 = bi::bf16_hi(bv);
+    *lo = bi::pack_bf16x2(__fsub_rn(__fmul_rn(a0, cs.x), __fmul_rn(b0, cs.y)),
+                          __fsub_rn(__fmul_rn(a1, cs.z), __fmul_rn(b1, cs.w)));
+    *hi = bi::pack_bf16x2(__fadd_rn(__fmul_rn(b0, cs.x), __fmul_rn(a0, cs.y)),
+                          __fadd_rn(__fmul_rn(b1, cs.z), __fmul_rn(a1, cs.w)));
 }
 
 // ------------------------------------------------------------------ KV append
@@ -74,7 +88,8 @@ __global__ void kv_append_kernel(const __nv_bfloat16* __restrict__ src, int64_t 
 __global__ void add_kernel(__nv_bfloat16* __restrict__ h, int64_t ldh, const __nv_bfloat16* __restrict__ d,
                            int64_t ldd, int64_t N) {
     const int64_t t = blockIdx.x;
-    for (int64_t i = threadIdx.x; i < N / 8; i += blockDim.x) {
+    const int64_t i = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;  // 8-element vector of the row
+    if (i < N / 8) {
         uint4* hp = reinterpret_cast<uint4*>(h + t * ldh) + i;
         const uint4 a = *hp;
         const uint4 b = *(reinterpret_cast<const uint4*>(d + t * ldd) + i);
@@ -92,7 +107,8 @@ __global__ void add_kernel(__nv_bfloat16* __restrict__ h, int64_t ldh, const __n
 __global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ gu, int64_t ld_gu, __nv_bfloat16* __restrict__ out,
                               int64_t ld_out, int64_t N) {
     const int64_t t = blockIdx.x;
-    for (int64_t i = threadIdx.x; i < N / 8; i += blockDim.x) {
+    const int64_t i = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;  // 8-element vector of the row
+    if (i < N / 8) {
         const uint4 g = *(reinterpret_cast<const uint4*>(gu + t * ld_gu) + i);
         const uint4 u = *(reinterpret_cast<const uint4*>(gu + t * ld_gu + N) + i);
         uint32_t gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w}, ov[4];
@@ -110,10 +126,11 @@ __global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ gu, int64_t ld_g
 // ------------------------------------------------------------------ argmax
 // The index of the largest fp32 value of each row; among equal values the smallest index.
 // NaN compares as smaller than everything.  One CTA per row, a fixed tree.
-__global__ void __launch_bounds__(256) argmax_kernel(const float* __restrict__ x, int64_t ld, int64_t N,
-                                                     int32_t* __restrict__ out) {
-    __shared__ float sv[256];
-    __shared__ int32_t si[256];
+constexpr int ARGMAX_THREADS = 1024;
+__global__ void __launch_bounds__(ARGMAX_THREADS) argmax_kernel(const float* __restrict__ x, int64_t ld, int64_t N,
+                                                                int32_t* __restrict__ out) {
+    __shared__ float sv[ARGMAX_THREADS];
+    __shared__ int32_t si[ARGMAX_THREADS];
     const int64_t t = blockIdx.x;
     float best = -INFINITY;
     int32_t bi_ = 0x7fffffff;
@@ -127,7 +144,7 @@ __global__ void __launch_bounds__(256) argmax_kernel(const float* __restrict__ x
     sv[threadIdx.x] = best;
     si[threadIdx.x] = bi_;
     __syncthreads();
-    for (int off = 128; off > 0; off >>= 1) {
+    for (int off = ARGMAX_THREADS / 2; off > 0; off >>= 1) {
         if ((int)threadIdx.x < off) {
             const float v = sv[threadIdx.x + off];
             const int32_t j = si[threadIdx.x + off];
@@ -158,15 +175,34 @@ BI_API int bi_embed(const int32_t* tokens, const void* table, void* out, int64_t
     return bi::launch_status();
 }
 
+BI_API int bi_rope_table(void* table, int64_t positions, int32_t head_dim, double theta, void* stream) {
+    if (positions < 0 || head_dim <= 0 || head_dim % 4 != 0 || !(theta > 1.0)) return BI_ERR_INVALID_ARG;
+    if (positions == 0) return BI_OK;
+    if (!table) return BI_ERR_INVALID_ARG;
+    if (!bi::aligned16(table)) return BI_ERR_MISALIGNED;
+    const int half = head_dim / 2;
+    if (positions > ((int64_t)1 << 38) / half) return BI_ERR_UNSUPPORTED_SHAPE;
+    const int64_t n = positions * half;
+    rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, bi::as_stream(stream)>>>(
+        static_cast<float2*>(table), positions, half, log(theta), head_dim);
+    return bi::launch_status();
+}
+
 BI_API int bi_rope(void* x, int64_t T, int64_t ld_row, int32_t heads, int32_t head_dim, const int32_t* pos,
-                   double theta, void* stream) {
-    if (T < 0 || heads <= 0 || head_dim <= 0 || head_dim % 2 != 0 || !(theta > 1.0) || !rows_ok(T))
+                   const void* table, int64_t table_rows, void* stream) {
+    if (T < 0 || heads <= 0 || head_dim <= 0 || head_dim % 4 != 0 || table_rows <= 0 || !rows_ok(T))
         return BI_ERR_INVALID_ARG;
     if (ld_row < (int64_t)heads * head_dim) return BI_ERR_INVALID_ARG;
     if (T == 0) return BI_OK;
-    if (!x || !pos) return BI_ERR_INVALID_ARG;
-    rope_kernel<<<(unsigned)T, 64, 0, bi::as_stream(stream)>>>(static_cast<__nv_bfloat16*>(x), ld_row, heads,
-                                                                head_dim, pos, log(theta));
+    if (!x || !pos || !table) return BI_ERR_INVALID_ARG;
+    if (!bi::aligned16(table) || (reinterpret_cast<uintptr_t>(x) & 3u) || ld_row % 2 != 0) return BI_ERR_MISALIGNED;
+    uint32_t* err = bi::device_error_word();
+    if (!err) return BI_ERR_CUDA;
+    const int work = heads * (head_dim / 4);
+    if ((work + 127) / 128 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
+    dim3 grid((unsigned)T, (unsigned)((work + 127) / 128));
+    rope_kernel<<<grid, 128, 0, bi::as_stream(stream)>>>(static_cast<__nv_bfloat16*>(x), ld_row, heads, head_dim, pos,
+                                                          static_cast<const float4*>(table), table_rows, err);
     return bi::launch_status();
 }
 
@@ -189,7 +225,9 @@ BI_API int bi_add(void* h, int64_t ldh, const void* d, int64_t ldd, int64_t T, i
     if (T == 0) return BI_OK;
     if (!h || !d) return BI_ERR_INVALID_ARG;
     if (N % 8 != 0 || ldh % 8 != 0 || ldd % 8 != 0 || !bi::aligned16(h) || !bi::aligned16(d)) return BI_ERR_MISALIGNED;
-    add_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(static_cast<__nv_bfloat16*>(h), ldh,
+    if ((N / 8 + 255) / 256 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
+    add_kernel<<<dim3((unsigned)T, (unsigned)((N / 8 + 255) / 256)), 256, 0, bi::as_stream(stream)>>>(
+        static_cast<__nv_bfloat16*>(h), ldh,
                                                                 static_cast<const __nv_bfloat16*>(d), ldd, N);
     return bi::launch_status();
 }
@@ -200,7 +238,9 @@ BI_API int bi_swiglu(const void* gu, int64_t ld_gu, void* out, int64_t ld_out, i
     if (!gu || !out) return BI_ERR_INVALID_ARG;
     if (N % 8 != 0 || ld_gu % 8 != 0 || ld_out % 8 != 0 || !bi::aligned16(gu) || !bi::aligned16(out))
         return BI_ERR_MISALIGNED;
-    swiglu_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(gu), ld_gu,
+    if ((N / 8 + 255) / 256 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
+    swiglu_kernel<<<dim3((unsigned)T, (unsigned)((N / 8 + 255) / 256)), 256, 0, bi::as_stream(stream)>>>(
+        static_cast<const __nv_bfloat16*>(gu), ld_gu,
                                                                    static_cast<__nv_bfloat16*>(out), ld_out, N);
     return bi::launch_status();
 }
@@ -209,6 +249,6 @@ BI_API int bi_argmax(const float* x, int64_t ld, int64_t T, int64_t N, int32_t* 
     if (T < 0 || N <= 0 || ld < N || !rows_ok(T) || N > 0x7fffffffLL) return BI_ERR_INVALID_ARG;
     if (T == 0) return BI_OK;
     if (!x || !out) return BI_ERR_INVALID_ARG;
-    argmax_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(x, ld, N, out);
+    argmax_kernel<<<(unsigned)T, ARGMAX_THREADS, 0, bi::as_stream(stream)>>>(x, ld, N, out);
     return bi::launch_status();
 }

@@ -12,7 +12,7 @@ the stream, and the few small int32 index arrays that this module builds on the 
 layer:
 
     x   = bi_rmsnorm(h)                   qkv = bi_gemm(x, Wqkv)            (bf16)
-    bi_rope(q and k heads of qkv, positions)
+    bi_rope(q and k heads of qkv, positions, the cos/sin table built once per engine)
     bi_kv_append(k, v -> the layer's packed caches at each token's slot row)
     att = bi_prefill_attn(q, caches)     or, for one new token per sequence,
           bi_decode_attn(q, caches)       (256-token split-KV, fixed split size)
@@ -60,6 +60,7 @@ class Decoder:
         self.k_cache = [torch.zeros(kv, dtype=torch.bfloat16, device=self.device) for _ in range(shape.layers)]
         self.v_cache = [torch.zeros(kv, dtype=torch.bfloat16, device=self.device) for _ in range(shape.layers)]
         self.length = np.zeros(max_seqs, np.int64)
+        self.rope_table = bi.bi_rope_table(self.cap, shape.head_dim, shape.theta, device=self.device)
         ws = bi.bi_decode_attn_workspace_size(rows, shape.q_heads, shape.head_dim, CHUNK)
         self.attn_ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
 
@@ -71,69 +72,69 @@ class Decoder:
             self.length[np.asarray(slots)] = 0
 
     # ------------------------------------------------------------------ one step
-    def forward(self, slots, tokens, phase: str = "prefill") -> torch.Tensor:
-        """Append tokens[i] (a list of ids) to sequence slots[i], for all i, and run the model over them.
-
-        slots must be strictly increasing.  phase "prefill" runs causal prefill attention over any
-        number of new tokens per sequence; "decode" takes exactly one new token per sequence.
-        Returns fp32 logits [len(slots), vocab] of each sequence's last new token."""
-        s, w, dev = self.s, self.w, self.device
+    def _plan(self, slots, tokens, phase):
+        """Check a step and build its host-side index arrays."""
         slots = [int(x) for x in slots]
         if not slots or any(b <= a for a, b in zip(slots, slots[1:])) or slots[0] < 0 or slots[-1] >= self.max_seqs:
             raise ValueError("slots must be strictly increasing and inside [0, max_seqs)")
         lens = np.array([len(t) for t in tokens], np.int64)
         if len(lens) != len(slots) or np.any(lens <= 0):
             raise ValueError("every listed sequence needs at least one new token")
-        if phase == "decode" and np.any(lens != 1):
-            raise ValueError("a decode step takes exactly one new token per sequence")
         if phase not in ("prefill", "decode"):
             raise ValueError("phase is 'prefill' or 'decode'")
+        if phase == "decode" and np.any(lens != 1):
+            raise ValueError("a decode step takes exactly one new token per sequence")
         start = self.length[slots]
         if np.any(start + lens > self.cap):
             raise ValueError("a sequence outgrows its cache slot")
-        Hq, Hkv, D, H = s.q_heads, s.kv_heads, s.head_dim, s.hidden
-        T, B = int(lens.sum()), len(slots)
         slot_arr = np.asarray(slots, np.int64)
-
-        # host-built index arrays (positions, cache rows, sequence boundaries)
         pos = np.concatenate([st + np.arange(n) for st, n in zip(start, lens)])
-        rows = np.repeat(slot_arr * self.cap, lens) + pos
         q_indptr = np.concatenate([[0], np.cumsum(lens)])
-        toks = np.concatenate([np.asarray(t, np.int32) for t in tokens])
-        d_tok, d_pos, d_rows = _dev_i32(toks, dev), _dev_i32(pos, dev), _dev_i32(rows, dev)
-        d_last = _dev_i32(q_indptr[1:] - 1, dev)
-        use_split = phase == "decode" and self.decode_attention == "split"
-        if use_split:
-            kv_indptr = np.concatenate([slot_arr * self.cap, [(slot_arr[-1] + 1) * self.cap]])
-            d_kv_indptr, d_kv_len = _dev_i32(kv_indptr, dev), _dev_i32(start + 1, dev)
-            d_seq = _dev_i32(np.arange(B), dev)
+        split = phase == "decode" and self.decode_attention == "split"
+        plan = {"T": int(lens.sum()), "B": len(slots), "split": split, "slots": slots, "lens": lens,
+                "tok": np.concatenate([np.asarray(t, np.int32) for t in tokens]), "pos": pos,
+                "rows": np.repeat(slot_arr * self.cap, lens) + pos, "last": q_indptr[1:] - 1}
+        if split:
+            plan["kv_indptr"] = np.concatenate([slot_arr * self.cap, [(slot_arr[-1] + 1) * self.cap]])
+            plan["kv_len"] = start + 1
+            plan["seq"] = np.arange(len(slots))
         else:
-            tiles = bi.prefill_tiles(lens)
-            d_q_indptr, d_tiles = _dev_i32(q_indptr, dev), _dev_i32(tiles, dev)
-            d_kv_base, d_pos0 = _dev_i32(slot_arr * self.cap, dev), _dev_i32(start, dev)
+            plan["tiles"] = bi.prefill_tiles(lens)
+            plan["q_indptr"], plan["kv_base"], plan["pos0"] = q_indptr, slot_arr * self.cap, start
+        return plan
 
+    _INDEX_KEYS = ("tok", "pos", "rows", "last", "kv_indptr", "kv_len", "seq", "tiles", "q_indptr", "kv_base", "pos0")
+
+    def _upload(self, plan) -> dict:
+        return {k: _dev_i32(plan[k], self.device) for k in self._INDEX_KEYS if k in plan}
+
+    def _run(self, T: int, split: bool, n_tiles: int, d: dict) -> torch.Tensor:
+        """The device part of a step: every launch reads its indices from the int32 tensors in d."""
+        s, w, dev = self.s, self.w, self.device
+        Hq, Hkv, D, H = s.q_heads, s.kv_heads, s.head_dim, s.hidden
         bf = torch.bfloat16
-        h = bi.bi_embed(d_tok, w["embed"])
+        h = bi.bi_embed(d["tok"], w["embed"])
         x = torch.empty((T, H), dtype=bf, device=dev)
         qkv = torch.empty((T, s.qkv_cols), dtype=bf, device=dev)
         att = torch.empty((T, Hq * D), dtype=bf, device=dev)
         o = torch.empty((T, H), dtype=bf, device=dev)
         gu = torch.empty((T, 2 * s.ffn), dtype=bf, device=dev)
         a = torch.empty((T, s.ffn), dtype=bf, device=dev)
-        qbuf = torch.empty((T, Hq, D), dtype=bf, device=dev) if use_split else None
+        qbuf = torch.empty((T, Hq, D), dtype=bf, device=dev) if split else None
         for l in range(s.layers):
             bi.bi_rmsnorm(h, w[f"l{l}.attn_norm"], y=x, eps=s.eps)
             bi.bi_gemm(x, w[f"l{l}.wqkv"], C=qkv)
-            bi.bi_rope(qkv, d_pos, Hq + Hkv, D, s.theta)
+            bi.bi_rope(qkv, d["pos"], Hq + Hkv, self.rope_table, D)
             kc, vc = self.k_cache[l], self.v_cache[l]
-            bi.bi_kv_append(qkv[:, Hq * D:(Hq + Hkv) * D], d_rows, kc)
-            bi.bi_kv_append(qkv[:, (Hq + Hkv) * D:], d_rows, vc)
-            if use_split:
-                bi.bi_kv_append(qkv, d_seq, qbuf)  # pack the query heads: [B, Hq, D]
-                bi.bi_decode_attn(qbuf, kc, vc, d_kv_indptr, d_kv_len, out=att.view(T, Hq, D),
+            bi.bi_kv_append(qkv[:, Hq * D:(Hq + Hkv) * D], d["rows"], kc)
+            bi.bi_kv_append(qkv[:, (Hq + Hkv) * D:], d["rows"], vc)
+            if split:
+                bi.bi_kv_append(qkv, d["seq"], qbuf)  # pack the query heads: [B, Hq, D]
+                bi.bi_decode_attn(qbuf, kc, vc, d["kv_indptr"], d["kv_len"], out=att.view(T, Hq, D),
                                   workspace=self.attn_ws)
             else:
-                bi.bi_prefill_attn(qkv, kc, vc, d_q_indptr, d_tiles, tiles[-1], d_kv_base, d_pos0, Hq, out=att)
+                bi.bi_prefill_attn(qkv, kc, vc, d["q_indptr"], d["tiles"], n_tiles, d["kv_base"], d["pos0"], Hq,
+                                   out=att)
             bi.bi_gemm(att, w[f"l{l}.wo"], C=o)
             bi.bi_add(h, o)
             bi.bi_rmsnorm(h, w[f"l{l}.mlp_norm"], y=x, eps=s.eps)
@@ -141,10 +142,24 @@ class Decoder:
             bi.bi_swiglu(gu, out=a)
             bi.bi_gemm(a, w[f"l{l}.wdown"], C=o)
             bi.bi_add(h, o)
-        self.length[slots] = start + lens
-        last = bi.bi_embed(d_last, h)  # row gather: the last new token of each sequence
+        last = bi.bi_embed(d["last"], h)  # row gather: the last new token of each sequence
         xf = bi.bi_rmsnorm(last, w["final_norm"], eps=s.eps)
         return bi.bi_gemm(xf, w["lm_head"], out_dtype=torch.float32)
+
+    def forward(self, slots, tokens, phase: str = "prefill") -> torch.Tensor:
+        """Append tokens[i] (a list of ids) to sequence slots[i], for all i, and run the model over them.
+
+        slots must be strictly increasing.  phase "prefill" runs causal prefill attention over any
+        number of new tokens per sequence; "decode" takes exactly one new token per sequence.
+        Returns fp32 logits [len(slots), vocab] of each sequence's last new token."""
+        plan = self._plan(slots, tokens, phase)
+        logits = self._run(plan["T"], plan["split"], plan.get("tiles", [0])[-1], self._upload(plan))
+        self.length[plan["slots"]] += plan["lens"]
+        return logits
+
+    def decode_graph(self, slots) -> "DecodeGraph":
+        """A CUDA graph of one greedy decode step over `slots` (see DecodeGraph)."""
+        return DecodeGraph(self, slots)
 
     # ------------------------------------------------------------------ greedy generation
     def generate(self, slots, prompts, steps: int, keep=None):
@@ -166,3 +181,63 @@ class Decoder:
                 break
             logits = self.forward(slots, [[int(t)] for t in toks[-1]], "decode")
         return [out[i] for i in keep], np.stack(toks, 1)
+
+
+class DecodeGraph:
+    """One greedy decode step over a fixed set of slots, captured once in a CUDA graph.
+
+    The graph reads the current tokens from a device buffer, appends them at each sequence's
+    next position, writes the logits to a static fp32 buffer, and writes the greedy next tokens
+    back into the token buffer.  It then advances the device copies of the positions, cache
+    rows and KV lengths (or, with prefill attention, the first query positions) by one.  Consecutive replays thus decode greedily with no host work.
+    The host mirrors the lengths in Decoder.length.
+
+    Every launch in the graph is the same launch as in Decoder.forward(..., "decode").  The graph
+    changes when work is issued, not what is computed, so a replayed step gives bitwise the
+    logits of the eager step.
+    """
+
+    def __init__(self, dec: Decoder, slots):
+        self.dec = dec
+        self.slots = [int(x) for x in slots]
+        B = len(self.slots)
+        plan = dec._plan(self.slots, [[0]] * B, "decode")
+        self.d = dec._upload(plan)
+        # positions, cache rows and KV lengths move together; keep them in one buffer so that one
+        # device add advances them all
+        adv = torch.stack([self.d["pos"], self.d["rows"]] + ([self.d["kv_len"]] if plan["split"] else []))
+        self.adv = adv.contiguous()
+        self.d["pos"], self.d["rows"] = self.adv[0], self.adv[1]
+        if plan["split"]:
+            self.d["kv_len"] = self.adv[2]
+        else:
+            self.d["pos0"] = self.adv[0]  # one query row per sequence: its first row is its only row
+        self.split, self.B = plan["split"], B
+        n_tiles = plan.get("tiles", [0])[-1]
+        stream = torch.cuda.Stream(dec.device)
+        stream.wait_stream(torch.cuda.current_stream(dec.device))
+        with torch.cuda.stream(stream):
+            dec._run(B, self.split, n_tiles, self.d)  # warm-up: per-device set-up happens outside the capture
+        torch.cuda.current_stream(dec.device).wait_stream(stream)
+        torch.cuda.synchronize(dec.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=stream):
+            self.logits = dec._run(B, self.split, n_tiles, self.d)
+            bi.bi_argmax(self.logits, out=self.d["tok"])
+            self.adv.add_(1)
+
+    def set_tokens(self, tokens) -> None:
+        """Tokens for the next replay (otherwise the previous replay's greedy tokens are used)."""
+        t = tokens if isinstance(tokens, torch.Tensor) else torch.as_tensor(np.asarray(tokens, np.int32))
+        self.d["tok"].copy_(t.to(self.dec.device, torch.int32))
+
+    def replay(self) -> torch.Tensor:
+        """One decode step; returns the static logits buffer (valid until the next replay)."""
+        if np.any(self.dec.length[self.slots] + 1 > self.dec.cap):
+            raise ValueError("a sequence outgrows its cache slot")
+        self.graph.replay()
+        self.dec.length[self.slots] += 1
+        return self.logits
+
+    def tokens(self) -> torch.Tensor:
+        return self.d["tok"]

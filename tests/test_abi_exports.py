@@ -79,10 +79,15 @@ def test_model_ops_host_checks(lib):
     assert lib.bi_embed(P(a), P(a), P(a), 0, 4096, 32000, s) == 0
     assert lib.bi_embed(P(a), P(a), P(a), 4, 0, 32000, s) == 1
     assert lib.bi_embed(P(a), P(a), P(a), 4, 4100, 32000, s) == 3
-    # rope: odd head_dim, theta <= 1
-    assert lib.bi_rope(P(a), 4, 4096, 32, 127, P(a), 500000.0, s) == 1
-    assert lib.bi_rope(P(a), 4, 4096, 32, 128, P(a), 1.0, s) == 1
-    assert lib.bi_rope(P(a), 0, 4096, 32, 128, P(a), 500000.0, s) == 0
+    # rope: head_dim not a multiple of 4, theta <= 1, empty, misaligned table
+    assert lib.bi_rope_table(P(a), 100, 126, 500000.0, s) == 1
+    assert lib.bi_rope_table(P(a), 100, 128, 1.0, s) == 1
+    assert lib.bi_rope_table(P(a), 0, 128, 500000.0, s) == 0
+    assert lib.bi_rope_table(P(a + 8), 100, 128, 500000.0, s) == 3
+    assert lib.bi_rope(P(a), 4, 4096, 32, 126, P(a), P(a), 100, s) == 1
+    assert lib.bi_rope(P(a), 0, 4096, 32, 128, P(a), P(a), 100, s) == 0
+    assert lib.bi_rope(P(a), 4, 4096, 32, 128, P(a), P(a + 8), 100, s) == 3
+    assert lib.bi_rope(P(a), 4, 4095, 32, 128, P(a), P(a), 100, s) == 1
     # kv append: source stride shorter than a row, misaligned row
     assert lib.bi_kv_append(P(a), 512, P(a), P(a), 4, 1024, 100, s) == 1
     assert lib.bi_kv_append(P(a), 1028, P(a), P(a), 4, 1028, 100, s) == 3

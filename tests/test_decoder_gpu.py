@@ -129,3 +129,21 @@ def test_decode_through_prefill_attention_equals_prefill(llama):
     step = dec.forward([0], [prompt[-1:]], "decode").cpu().numpy()
     assert np.array_equal(full.view(np.uint32), step.view(np.uint32))
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("mode", ["split", "prefill"])
+def test_graph_replayed_decode_equals_eager_decode(llama, mode):
+    shape, w = llama
+    lens = inputs.prompt_lengths(5)
+    prompts = _prompts(range(5), lens, shape.vocab)
+    dec = Decoder(shape, w, max_seqs=5, max_len=2048 + 10, decode_attention=mode)
+    eager, toks = dec.generate(list(range(5)), prompts, 6)
+    dec.reset()
+    dec.forward(list(range(5)), prompts, "prefill")
+    g = dec.decode_graph(list(range(5)))
+    g.set_tokens(toks[:, 0])
+    for step in range(1, 7):
+        logits = g.replay().cpu().numpy()
+        for b in range(5):
+            assert np.array_equal(logits[b].view(np.uint32), eager[b][step].view(np.uint32)), (step, b)
+        assert np.array_equal(g.tokens().cpu().numpy(), toks[:, step])

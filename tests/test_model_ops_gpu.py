@@ -42,7 +42,8 @@ def test_rope_parity(heads, ld):
     x = inputs.normal_bf16(32, (T, ld))
     pos = np.random.default_rng(33).integers(0, 2200, T).astype(np.int32)
     pos[:3] = [0, 1, 2111]
-    got = host(binding.bi_rope(dev(x), dev(pos), heads, D, 500000.0))
+    table = binding.bi_rope_table(2200, D, 500000.0)
+    got = host(binding.bi_rope(dev(x), dev(pos), heads, table, D))
     exact = od.rope(x, pos, heads, D, 500000.0)
     ref = oracle.round_bf16(exact)
     # one bf16 rounding on each side, plus the fp32 error of a rotation (a few 2^-24 of the
@@ -56,6 +57,22 @@ def test_rope_parity(heads, ld):
     assert (d > 0).mean() < 1e-3, (d > 0).mean()
     assert np.array_equal(got[:, heads * D:], x[:, heads * D:])  # columns past the heads untouched
     assert np.array_equal(got[0], x[0])  # position 0 is the identity
+
+
+def test_rope_table_and_bad_position():
+    t = host(binding.bi_rope_table(3000, 128, 500000.0)).astype(np.float64)
+    i = np.arange(64)
+    for p in (0, 1, 2999):
+        ang = p * np.power(500000.0, -2.0 * i / 128)
+        assert np.allclose(t[p, :, 0], np.cos(ang), rtol=0, atol=2 ** -24)
+        assert np.allclose(t[p, :, 1], np.sin(ang), rtol=0, atol=2 ** -24)
+    x = dev(inputs.normal_bf16(41, (2, 256)))
+    x0 = x.clone()
+    binding.bi_clear_device_error()
+    binding.bi_rope(x, dev(np.array([5, 3000], np.int32)), 2, binding.bi_rope_table(3000, 128))
+    assert binding.bi_get_device_error() & 0x1000
+    binding.bi_clear_device_error()
+    assert torch.equal(x[1], x0[1]) and not torch.equal(x[0], x0[0])
 
 
 def test_kv_append_scatters_rows_exactly():
