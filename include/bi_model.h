@@ -122,7 +122,7 @@ int bi_argmax(const float* x, int64_t ld, int64_t T, int64_t N, int32_t* out, vo
  *                 Rows q_indptr[b] .. q_indptr[b+1]-1 belong to sequence b.
  *   q_indptr      int32 [B+1], non-decreasing, q_indptr[B] <= q_rows.
  *   q_tile_indptr int32 [B+1]: q_tile_indptr[0] = 0 and
- *                 q_tile_indptr[b+1] = q_tile_indptr[b] + ceil((q_indptr[b+1] - q_indptr[b]) / 64).
+ *                 q_tile_indptr[b+1] = q_tile_indptr[b] + ceil((q_indptr[b+1] - q_indptr[b]) / 128).
  *                 n_tiles = q_tile_indptr[B].  Built on the host with the lengths.
  *   q_pos0        int32 [B]: the position of sequence b's first query row.  Query row i of
  *                 the sequence is at position q_pos0[b] + i.
@@ -137,7 +137,16 @@ int bi_argmax(const float* x, int64_t ld, int64_t T, int64_t N, int32_t* out, vo
  *
  * Query row i attends to the keys at positions 0 .. q_pos0[b] + i:
  *   out = softmax(scale * q k^T) v.
- * Scores are fp32.  P.V multiplies P as a bf16 high part plus a bf16 low remainder.
+ * Both products run on the tensor cores (tcgen05, fp32 accumulators in TMEM), one CTA per
+ * (128-row query tile, query head).  Scores are fp32, and the softmax works in base 2:
+ * p = 2^(s * scale * log2(e) - m), with the hardware's approximate exp2.  Each row keeps a
+ * reference max m.  It raises m only when a block's max exceeds it by more than 8 (a factor
+ * of 256), and then rescales the accumulated output and sum.  P.V multiplies P as a bf16
+ * high part (p cut to 8 significant bits) plus the bf16-rounded remainder.  The sum of P
+ * follows a fixed tree.  Values past a tile's last
+ * position are zeroed before they meet a zero P.  Every choice is row-local.  Bitwise
+ * invariance covers every output bit, except the sign of an output element that is exactly
+ * zero.
  *
  * Constraints:
  *   - head_dim must be 128 (BI_ERR_UNSUPPORTED_SHAPE otherwise), and Hq a multiple of Hkv.

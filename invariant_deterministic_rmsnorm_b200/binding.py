@@ -352,11 +352,14 @@ def bi_argmax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> 
     return out
 
 
+PREFILL_TILE_ROWS = 128
+
+
 def prefill_tiles(q_lens) -> list:
-    """q_tile_indptr for query lengths q_lens: prefix sums of ceil(len / 64)."""
+    """q_tile_indptr for query lengths q_lens: prefix sums of ceil(len / 128)."""
     out = [0]
     for n in q_lens:
-        out.append(out[-1] + (int(n) + 63) // 64)
+        out.append(out[-1] + (int(n) + PREFILL_TILE_ROWS - 1) // PREFILL_TILE_ROWS)
     return out
 
 

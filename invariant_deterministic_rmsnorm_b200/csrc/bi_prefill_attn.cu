@@ -1,4 +1,5 @@
-// bi_prefill_attn.cu -- batch-invariant causal prefill attention (grouped-query, variable length).
+// bi_prefill_attn.cu -- batch-invariant causal prefill attention (grouped-query, variable length)
+// on the sm_100 tensor cores (tcgen05, accumulators in TMEM).
 //
 // Source: "Defeating Nondeterminism in LLM Inference" (Spanish summary), section "Attention".
 // FlashAttention-2-style kernels are batch-invariant when they parallelise over queries and
@@ -11,15 +12,24 @@
 // position q_pos0[b] + i.  Keys and values of sequence b are rows kv_indptr[b] + p of the packed
 // caches [tokens, Hkv, 128], for positions p = 0 .. position of the query (causal).
 //
-// One CTA per (64-row query tile of a sequence, query head).  Each of its 4 warps owns 16
-// query rows.  KV blocks of 64 positions, starting at position 0, are visited in ascending
-// order.  For each block:
-//   S = scale * Q K^T                  mma.sync m16n8k16, bf16 products, fp32 sums
-//   causal mask, then the online softmax: m' = max(m, rowmax S);  c = e^(m - m');  P = e^(S - m')
-//   l = l c + rowsum P;  O = O c + P V  (P split into bf16 hi + lo parts, both multiplied by V)
-// and out = O / l rounded to bf16.  Row i's arithmetic depends only on its own sequence's query
-// row, keys and values.  Blocks entirely above a row's position contribute exact zeros and
-// factors of one, so the tile a row shares with other rows never changes its bits.
+// One CTA per (128-row query tile of a sequence, query head), 6 warps:
+//   warp 0      TMA producer: the Q tile once, then K and V blocks of 64 positions into a
+//               3-stage ring
+//   warp 1      tcgen05.mma issuer (and TMEM owner):
+//                 S_j = Q K_j^T into one of two TMEM score buffers;
+//                 O += P_hi V_j + P_lo V_j into the TMEM output accumulator
+//   warps 2..9  softmax and epilogue, two threads per query row (TMEM lane): one takes the
+//               first 32 keys of each block and output dims 0..63, the other the rest
+// KV blocks of 64 positions, starting at position 0, are visited in ascending order.  For
+// block j, each row computes, in base-2 units:
+//   t = S_j * scale * log2(e) (masked to -inf past the row's position)
+//   m' = m, or the block max when that exceeds m by more than 8 (then O and l are rescaled
+//        by 2^(m - m'), read from and written back to TMEM)
+//   p = 2^(t - m') (the hardware's approximate exp2);  l += sum p (a fixed summation tree);
+//   P = hi + lo, hi = p cut to bf16, lo = bf16(p - hi)
+// and out = O / l rounded to bf16.  Every decision above is row-local.  Blocks past a row's
+// position contribute exact zeros: masked scores, zeroed values past the tile's last position.
+// So the rows a tile shares with a row never change its bits.
 #include <mutex>
 
 #include "bi_common.cuh"
@@ -32,33 +42,89 @@ using namespace bi::sm100;
 namespace {
 
 constexpr int D = 128;
-constexpr int QT = 64;                 // query rows per CTA
-constexpr int KB = 64;                 // keys per block
-constexpr int THREADS = 128;           // 4 warps x 16 query rows
-constexpr int HALF_BYTES = 64 * 64 * 2;  // one TMA box: 64 rows x 64 dims = 8 KB
-constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 64 rows x 128 dims = 16 KB
-constexpr size_t SMEM_BYTES = 1024 + TILE_BYTES /*Q*/ + 2 * 2 * TILE_BYTES /*K,V x 2 stages*/ + 64;
+constexpr int QT = 128;               // query rows per CTA (the MMA's M)
+constexpr int KB = 64;                // keys per block
+constexpr int NST = 3;                // K/V ring stages
+constexpr int THREADS = 320;          // producer, MMA, 8 softmax warps
+constexpr int Q_BOX = 64 * QT * 2;    // 64 dims x 128 rows = 16 KB
+constexpr int KV_BOX = 64 * KB * 2;   // 64 dims x 64 keys = 8 KB
+constexpr int Q_BYTES = 2 * Q_BOX;    // 32 KB
+constexpr int KV_BLOCK = 2 * KV_BOX;  // 16 KB: K (or V) of one block
+constexpr int P_BYTES = QT * KB * 2;  // 16 KB: one bf16 P tile
+constexpr float RESCALE_GAP = 8.0f;   // raise the reference max only past this margin (base 2: x256)
+constexpr uint32_t TMEM_COLS = 256;   // S x 2 (64 columns each) + O (128 columns)
+constexpr uint32_t O_COL = 128;
 
-__device__ __forceinline__ uint32_t tile_addr(uint32_t base, int row, int dim) {
-    return swz(base + (uint32_t)(dim >> 6) * HALF_BYTES + (uint32_t)row * 128 + (uint32_t)(dim & 63) * 2, 7u);
+struct Bars {
+    uint64_t q_full;
+    uint64_t kv_full[NST];
+    uint64_t kv_empty[NST];
+    uint64_t s_full[2];
+    uint64_t p_full;   // the softmax warps wrote P_j (and rescaled O)
+    uint64_t p_empty;  // PV_j done: the P tiles are free and O is stable
+    uint64_t o_full;   // the last PV is done
+    uint64_t drain;    // every MMA this CTA issued has completed
+    uint64_t xchg;     // the 8 softmax warps swapped their partial row maxima (or sums)
+    float xmax[2][2][QT];  // [block parity][half][row]
+    float xsum[2][QT];     // [half][row]
+    uint32_t tmem_addr;
+    int abort;
+};
+
+constexpr size_t SMEM_BYTES = 1024 + Q_BYTES + 2 * NST * KV_BLOCK + 2 * P_BYTES + sizeof(Bars) + 64;
+
+__device__ __forceinline__ void fail(uint32_t* err, volatile int* abort, uint32_t bit) {
+    atomicOr(err, bit);
+    *abort = 1;
 }
 
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) { return bi::pack_bf16x2(lo, hi); }
+// 2^x with the hardware's approximate base-2 exponential (relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
-__global__ void __launch_bounds__(THREADS, 2)
-prefill_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ q_indptr,
-                    const int32_t* __restrict__ q_tile_indptr, const int32_t* __restrict__ kv_indptr,
-                    const int32_t* __restrict__ q_pos0, int B, int Hq, int Hkv, int q_rows, int cache_tokens,
-                    float scale, __nv_bfloat16* __restrict__ out, int64_t ldo, uint32_t* err) {
+// Generic-proxy writes to shared memory become visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+           "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+           "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+           "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__global__ void __launch_bounds__(THREADS, 1)
+prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ q_indptr,
+                       const int32_t* __restrict__ q_tile_indptr, const int32_t* __restrict__ kv_indptr,
+                       const int32_t* __restrict__ q_pos0, int B, int Hq, int Hkv, int q_rows, int cache_tokens,
+                       int n_tiles, float scale_log2, __nv_bfloat16* __restrict__ out, int64_t ldo, uint32_t* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sQ = smem_u32(base);
-    const uint32_t sKV = sQ + TILE_BYTES;  // stage s: K at sKV + s*2*TILE, V at + TILE
-    uint64_t* bars = reinterpret_cast<uint64_t*>(base + TILE_BYTES + 4 * TILE_BYTES);  // [0] Q, [1..2] stages
+    const uint32_t sK = sQ + Q_BYTES;          // stage s at sK + s * KV_BLOCK
+    const uint32_t sV = sK + NST * KV_BLOCK;   // stage s at sV + s * KV_BLOCK
+    const uint32_t sPh = sV + NST * KV_BLOCK;  // P high parts
+    const uint32_t sPl = sPh + P_BYTES;        // P low parts
+    Bars* bars = reinterpret_cast<Bars*>(base + Q_BYTES + 2 * NST * KV_BLOCK + 2 * P_BYTES);
+    volatile int* abort = &bars->abort;
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile = blockIdx.x, h = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = n_tiles - 1 - (int)blockIdx.x;  // the longer tiles of a sequence start first
+    const int h = blockIdx.y;
     const int g = h / (Hq / Hkv);
 
     // the sequence that owns this tile: the last b with q_tile_indptr[b] <= tile
@@ -69,219 +135,299 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     const int b = lo;
     const int qt = tile - q_tile_indptr[b];
-    const int q_row0 = q_indptr[b] + qt * QT;               // first query row of the tile
-    const int n_q = min(QT, q_indptr[b + 1] - q_row0);      // live query rows
-    const int pos0 = q_pos0[b] + qt * QT;                   // position of the tile's first row
-    const int kv_base = kv_indptr[b];
-    const int last_pos = pos0 + n_q - 1;                    // highest position any live row sees
-    const int n_blocks = last_pos / KB + 1;
+    const int q_row0 = q_indptr[b] + qt * QT;            // first query row of the tile
+    const int n_q = min(QT, q_indptr[b + 1] - q_row0);   // live query rows
     if (n_q <= 0) return;  // a tile index past the last sequence's tiles
-    // the documented layout, checked before any copy or store: rows inside q/out, positions
-    // inside the caches
+    const int pos0 = q_pos0[b] + qt * QT;                // position of the tile's first row
+    const int kv_base = kv_indptr[b];
+    const int last_pos = pos0 + n_q - 1;                 // the highest position any live row sees
+    const int nb = last_pos / KB + 1;
+    // the documented layout, checked before any copy or store
     if (q_indptr[b + 1] > q_rows || q_indptr[b] < 0 || pos0 < 0 || kv_base < 0 ||
         (int64_t)kv_base + last_pos >= (int64_t)cache_tokens) {
-        if (tid == 0) atomicOr(err, bi::DEVERR_BAD_PREFILL);
+        if (threadIdx.x == 0) atomicOr(err, bi::DEVERR_BAD_PREFILL);
         return;
     }
 
-    __shared__ int s_abort;  // set once a wait has run out: later waits give up at once, no new copies
-    if (tid == 0) {
-        s_abort = 0;
-        for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bars->q_full), 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(smem_u32(&bars->kv_full[s]), 1);
+            mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bars->s_full[0]), 1);
+        mbar_init(smem_u32(&bars->s_full[1]), 1);
+        mbar_init(smem_u32(&bars->p_full), 8);
+        mbar_init(smem_u32(&bars->p_empty), 1);
+        mbar_init(smem_u32(&bars->o_full), 1);
+        mbar_init(smem_u32(&bars->drain), 1);
+        mbar_init(smem_u32(&bars->xchg), 8);
+        bars->abort = 0;
         fence_barrier_init();
         fence_proxy_async_shared();
     }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&bars->tmem_addr), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    auto issue_kv = [&](int kb) {
-        const int st = kb & 1;
-        const uint32_t bar = smem_u32(&bars[1 + st]);
-        const uint32_t dk = sKV + st * 2 * TILE_BYTES;
-        mbar_arrive_expect_tx(bar, 2 * TILE_BYTES);
-        for (int hf = 0; hf < 2; ++hf) {
-            tma_load_2d(dk + hf * HALF_BYTES, &tmK, g * D + hf * 64, kv_base + kb * KB, bar);
-            tma_load_2d(dk + TILE_BYTES + hf * HALF_BYTES, &tmV, g * D + hf * 64, kv_base + kb * KB, bar);
-        }
-    };
-    if (tid == 0) {
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
-        const uint32_t qb = smem_u32(&bars[0]);
-        mbar_arrive_expect_tx(qb, TILE_BYTES);
-        for (int hf = 0; hf < 2; ++hf) tma_load_2d(sQ + hf * HALF_BYTES, &tmQ, h * D + hf * 64, q_row0, qb);
-        issue_kv(0);
-    }
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_addr;
 
-    int issued = 0;  // (thread 0) KV blocks whose copies were started
-    const int gq = lane >> 2, cq = lane & 3;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars[0]), 0u, &s_abort));
-    if (!ok && lane == 0) {
-        atomicOr(err, bi::DEVERR_WAIT_FULL);
-        s_abort = 1;
-    }
-    uint32_t qa[8][4];
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) ldmatrix_x4(tile_addr(sQ, warp * 16 + (lane & 15), kk * 16 + (lane >> 4) * 8), qa[kk]);
-
-    // this thread's two query rows and their positions
-    const int qpos_a = pos0 + warp * 16 + gq, qpos_b = qpos_a + 8;
-    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-    float o[16][4];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-
-    for (int kb = 0; kb < n_blocks; ++kb) {
-        // the stage of block kb + 1 was released by the barrier that ended block kb - 1
-        if (tid == 0 && kb + 1 < n_blocks && *(volatile int*)&s_abort == 0) {
-            issue_kv(kb + 1);
-            issued = kb + 1;
-        }
-        const int st = kb & 1;
-        const bool w_ok =
-            __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars[1 + st]), (uint32_t)(kb >> 1) & 1u, &s_abort));
-        if (!w_ok) {
-            ok = false;
-            if (lane == 0) {
-                atomicOr(err, bi::DEVERR_WAIT_FULL);
-                s_abort = 1;
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            const uint32_t qb = smem_u32(&bars->q_full);
+            mbar_arrive_expect_tx(qb, Q_BYTES);
+            tma_load_2d(sQ, &tmQ, h * D, q_row0, qb);
+            tma_load_2d(sQ + Q_BOX, &tmQ, h * D + 64, q_row0, qb);
+            int issued = 0;
+            for (int j = 0; j < nb; ++j) {
+                const int s = j % NST;
+                if (!mbar_wait(smem_u32(&bars->kv_empty[s]), ((uint32_t)(j / NST) & 1u) ^ 1u, abort)) {
+                    fail(err, abort, bi::DEVERR_WAIT_TMA);
+                    break;
+                }
+                const uint32_t fb = smem_u32(&bars->kv_full[s]);
+                mbar_arrive_expect_tx(fb, 2 * KV_BLOCK);
+                const int row = kv_base + j * KB;
+                tma_load_2d(sK + s * KV_BLOCK, &tmK, g * D, row, fb);
+                tma_load_2d(sK + s * KV_BLOCK + KV_BOX, &tmK, g * D + 64, row, fb);
+                tma_load_2d(sV + s * KV_BLOCK, &tmV, g * D, row, fb);
+                tma_load_2d(sV + s * KV_BLOCK + KV_BOX, &tmV, g * D + 64, row, fb);
+                issued = j + 1;
+            }
+            if (*abort) {  // let the copies in flight land before the CTA's shared memory is released
+                (void)mbar_wait(smem_u32(&bars->q_full), 0u, nullptr);
+                for (int j = issued > NST ? issued - NST : 0; j < issued; ++j)
+                    (void)mbar_wait(smem_u32(&bars->kv_full[j % NST]), (uint32_t)(j / NST) & 1u, nullptr);
             }
         }
-        const uint32_t sK = sKV + st * 2 * TILE_BYTES, sV = sK + TILE_BYTES;
-        if (w_ok) {
-            // ---- S = Q K^T for this warp's 16 rows x 64 keys
-            float s[8][4];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-                for (int np = 0; np < 4; ++np) {  // pairs of 8-key n-tiles
-                    uint32_t bb[4];
-                    const int mi = lane >> 3;
-                    ldmatrix_x4(tile_addr(sK, np * 16 + (mi >> 1) * 8 + (lane & 7), kk * 16 + (mi & 1) * 8), bb);
-                    const uint32_t b0[2] = {bb[0], bb[1]}, b1[2] = {bb[2], bb[3]};
-                    mma_m16n8k16_bf16(s[2 * np], qa[kk], b0);
-                    mma_m16n8k16_bf16(s[2 * np + 1], qa[kk], b1);
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = make_idesc_bf16_f32(QT, KB, 0, 0);  // Q and K both K-major
+            constexpr uint32_t idesc_o = make_idesc_bf16_f32(QT, D, 0, 1);   // P K-major, V N-major
+            // S_j = Q K_j^T into score buffer j % 2 (8 steps of 16 dims; dims 64..127 sit in the second box)
+            auto issue_s = [&](int j) -> bool {
+                const int s = j % NST;
+                if (!mbar_wait(smem_u32(&bars->kv_full[s]), (uint32_t)(j / NST) & 1u, abort)) {
+                    fail(err, abort, bi::DEVERR_WAIT_FULL);
+                    return false;
                 }
-            }
-            // ---- scale, causal mask, online softmax (rows a = gq, b = gq + 8 of this warp)
-            float mx_a = -INFINITY, mx_b = -INFINITY;
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(j & 1) * KB;
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int kpos = kb * KB + nt * 8 + 2 * cq + (e & 1);
-                    const int qpos = (e >> 1) ? qpos_b : qpos_a;
-                    const float v = kpos <= qpos ? __fmul_rn(s[nt][e], scale) : -INFINITY;
-                    s[nt][e] = v;
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t off = (uint32_t)(k & 3) * 32u;
+                    const uint64_t ad = make_smem_desc(sQ + (uint32_t)(k >> 2) * Q_BOX + off, 16, 1024, 2);
+                    const uint64_t bd =
+                        make_smem_desc(sK + (uint32_t)s * KV_BLOCK + (uint32_t)(k >> 2) * KV_BOX + off, 16, 1024, 2);
+                    mma_bf16_ss(d, ad, bd, idesc_s, k > 0 ? 1u : 0u);
                 }
-                mx_a = fmaxf(mx_a, fmaxf(s[nt][0], s[nt][1]));
-                mx_b = fmaxf(mx_b, fmaxf(s[nt][2], s[nt][3]));
-            }
-            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-            const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-            // a fully masked block keeps m: the factor is exactly 1 and P is exactly 0
-            const float c_a = (mn_a == -INFINITY) ? 1.f : expf(__fsub_rn(m_a, mn_a));
-            const float c_b = (mn_b == -INFINITY) ? 1.f : expf(__fsub_rn(m_b, mn_b));
-            float sum_a = 0.f, sum_b = 0.f;
-            uint32_t pa_hi[4][4], pa_lo[4][4];  // A fragments of P for the 4 16-key steps
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                float p[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float mref = (e >> 1) ? mn_b : mn_a;
-                    p[e] = (s[nt][e] == -INFINITY) ? 0.f : expf(__fsub_rn(s[nt][e], mref));
+                mma_commit(smem_u32(&bars->s_full[j & 1]));
+                return true;
+            };
+            bool ok = mbar_wait(smem_u32(&bars->q_full), 0u, abort);
+            if (!ok) fail(err, abort, bi::DEVERR_WAIT_FULL);
+            for (int j = 0; ok && j < nb && j < 2; ++j) ok = issue_s(j);
+            for (int j = 0; ok && j < nb; ++j) {
+                if (!mbar_wait(smem_u32(&bars->p_full), (uint32_t)j & 1u, abort)) {
+                    fail(err, abort, bi::DEVERR_WAIT_FULL);
+                    ok = false;
+                    break;
                 }
-                sum_a = __fadd_rn(sum_a, __fadd_rn(p[0], p[1]));
-                sum_b = __fadd_rn(sum_b, __fadd_rn(p[2], p[3]));
-                float ph[4], pl[4];
+                tc_fence_after();
+                const int s = j % NST;
+                // O += P_hi V_j + P_lo V_j (4 steps of 16 keys each)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    ph[e] = __bfloat162float(__float2bfloat16_rn(p[e]));
-                    pl[e] = __fsub_rn(p[e], ph[e]);
-                }
-                const int ks = nt >> 1, half = nt & 1;  // n-tile nt covers keys 8*(nt&1) of step ks
-                pa_hi[ks][half * 2 + 0] = pack2(ph[0], ph[1]);
-                pa_hi[ks][half * 2 + 1] = pack2(ph[2], ph[3]);
-                pa_lo[ks][half * 2 + 0] = pack2(pl[0], pl[1]);
-                pa_lo[ks][half * 2 + 1] = pack2(pl[2], pl[3]);
-            }
-            sum_a = __fadd_rn(sum_a, __shfl_xor_sync(0xffffffffu, sum_a, 1));
-            sum_a = __fadd_rn(sum_a, __shfl_xor_sync(0xffffffffu, sum_a, 2));
-            sum_b = __fadd_rn(sum_b, __shfl_xor_sync(0xffffffffu, sum_b, 1));
-            sum_b = __fadd_rn(sum_b, __shfl_xor_sync(0xffffffffu, sum_b, 2));
-            l_a = __fmaf_rn(l_a, c_a, sum_a);
-            l_b = __fmaf_rn(l_b, c_b, sum_b);
-            m_a = mn_a;
-            m_b = mn_b;
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t sP = part == 0 ? sPh : sPl;
 #pragma unroll
-            for (int dt = 0; dt < 16; ++dt) {
-                o[dt][0] = __fmul_rn(o[dt][0], c_a);
-                o[dt][1] = __fmul_rn(o[dt][1], c_a);
-                o[dt][2] = __fmul_rn(o[dt][2], c_b);
-                o[dt][3] = __fmul_rn(o[dt][3], c_b);
-            }
-            // ---- O += P V (keys past the last live position are masked in the V fragments)
-            const int key_limit = last_pos - kb * KB;  // keys j <= key_limit of this block may be read
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                // A operand: rows (gq, gq+8) x keys of step ks; registers: (row a, keys lo),
-                // (row b, keys lo), (row a, keys hi), (row b, keys hi)
-                const uint32_t ah[4] = {pa_hi[ks][0], pa_hi[ks][1], pa_hi[ks][2], pa_hi[ks][3]};
-                const uint32_t al[4] = {pa_lo[ks][0], pa_lo[ks][1], pa_lo[ks][2], pa_lo[ks][3]};
-#pragma unroll
-                for (int dp = 0; dp < 8; ++dp) {  // pairs of 8-dim n-tiles
-                    uint32_t vb[4];
-                    const int mi = lane >> 3;
-                    ldmatrix_x4_trans(tile_addr(sV, ks * 16 + (lane & 7) + (mi & 1) * 8, dp * 16 + (mi >> 1) * 8), vb);
-                    if (ks * 16 + 15 > key_limit) {
-                        // keys 2cq, 2cq+1 (+8) of this step: zero the halves past the limit
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int kj = ks * 16 + 2 * cq + (r & 1) * 8;
-                            uint32_t m = 0u;
-                            if (kj <= key_limit) m |= 0x0000FFFFu;
-                            if (kj + 1 <= key_limit) m |= 0xFFFF0000u;
-                            vb[r] &= m;
-                        }
+                    for (int k = 0; k < KB / 16; ++k) {
+                        const uint64_t ad = make_smem_desc(sP + (uint32_t)k * 32u, 16, 1024, 2);
+                        const uint64_t bd = make_smem_desc(sV + (uint32_t)s * KV_BLOCK + (uint32_t)k * 16u * 128u,
+                                                           KV_BOX, 1024, 2);
+                        mma_bf16_ss(tmem + O_COL, ad, bd, idesc_o, (j > 0 || part > 0 || k > 0) ? 1u : 0u);
                     }
-                    const uint32_t v0[2] = {vb[0], vb[1]}, v1[2] = {vb[2], vb[3]};
-                    mma_m16n8k16_bf16(o[2 * dp], ah, v0);
-                    mma_m16n8k16_bf16(o[2 * dp], al, v0);
-                    mma_m16n8k16_bf16(o[2 * dp + 1], ah, v1);
-                    mma_m16n8k16_bf16(o[2 * dp + 1], al, v1);
+                }
+                mma_commit(smem_u32(&bars->p_empty));
+                mma_commit(smem_u32(&bars->kv_empty[s]));
+                if (j + 2 < nb) ok = issue_s(j + 2);
+            }
+            if (ok && !*abort) mma_commit(smem_u32(&bars->o_full));
+            // every MMA issued above completes before TMEM is released
+            mma_commit(smem_u32(&bars->drain));
+            (void)mbar_wait(smem_u32(&bars->drain), 0u, nullptr);
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax + epilogue
+        // Two threads share a query row: `half` 0 takes keys 0..31 of every block and output
+        // dims 0..63, half 1 keys 32..63 and dims 64..127.  They swap their partial row maxima
+        // (and at the end their partial sums) through shared memory behind an mbarrier.
+        const int sw = warp - 2;             // softmax warp 0..7
+        const int half = sw >> 2;
+        const int quarter = warp & 3;        // this warp reads TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;   // query row of the tile
+        const bool live = r < n_q;
+        const int qpos = pos0 + r;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nb; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->s_full[j & 1]), (uint32_t)(j >> 1) & 1u, abort));
+            if (!ok) {
+                if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+                break;
+            }
+            tc_fence_after();
+            float sv[32];
+            {
+                uint32_t r0[32];
+                tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(j & 1) * KB + (uint32_t)half * 32u, r0);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) sv[c] = __uint_as_float(r0[c]);
+            }
+            const int kpos0 = j * KB + half * 32;  // position of this thread's first key in the block
+            // scores in base-2 units: t = s * scale * log2(e); keys past the row's position are -inf.
+            // A warp whose rows all sit at or past its last key of the block needs no mask.
+            const bool unmasked = __all_sync(0xffffffffu, live && kpos0 + 31 <= qpos);
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const float v = (unmasked || (live && kpos0 + c <= qpos)) ? __fmul_rn(sv[c], scale_log2) : -INFINITY;
+                sv[c] = v;
+                mx4[c & 3] = fmaxf(mx4[c & 3], v);
+            }
+            const float mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            bars->xmax[j & 1][half][r] = mine;
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->xchg));
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->xchg), (uint32_t)j & 1u, abort));
+            if (!ok) {
+                if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_CLUSTER);
+                break;
+            }
+            const float mx = fmaxf(mine, bars->xmax[j & 1][half ^ 1][r]);
+            float m_new = m_ref;
+            if (m_ref == -INFINITY || mx > m_ref + RESCALE_GAP) m_new = fmaxf(m_ref, mx);
+            const bool need = m_new != m_ref && m_ref != -INFINITY;
+            const float c_fac = need ? ex2_approx(__fsub_rn(m_ref, m_new)) : 1.0f;
+            // PV_{j-1} must be done before P is overwritten or O is rescaled
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->p_empty), (uint32_t)(j - 1) & 1u, abort));
+                if (!ok) {
+                    if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+                    break;
+                }
+                tc_fence_after();
+            }
+            if (__any_sync(0xffffffffu, need)) {  // a warp-collective TMEM round trip; c_fac is 1 where not needed
+#pragma unroll 1
+                for (int c = 0; c < D / 2; c += 32) {
+                    const uint32_t col = O_COL + (uint32_t)(half * (D / 2) + c);
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(tmem + lane_off + col, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), c_fac));
+                    tmem_st_32x32b_x32(tmem + lane_off + col, o);
+                }
+                tmem_wait_st();
+            }
+            if (need) l = __fmul_rn(l, c_fac);
+            m_ref = m_new;
+            // p = 2^(t - m_ref); P = hi + lo with hi = p cut to bf16 (exact top 8 significant bits)
+            // and lo = bf16(p - hi) (p - hi is exact in fp32); both go to the 128B-swizzled
+            // K-major P tiles.  The partial row sum is four interleaved sums, added in a fixed order.
+            const uint32_t row_off = (uint32_t)r * 128u;
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t ph[4], pl[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = ex2_approx(__fsub_rn(sv[cc * 8 + 2 * e], m_ref));
+                    const float p1 = ex2_approx(__fsub_rn(sv[cc * 8 + 2 * e + 1], m_ref));
+                    l4[e] = __fadd_rn(__fadd_rn(l4[e], p0), p1);
+                    const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                    ph[e] = __byte_perm(u0, u1, 0x7632);  // the top halves: bf16(p0) | bf16(p1) << 16, cut
+                    pl[e] = bi::pack_bf16x2(__fsub_rn(p0, __uint_as_float(u0 & 0xFFFF0000u)),
+                                            __fsub_rn(p1, __uint_as_float(u1 & 0xFFFF0000u)));
+                }
+                const int ch = half * 4 + cc;  // 16-byte chunk (8 keys) of the row
+                const uint32_t off = row_off + ((uint32_t)(ch ^ (r & 7)) << 4);
+                st_shared_v4(sPh + off, ph[0], ph[1], ph[2], ph[3]);
+                st_shared_v4(sPl + off, pl[0], pl[1], pl[2], pl[3]);
+            }
+            l = __fadd_rn(l, __fadd_rn(__fadd_rn(l4[0], l4[1]), __fadd_rn(l4[2], l4[3])));
+            // values past the tile's last position (another sequence's rows, or never written) are
+            // zeroed, so that a zero P never meets a non-finite V; half h clears box h of the row
+            const int vrow_pos = j * KB + r;
+            if (j * KB + KB - 1 > last_pos && r < KB && vrow_pos > last_pos) {
+                const int s = j % NST;
+                // the stage's copy completed before S_j was issued; this wait makes its bytes
+                // visible to this thread before they are overwritten
+                if (mbar_wait(smem_u32(&bars->kv_full[s]), (uint32_t)(j / NST) & 1u, abort)) {
+                    const uint32_t v0 = sV + (uint32_t)s * KV_BLOCK + (uint32_t)half * KV_BOX + (uint32_t)r * 128u;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) st_shared_v4(v0 + q * 16, 0u, 0u, 0u, 0u);
+                } else {
+                    fail(err, abort, bi::DEVERR_WAIT_FULL);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->p_full));
+        }
+        // ---------------------------------------------------------------- epilogue: out = O / l
+        if (ok) {  // the row sum: half 0's part plus half 1's part, in that order
+            bars->xsum[half][r] = l;
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->xchg));
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->xchg), (uint32_t)nb & 1u, abort));
+            if (!ok && lane == 0) fail(err, abort, bi::DEVERR_WAIT_CLUSTER);
+            l = __fadd_rn(bars->xsum[0][r], bars->xsum[1][r]);
+        }
+        if (ok) {
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full), 0u, abort));
+            if (!ok && lane == 0) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+        }
+        if (ok) {
+            tc_fence_after();
+            __nv_bfloat16* dst = out + (int64_t)(q_row0 + r) * ldo + (int64_t)h * D + half * (D / 2);
+#pragma unroll 1
+            for (int c = 0; c < D / 2; c += 32) {
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(tmem + lane_off + O_COL + (uint32_t)(half * (D / 2) + c), o);
+                tmem_wait_ld();
+                if (live) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = bi::pack_bf16x2(__fdiv_rn(__uint_as_float(o[2 * i]), l),
+                                                __fdiv_rn(__uint_as_float(o[2 * i + 1]), l));
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4)
+                        *reinterpret_cast<uint4*>(dst + c + 2 * i) = make_uint4(pk[i], pk[i + 1], pk[i + 2], pk[i + 3]);
                 }
             }
         }
-        __syncthreads();  // every warp is done with this stage before it is refilled
     }
 
-    if (tid == 0 && *(volatile int*)&s_abort) {
-        // a wait ran out: let the copies still in flight land (bounded) before the CTA's shared
-        // memory is released.  At most the Q tile and the last two KV blocks can be pending.
-        mbar_wait(smem_u32(&bars[0]), 0u, nullptr);
-        for (int j = issued > 0 ? issued - 1 : 0; j <= issued; ++j)
-            mbar_wait(smem_u32(&bars[1 + (j & 1)]), (uint32_t)(j >> 1) & 1u, nullptr);
-    }
-    // ---- out = O / l for the live rows of this warp
-    const int row_a = warp * 16 + gq, row_b = row_a + 8;
-    if (ok) {
-#pragma unroll
-        for (int dt = 0; dt < 16; ++dt) {
-            const int d = dt * 8 + 2 * cq;
-            if (row_a < n_q) {
-                __nv_bfloat16* p = out + (int64_t)(q_row0 + row_a) * ldo + (int64_t)h * D + d;
-                *reinterpret_cast<uint32_t*>(p) = pack2(__fdiv_rn(o[dt][0], l_a), __fdiv_rn(o[dt][1], l_a));
-            }
-            if (row_b < n_q) {
-                __nv_bfloat16* p = out + (int64_t)(q_row0 + row_b) * ldo + (int64_t)h * D + d;
-                *reinterpret_cast<uint32_t*>(p) = pack2(__fdiv_rn(o[dt][2], l_b), __fdiv_rn(o[dt][3], l_b));
-            }
-        }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
@@ -291,7 +437,7 @@ bool ensure_attr() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::call_once(once[dev], [&] {
-        okd[dev] = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        okd[dev] = cudaFuncSetAttribute(prefill_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)SMEM_BYTES) == cudaSuccess;
     });
     return okd[dev];
@@ -326,8 +472,8 @@ BI_API int bi_prefill_attn(const void* q, int64_t ldq, int64_t q_rows, const voi
                           64, KB, CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
     dim3 grid((unsigned)n_tiles, (unsigned)Hq);
-    prefill_attn_kernel<<<grid, THREADS, SMEM_BYTES, bi::as_stream(stream)>>>(
-        tmQ, tmK, tmV, q_indptr, q_tile_indptr, kv_indptr, q_pos0, B, Hq, Hkv, (int)q_rows, (int)cache_tokens, scale,
-        static_cast<__nv_bfloat16*>(out), ldo, err);
+    prefill_attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, bi::as_stream(stream)>>>(
+        tmQ, tmK, tmV, q_indptr, q_tile_indptr, kv_indptr, q_pos0, B, Hq, Hkv, (int)q_rows, (int)cache_tokens,
+        n_tiles, (float)((double)scale * 1.4426950408889634), static_cast<__nv_bfloat16*>(out), ldo, err);
     return bi::launch_status();
 }

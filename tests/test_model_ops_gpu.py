@@ -153,6 +153,7 @@ def _oracle_prefill(q, k, v, q_lens, pos0, kv_base):
     ([1, 63, 64, 65, 200, 7], [0, 0, 0, 0, 0, 0]),        # ragged tiles and KV blocks
     ([130, 5, 64], [300, 1, 63]),                          # chunked prefill over a cached prefix
     ([1, 1, 1], [0, 1000, 2047]),                          # single rows (decode through prefill)
+    ([300, 129, 128, 127], [0, 0, 5, 700]),                # several 128-row tiles, ragged last tiles
 ])
 def test_prefill_attention_parity(q_lens, pos0):
     q, k, v, ql, p0, kb = _prefill_case(q_lens, pos0)
