@@ -688,8 +688,9 @@ def run_sweep(args):
         g = torch.Generator(device=device).manual_seed(seed)
         return torch.randn((M, cols), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
 
+    only = set(args.sweep_ops)
     # GEMM
-    for i, (K, N) in enumerate(GEMM_SHAPES):
+    for i, (K, N) in enumerate(GEMM_SHAPES if "gemm" in only else []):
         table = []
         for M in (1, 16, 64, 128, 256, 512, 1024, 2048, 4096, 8192):
             R = _copies(2 * (M * K + K * N + M * N))
@@ -706,7 +707,7 @@ def run_sweep(args):
     # RMSNorm
     table = []
     w = _to_dev(inputs.rmsnorm_case(1, HIDDEN, "bf16")[1], device)
-    for M in (1, 64, 256, 1024, 4096, 8192, 16384):
+    for M in ((1, 64, 256, 1024, 4096, 8192, 16384) if "rmsnorm" in only else ()):
         R = _copies(2 * 2 * HIDDEN * M)
         xs = [rows_dev(70 + j, M, HIDDEN) for j in range(R)]
         ys = [torch.empty_like(xs[0]) for _ in range(R)]
@@ -717,9 +718,10 @@ def run_sweep(args):
         table.append({"M": M, "bi_gbs": round(by / (t_bi / 1e3), 1), "split_gbs": round(by / (t_sp / 1e3), 1),
                       "bi_frac": round(by / (t_bi / 1e3) / peaks["hbm_gbs"], 3)})
         del xs, ys
-    emit({"op": "rmsnorm", "H": HIDDEN, "dtype": "bf16", "rows": table})
+    if table:
+        emit({"op": "rmsnorm", "H": HIDDEN, "dtype": "bf16", "rows": table})
     # LoRA shrink and expand
-    for r in (8, 16, 64):
+    for r in ((8, 16, 64) if "lora" in only else ()):
         A_l = rows_dev(80, HIDDEN, r).mul_(0.02)
         B_l = rows_dev(81, r, HIDDEN).mul_(0.02)
         table = []
@@ -745,6 +747,8 @@ def run_sweep(args):
             del xs, ys
         emit({"op": "lora", "r": r, "K": HIDDEN, "N": HIDDEN, "split_k": 8, "rows": table})
     # decode attention: prefixes of one packed cache of 128 requests
+    if "attn" not in only:
+        return
     kv_len = inputs.kv_lengths(128)
     indptr, T = inputs.kv_layout(kv_len, 256)
     g = torch.Generator(device=device).manual_seed(5)
@@ -880,6 +884,131 @@ def run_decoder(args):
         del g
 
 
+class FastOps:
+    """Batch-dependent fast paths for the decoder's three batch-sensitive ops: cuBLAS through
+    torch.mm, RMSNorm split over a cluster with the split chosen by M, decode attention with the
+    chunk size chosen by the batch size.  Used only by the --contrast measurement."""
+
+    @staticmethod
+    def gemm(A, W, C=None, out_dtype=None):
+        import torch
+        if C is not None:
+            return torch.mm(A, W, out=C)
+        if out_dtype == torch.float32:
+            return torch.mm(A, W, out_dtype=torch.float32)
+        return torch.mm(A, W)
+
+    @staticmethod
+    def rmsnorm(x, w, y=None, eps=1e-6):
+        import torch
+        from invariant_deterministic_rmsnorm_b200 import binding as B
+        if y is None:
+            y = torch.empty_like(x)
+        for r0 in range(0, x.shape[0], 65535):  # the comparator's grid takes at most 65535 rows a call
+            B.bi_ctrl_rmsnorm_split(x[r0:r0 + 65535], w, y=y[r0:r0 + 65535], eps=eps)
+        return y
+
+    @staticmethod
+    def decode_attn(q, k, v, kv_indptr, kv_len, out, workspace):
+        from invariant_deterministic_rmsnorm_b200 import binding as B
+        return B.bi_ctrl_decode_attn_adaptive(q, k, v, kv_indptr, kv_len, out=out)
+
+
+def run_contrast(args):
+    """Position-invariant scheduling against batch-invariant kernels, on the same synthetic decoder.
+
+    The alternative (the CoRun comment thread, "thecolony.si" page) keeps the fast, batch-dependent
+    kernels and fixes the shapes instead: every request is prefilled alone, and decode always
+    runs a fixed 128-slot batch (empty slots hold a short filler prompt), replayed from one CUDA
+    graph.  Printed: decode tokens/s at several real batch sizes for the BI decoder (true batch),
+    the fast kernels at the true batch (dynamic shapes), and the fast kernels at the fixed shape;
+    then, bit for bit, whether a probe request's logits over prefill + 16 greedy steps stay the
+    same when its co-residents or its slot change."""
+    import torch
+    from invariant_deterministic_rmsnorm_b200 import binding as B
+    from invariant_deterministic_rmsnorm_b200.decoder import Decoder
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    shape = inputs.LLAMA3_8B_4L
+    w = inputs.decoder_weights_device(shape, device=device)
+    BF, probe_steps = 128, 16
+    steps = max(4, args.steps)
+    max_len = 2048 + 2 * (steps + args.warmup + probe_steps) + 8
+    lens = inputs.prompt_lengths(BF)
+    prompts = [inputs.prompt(i, int(n), shape.vocab) for i, n in enumerate(lens)]
+    filler = inputs.prompt(inputs.SEED_FILLER_BASE, 16, shape.vocab)
+    dec = {"bi": Decoder(shape, w, BF, max_len), "fast": Decoder(shape, w, BF, max_len, ops=FastOps)}
+
+    def fill(d, slots, contents, isolated):
+        """Prefill; returns the greedy next token of every listed slot."""
+        d.reset()
+        if isolated:
+            return [int(B.bi_argmax(d.forward([s], [c]))[0]) for s, c in zip(slots, contents)]
+        return B.bi_argmax(d.forward(slots, contents)).cpu().tolist()
+
+    def step_ms(d, slots):
+        g = d.decode_graph(slots)
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / steps
+
+    rows = []
+    for b in args.contrast_batches:
+        real = list(range(b))
+        fill(dec["bi"], real, prompts[:b], False)
+        t_bi = step_ms(dec["bi"], real)
+        fill(dec["fast"], real, prompts[:b], False)
+        t_dyn = step_ms(dec["fast"], real)
+        fill(dec["fast"], list(range(BF)), prompts[:b] + [filler] * (BF - b), True)
+        t_fix = step_ms(dec["fast"], list(range(BF)))
+        rows.append({"requests": b, "bi_ms": round(t_bi, 4), "bi_tokens_per_s": round(b / t_bi * 1e3),
+                     "fast_dynamic_ms": round(t_dyn, 4), "fast_dynamic_tokens_per_s": round(b / t_dyn * 1e3),
+                     "fast_fixed128_ms": round(t_fix, 4), "fast_fixed128_tokens_per_s": round(b / t_fix * 1e3)})
+    print(json.dumps({"contrast": "decode_throughput", "fixed_slots": BF, "steps": steps, "rows": rows}), flush=True)
+
+    probe = prompts[0]
+
+    def probe_logits(d, slots, contents, at, isolated):
+        """The probe's (contents[at]) logits at each of probe_steps greedy decode steps after the prefill."""
+        first = fill(d, slots, contents, isolated)
+        g = d.decode_graph(slots)
+        g.set_tokens(first)
+        got = []
+        for _ in range(probe_steps):
+            got.append(g.replay()[at].cpu().numpy().copy())
+        del g
+        return np.stack(got)
+
+    def same(a, b):
+        return bool(np.array_equal(a.view(np.uint32), b.view(np.uint32)))
+
+    others = prompts[1:BF]
+    fixed_alone = probe_logits(dec["fast"], list(range(BF)), [filler] * 5 + [probe] + [filler] * (BF - 6), 5, True)
+    fixed_busy = probe_logits(dec["fast"], list(range(BF)), others[:5] + [probe] + others[5:BF - 1], 5, True)
+    fixed_moved = probe_logits(dec["fast"], list(range(BF)), [filler] * 77 + [probe] + [filler] * (BF - 78), 77, True)
+    dyn_alone = probe_logits(dec["fast"], [0], [probe], 0, False)
+    dyn_busy = probe_logits(dec["fast"], list(range(37)), others[:5] + [probe] + others[5:36], 5, False)
+    bi_alone = probe_logits(dec["bi"], [0], [probe], 0, False)
+    bi_busy = probe_logits(dec["bi"], list(range(37)), others[:5] + [probe] + others[5:36], 5, False)
+    bi_fixed = probe_logits(dec["bi"], list(range(BF)), others[:5] + [probe] + others[5:BF - 1], 5, False)
+    print(json.dumps({"contrast": "composition", "probe_len": len(probe), "decode_steps": probe_steps,
+                      "fast_fixed128_alone_vs_busy_same_slot": same(fixed_alone, fixed_busy),
+                      "fast_fixed128_slot5_vs_slot77": same(fixed_alone, fixed_moved),
+                      "fast_dynamic_alone_vs_batch37": same(dyn_alone, dyn_busy),
+                      "fast_dynamic_max_abs_diff": float(np.abs(dyn_alone - dyn_busy).max()),
+                      "bi_alone_vs_batch37": same(bi_alone, bi_busy),
+                      "bi_alone_vs_batch128_batched_prefill": same(bi_alone, bi_fixed),
+                      "fast_vs_bi_max_abs_diff": float(np.abs(fixed_alone - bi_alone).max())}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -893,11 +1022,17 @@ def main():
     ap.add_argument("--replays", type=int, default=200)
     ap.add_argument("--sweep", action="store_true",
                     help="print per-op throughput across batch sizes (one GPU) instead of the benchmark line")
+    ap.add_argument("--sweep-ops", nargs="+", default=["gemm", "rmsnorm", "lora", "attn"],
+                    choices=["gemm", "rmsnorm", "lora", "attn"], help="ops the sweep covers")
     ap.add_argument("--attn-batch", type=int, default=ATTN_BATCH,
                     help="decode requests in the step (smaller for profiler captures)")
     ap.add_argument("--decoder", action="store_true",
                     help="time the 4-layer Llama-3-8B-shaped decoder (prefill and graph-replayed decode, one GPU)")
     ap.add_argument("--decoder-batches", type=int, nargs="+", default=[1, 8, 32, 128])
+    ap.add_argument("--contrast", action="store_true",
+                    help="position-invariant scheduling (fixed-shape decode over batch-dependent fast kernels) "
+                         "against the batch-invariant decoder (one GPU)")
+    ap.add_argument("--contrast-batches", type=int, nargs="+", default=[1, 8, 32, 128])
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -910,6 +1045,9 @@ def main():
         return
     if args.decoder:
         run_decoder(args)
+        return
+    if args.contrast:
+        run_contrast(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -38,6 +38,25 @@ from .inputs import DecoderShape
 CHUNK = 256
 
 
+class BIOps:
+    """The three batch-dependent-in-general ops of a step, on the library's batch-invariant kernels.
+
+    A Decoder takes another table with the same three calls only to measure an alternative
+    (see bench.py --contrast).  The default is always this one."""
+
+    @staticmethod
+    def gemm(A, W, C=None, out_dtype=torch.bfloat16):
+        return bi.bi_gemm(A, W, C=C, out_dtype=out_dtype)
+
+    @staticmethod
+    def rmsnorm(x, w, y=None, eps=1e-6):
+        return bi.bi_rmsnorm(x, w, y=y, eps=eps)
+
+    @staticmethod
+    def decode_attn(q, k, v, kv_indptr, kv_len, out, workspace):
+        return bi.bi_decode_attn(q, k, v, kv_indptr, kv_len, out=out, workspace=workspace)
+
+
 def _dev_i32(a, device) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(device, non_blocking=False)
 
@@ -46,7 +65,7 @@ class Decoder:
     """A decoder with weights `weights` (bf16 device tensors named as DecoderShape.matrices())."""
 
     def __init__(self, shape: DecoderShape, weights: dict, max_seqs: int, max_len: int, device="cuda",
-                 decode_attention: str = "split"):
+                 decode_attention: str = "split", ops=BIOps):
         if shape.head_dim != 128:
             raise ValueError("the attention kernels take head_dim 128")
         if decode_attention not in ("split", "prefill"):
@@ -55,6 +74,7 @@ class Decoder:
         self.max_seqs = max_seqs
         self.cap = (max_len + CHUNK - 1) // CHUNK * CHUNK
         self.decode_attention = decode_attention
+        self.ops = ops
         rows = max_seqs * self.cap
         kv = (rows, shape.kv_heads, shape.head_dim)
         self.k_cache = [torch.zeros(kv, dtype=torch.bfloat16, device=self.device) for _ in range(shape.layers)]
@@ -110,7 +130,7 @@ class Decoder:
 
     def _run(self, T: int, split: bool, n_tiles: int, d: dict) -> torch.Tensor:
         """The device part of a step: every launch reads its indices from the int32 tensors in d."""
-        s, w, dev = self.s, self.w, self.device
+        s, w, dev, ops = self.s, self.w, self.device, self.ops
         Hq, Hkv, D, H = s.q_heads, s.kv_heads, s.head_dim, s.hidden
         bf = torch.bfloat16
         h = bi.bi_embed(d["tok"], w["embed"])
@@ -122,29 +142,28 @@ class Decoder:
         a = torch.empty((T, s.ffn), dtype=bf, device=dev)
         qbuf = torch.empty((T, Hq, D), dtype=bf, device=dev) if split else None
         for l in range(s.layers):
-            bi.bi_rmsnorm(h, w[f"l{l}.attn_norm"], y=x, eps=s.eps)
-            bi.bi_gemm(x, w[f"l{l}.wqkv"], C=qkv)
+            ops.rmsnorm(h, w[f"l{l}.attn_norm"], y=x, eps=s.eps)
+            ops.gemm(x, w[f"l{l}.wqkv"], C=qkv)
             bi.bi_rope(qkv, d["pos"], Hq + Hkv, self.rope_table, D)
             kc, vc = self.k_cache[l], self.v_cache[l]
             bi.bi_kv_append(qkv[:, Hq * D:(Hq + Hkv) * D], d["rows"], kc)
             bi.bi_kv_append(qkv[:, (Hq + Hkv) * D:], d["rows"], vc)
             if split:
                 bi.bi_kv_append(qkv, d["seq"], qbuf)  # pack the query heads: [B, Hq, D]
-                bi.bi_decode_attn(qbuf, kc, vc, d["kv_indptr"], d["kv_len"], out=att.view(T, Hq, D),
-                                  workspace=self.attn_ws)
+                ops.decode_attn(qbuf, kc, vc, d["kv_indptr"], d["kv_len"], att.view(T, Hq, D), self.attn_ws)
             else:
                 bi.bi_prefill_attn(qkv, kc, vc, d["q_indptr"], d["tiles"], n_tiles, d["kv_base"], d["pos0"], Hq,
                                    out=att)
-            bi.bi_gemm(att, w[f"l{l}.wo"], C=o)
+            ops.gemm(att, w[f"l{l}.wo"], C=o)
             bi.bi_add(h, o)
-            bi.bi_rmsnorm(h, w[f"l{l}.mlp_norm"], y=x, eps=s.eps)
-            bi.bi_gemm(x, w[f"l{l}.wgu"], C=gu)
+            ops.rmsnorm(h, w[f"l{l}.mlp_norm"], y=x, eps=s.eps)
+            ops.gemm(x, w[f"l{l}.wgu"], C=gu)
             bi.bi_swiglu(gu, out=a)
-            bi.bi_gemm(a, w[f"l{l}.wdown"], C=o)
+            ops.gemm(a, w[f"l{l}.wdown"], C=o)
             bi.bi_add(h, o)
         last = bi.bi_embed(d["last"], h)  # row gather: the last new token of each sequence
-        xf = bi.bi_rmsnorm(last, w["final_norm"], eps=s.eps)
-        return bi.bi_gemm(xf, w["lm_head"], out_dtype=torch.float32)
+        xf = ops.rmsnorm(last, w["final_norm"], eps=s.eps)
+        return ops.gemm(xf, w["lm_head"], out_dtype=torch.float32)
 
     def forward(self, slots, tokens, phase: str = "prefill") -> torch.Tensor:
         """Append tokens[i] (a list of ids) to sequence slots[i], for all i, and run the model over them.
