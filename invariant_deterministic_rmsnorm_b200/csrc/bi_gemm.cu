@@ -255,6 +255,238 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     }
 }
 
+// ------------------------------------------------------------------ the CTA-pair kernel
+// A 2-CTA cluster computes a 256 x 256 output tile with tcgen05.mma.cta_group::2: CTA r of the
+// pair loads rows [128r, 128r + 128) of the A tile and columns [128r, 128r + 128) of the W tile,
+// and holds rows [128r, 128r + 128) x all 256 columns of the accumulator in its TMEM.  Per SM
+// that is 32 KB of operands per 64-deep K block for the same MMA work the single-CTA 128 x 256
+// tile gets from 48 KB; an SM can take in about 64 bytes a cycle from L2, and this is what lets
+// the tensor pipe stay busy.  Each output element is still one fp32 chain over K in ascending
+// 16-deep steps, and the plan depends on (N, K) only.
+namespace pair {
+constexpr int ROWS = 128;                 // A rows per CTA
+constexpr int COLS = 128;                 // W columns per CTA
+constexpr int TILE_M = 2 * ROWS;          // 256
+constexpr int TILE_N = 2 * COLS;          // 256
+constexpr int A_ST = ROWS * BK * 2;       // 16 KB
+constexpr int B_ST = COLS * BK * 2;       // 16 KB: two boxes of 64 columns x 64 K-rows
+constexpr int ST_BYTES = A_ST + B_ST;     // 32 KB per CTA per stage
+constexpr int STAGES = 6;
+constexpr uint32_t ACC_COLS = TILE_N;     // one fp32 accumulator: 256 TMEM columns
+constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+struct Bars {
+    uint64_t full[STAGES];   // leader: both CTAs' bytes of stage s have landed
+    uint64_t empty[STAGES];  // each CTA: the MMAs have read its stage s
+    uint64_t tfull[2];       // each CTA: accumulator b holds a finished tile
+    uint64_t tempty[2];      // leader: both CTAs' epilogues have read accumulator b
+    uint64_t drain;          // leader: every MMA issued has completed
+    uint32_t tmem_addr;
+    int abort;
+};
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * ST_BYTES + sizeof(Bars) + 64;
+}  // namespace pair
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                         void* __restrict__ C, int M, int N, int K, int c_bf16, int gm, uint32_t* err) {
+    using pair::ROWS;
+    using pair::COLS;
+    using pair::TILE_M;
+    using pair::TILE_N;
+    using pair::A_ST;
+    using pair::B_ST;
+    using pair::ST_BYTES;
+    using pair::STAGES;
+    using pair::ACC_COLS;
+    using pair::TMEM_COLS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * A_ST;
+    pair::Bars* bars = reinterpret_cast<pair::Bars*>(sB + STAGES * B_ST);
+    volatile int* abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: the leader, which issues the MMAs
+    const int pair_id = (int)(blockIdx.x >> 1), n_pairs = (int)(gridDim.x >> 1);
+    const int tiles_m = (M + TILE_M - 1) / TILE_M;
+    const int tiles_n = (N + TILE_N - 1) / TILE_N;
+    const int num_tiles = tiles_m * tiles_n;
+    const int num_kb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&bars->full[s]), 1);
+            mbar_init(smem_u32(&bars->empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&bars->tfull[b]), 1);
+            mbar_init(smem_u32(&bars->tempty[b]), 2 * EPI_WARPS);
+        }
+        mbar_init(smem_u32(&bars->drain), 1);
+        bars->abort = 0;
+        fence_barrier_init();
+        fence_proxy_async_shared();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(&bars->tmem_addr), TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    // both CTAs' barriers are initialised and their TMEM allocated before any signal crosses the pair
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = bars->tmem_addr;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;  // k-blocks issued by this CTA so far (the ring runs across tiles)
+            for (int t = pair_id; t < num_tiles && !*abort; t += n_pairs) {
+                int mt, nt;
+                tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
+                const int m0 = mt * TILE_M + (int)rank * ROWS, n0 = nt * TILE_N + (int)rank * COLS;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = (int)(it % STAGES);
+                    const uint32_t round = it / STAGES;
+                    if (!mbar_wait(smem_u32(&bars->empty[s]), (round & 1u) ^ 1u, abort)) {
+                        fail(err, abort, bi::DEVERR_WAIT_TMA);
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&bars->full[s]);
+                    if (rank == 0) mbar_arrive_expect_tx(fb, 2 * ST_BYTES);  // this stage of both CTAs
+                    const uint32_t fb_leader = mapa(fb, 0);
+                    tma_load_2d_pair(smem_u32(sA + s * A_ST), &tmA, kb * BK, m0, fb_leader);
+                    tma_load_2d_pair(smem_u32(sB + s * B_ST), &tmW, n0, kb * BK, fb_leader);
+                    tma_load_2d_pair(smem_u32(sB + s * B_ST + B_BOX), &tmW, n0 + 64, kb * BK, fb_leader);
+                }
+            }
+            if (*abort) {
+                // let loads already in flight land before the CTA's shared memory is released: the
+                // leader tracks both CTAs' bytes; the peer waits a fixed time
+                if (rank == 0) {
+                    for (uint32_t i = it > (uint32_t)STAGES ? it - STAGES : 0u; i < it; ++i)
+                        (void)mbar_wait(smem_u32(&bars->full[i % STAGES]), (i / STAGES) & 1u, nullptr);
+                } else {
+                    const uint64_t t0 = globaltimer();
+                    while (globaltimer() - t0 < 200000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = make_idesc_bf16_f32(TILE_M, TILE_N, 0, 1);
+            const uint32_t peer_empty0 = mapa(smem_u32(&bars->empty[0]), 1);
+            const uint32_t peer_tfull0 = mapa(smem_u32(&bars->tfull[0]), 1);
+            uint32_t it = 0, local = 0;
+            for (int t = pair_id; t < num_tiles && !*abort; t += n_pairs, ++local) {
+                const uint32_t acc = local & 1u, use = local >> 1;
+                if (!mbar_wait(smem_u32(&bars->tempty[acc]), (use & 1u) ^ 1u, abort)) {
+                    fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = (int)(it % STAGES);
+                    const uint32_t round = it / STAGES;
+                    if (!mbar_wait(smem_u32(&bars->full[s]), round & 1u, abort)) {
+                        fail(err, abort, bi::DEVERR_WAIT_FULL);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA + s * A_ST);
+                    const uint32_t b_base = smem_u32(sB + s * B_ST);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        const uint64_t adesc = make_smem_desc(a_base + k * UMMA_K * 2, 16, 1024, 2);
+                        const uint64_t bdesc = make_smem_desc(b_base + k * UMMA_K * 128, B_BOX, 1024, 2);
+                        mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    // stage s of both CTAs is free once these MMAs have read it
+                    mma_commit_pair(smem_u32(&bars->empty[s]));
+                    mma_commit_pair(peer_empty0 + (uint32_t)s * 8u);
+                }
+                mma_commit_pair(smem_u32(&bars->tfull[acc]));  // both CTAs' accumulator rows complete
+                mma_commit_pair(peer_tfull0 + acc * 8u);
+            }
+            mma_commit_pair(smem_u32(&bars->drain));  // TMEM is released only after every MMA completed
+            (void)mbar_wait(smem_u32(&bars->drain), 0u, nullptr);
+        }
+    } else {
+        const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter .. +31
+        const uint32_t tempty0 = rank == 0 ? smem_u32(&bars->tempty[0]) : mapa(smem_u32(&bars->tempty[0]), 0);
+        uint32_t local = 0;
+        for (int t = pair_id; t < num_tiles; t += n_pairs, ++local) {
+            const uint32_t acc = local & 1u, use = local >> 1;
+            const bool ok = mbar_wait(smem_u32(&bars->tfull[acc]), use & 1u, abort);
+            if (!ok) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+            // tcgen05.ld is warp-collective: the whole warp takes the same branch
+            if (!__all_sync(0xffffffffu, ok && !*abort)) break;
+            tc_fence_after();
+            int mt, nt;
+            tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
+            const int row = mt * TILE_M + (int)rank * ROWS + quarter * 32 + lane;
+            const uint32_t lane_addr = tmem_base + acc * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < TILE_N; c += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(lane_addr + (uint32_t)c, r);
+                tmem_wait_ld();
+                if (c == TILE_N - 32) {  // every column of this accumulator is in registers: hand it back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8u);
+                }
+                const int col = nt * TILE_N + c;
+                if (row < M && col < N) {
+                    if (!c_bf16) {
+                        float* dst = static_cast<float*>(C) + (int64_t)row * N + col;
+                        if (col + 32 <= N) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<uint4*>(dst + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < N - col) dst[i] = __uint_as_float(r[i]);
+                        }
+                    } else {
+                        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(C) + (int64_t)row * N + col;
+                        uint32_t p[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            p[i] = bi::pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        if (col + 32 <= N) {
+#pragma unroll
+                            for (int i = 0; i < 16; i += 4)
+                                *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(p[i], p[i + 1], p[i + 2], p[i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < N - col) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // no CTA of the pair leaves (or frees TMEM) while the other may still signal it
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 int num_sms() {
     static int cached[64];
@@ -312,13 +544,41 @@ int launch_gemm_bn(const void* A, int64_t lda, const void* W, int64_t ldw, void*
     return bi::launch_status();
 }
 
+// The CTA-pair kernel: 256 x 256 tiles over 2-CTA clusters, one cluster per SM pair at most.
+int launch_gemm_pair(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N,
+                     int64_t K, bool c_bf16, cudaStream_t stream) {
+    uint32_t* err = bi::device_error_word();
+    if (!err) return BI_ERR_CUDA;
+    static std::once_flag once[64];
+    static bool attr_ok[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BI_ERR_CUDA;
+    std::call_once(once[dev], [&] {
+        attr_ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)pair::SMEM_BYTES) == cudaSuccess;
+    });
+    if (!attr_ok[dev]) return BI_ERR_CUDA;
+    CUtensorMap tmA, tmW;
+    if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK,
+                          pair::ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    if (!bi::make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)N, (uint64_t)K, (uint64_t)ldw * 2, 64,
+                          BK, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    const int64_t tiles = ((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N);
+    const int sms = num_sms();
+    if (sms < 2) return BI_ERR_CUDA;
+    const int gm = 16;  // row tiles per group of the tile walk (L2 reuse of A and W blocks)
+    const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+    bi_gemm_bf16_pair_kernel<<<dim3((unsigned)(2 * pairs)), THREADS, pair::SMEM_BYTES, stream>>>(
+        tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, err);
+    return bi::launch_status();
+}
+
 int launch_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N, int64_t K,
                 bool c_bf16, cudaStream_t stream) {
-    switch (plan_bn(N, K)) {
-        case 64: return launch_gemm_bn<64>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
-        case 128: return launch_gemm_bn<128>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
-        default: return launch_gemm_bn<256>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
-    }
+    (void)plan_bn;
+    return launch_gemm_pair(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
 }
 
 int gemm_shape_checks(const void* A, const void* W, const void* C, int64_t M, int64_t N, int64_t K, int c_dtype) {
