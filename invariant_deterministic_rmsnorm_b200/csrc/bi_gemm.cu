@@ -6,21 +6,28 @@
 // "Multiplicación de matrices".  The matmul is tile-parallel over 2-D output tiles.
 // Small batches tempt implementations into split-K, and a split chosen by batch size
 // breaks batch invariance.  The fix the section gives is to force one kernel
-// configuration for every batch size.  Here the configuration is fixed by (N, K)
-// alone: the tile (128 x 256), the MMA shape (128 x 256 x 16), the K-block order
-// (ascending, 64 at a time) and the split count (1).  A row's tile position and
-// the batch size M change which CTA computes the row.  They never change the
-// instructions that produce its bits.  Rows past M are zero-filled by the TMA unit
-// and are never stored.
+// configuration for every batch size.  Here the configuration is fixed by (N, K) and the
+// device alone, never by M:
+//   - N up to 256 x (SM pairs) (18944 on a B200): 256 x 256 tiles over a 2-CTA cluster,
+//     tcgen05.mma.cta_group::2 256 x 256 x 16;
+//   - wider N: 128 x 256 tiles on one CTA, tcgen05.mma.cta_group::1 128 x 256 x 16.
+// In both, the K-block order is ascending (64 at a time) and the split count is 1.  A row's
+// tile position and the batch size M change which CTA computes the row.  They never change
+// the instructions that produce its bits.  Rows past M are zero-filled by the TMA unit and
+// are never stored.
 //
-// CTA structure (192 threads):
-//   warp 0      TMA producer: A tile [128 x 64] and W tile [64 x 256] per stage, 4-stage ring
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (4 MMAs of K = 16 per stage)
-//   warps 2..5  epilogue: tcgen05.ld of the 128 x 256 fp32 accumulator, convert, store
+// CTA structure (192 threads; in the pair kernel two CTAs per cluster):
+//   warp 0      TMA producer.  Pair kernel: 128 rows of A [128 x 64] and 128 columns of W
+//               [64 x 128] per stage, 6-stage ring, completion bytes of both CTAs counted by
+//               the leader.  Single-CTA kernel: A [128 x 64] and W [64 x 256], 4-stage ring.
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer (the leader's, in the pair
+//               kernel): 4 MMAs of K = 16 per stage
+//   warps 2..5  epilogue: tcgen05.ld of this CTA's 128 x 256 fp32 accumulator rows, convert,
+//               store
 // Shared-memory operand layouts are the 128-byte-swizzled canonical forms that the TMA
-// unit writes.  A is K-major (one 128-byte row per M row).  W is N-major: four boxes
-// of 64 N-columns x 64 K-rows, the leading-dimension offset is the box stride (8 KB),
-// and the stride offset is 8 K-rows (1 KB).
+// unit writes.  A is K-major (one 128-byte row per M row).  W is N-major: boxes of 64
+// N-columns x 64 K-rows; the leading-dimension offset is the box stride (8 KB), and the
+// stride offset is 8 K-rows (1 KB).
 #include <mutex>
 
 #include "bi_common.cuh"
@@ -51,7 +58,7 @@ struct Tile {
     static constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
 };
 
-struct Bars {
+struct Bars1 {
     uint64_t full[MAX_STAGES];
     uint64_t empty[MAX_STAGES];
     uint64_t tfull[2];   // accumulator b holds a finished tile
@@ -78,6 +85,8 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
     n_tile = r / gsm;
 }
 
+// ------------------------------------------------------------------ the single-CTA kernel
+// One CTA computes a 128 x 256 tile with tcgen05.mma.cta_group::1 (4-stage ring of 48 KB).
 template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
 bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
@@ -91,7 +100,7 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * A_STAGE;
-    Bars* bars = reinterpret_cast<Bars*>(sB + STAGES * B_STAGE);
+    Bars1* bars = reinterpret_cast<Bars1*>(sB + STAGES * B_STAGE);
     volatile int* abort = &bars->abort;
 
     const int warp = threadIdx.x >> 5;
@@ -254,6 +263,7 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
+
 
 // ------------------------------------------------------------------ the CTA-pair kernel
 // A 2-CTA cluster computes a 256 x 256 output tile with tcgen05.mma.cta_group::2: CTA r of the
@@ -513,13 +523,6 @@ bool ensure_smem_attr() {
     return ok[dev];
 }
 
-// The tile width for a weight of shape [K, N].  A function of (N, K) only, never of M, so every
-// batch size runs the same MMA shape and K order on every row.
-int plan_bn(int64_t N, int64_t K) {
-    (void)N; (void)K;
-    return 256;
-}
-
 // Launch the GEMM on operands with arbitrary (16-byte multiple) row strides: A [M, K] with
 // row stride lda, W [K, N] with row stride ldw, C [M, N] with row stride N.
 template <int BN>
@@ -575,10 +578,21 @@ int launch_gemm_pair(const void* A, int64_t lda, const void* W, int64_t ldw, voi
     return bi::launch_status();
 }
 
+// The plan for a weight of shape [K, N], a function of (N, K) and the device only, never of M:
+// CTA pairs when a row of 256-wide pair tiles fits the GPU's SM pairs (N <= 18944 on a B200),
+// single CTAs with 128 x 256 tiles for wider weights.  A wide weight then has enough column
+// tiles to occupy every SM at any M in one round, where pair tiles would need two rounds
+// for the small batches of decoding.
+bool use_pairs(int64_t N, int64_t K) {
+    (void)K;
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    return (N + pair::TILE_N - 1) / pair::TILE_N <= sms / 2;
+}
+
 int launch_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N, int64_t K,
                 bool c_bf16, cudaStream_t stream) {
-    (void)plan_bn;
-    return launch_gemm_pair(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
+    if (use_pairs(N, K)) return launch_gemm_pair(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
+    return launch_gemm_bn<256>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
 }
 
 int gemm_shape_checks(const void* A, const void* W, const void* C, int64_t M, int64_t N, int64_t K, int c_dtype) {
@@ -589,7 +603,8 @@ int gemm_shape_checks(const void* A, const void* W, const void* C, int64_t M, in
     if (!bi::aligned16(A) || !bi::aligned16(W) || !bi::aligned16(C)) return BI_ERR_MISALIGNED;
     if (K % 8 != 0 || N % 8 != 0) return BI_ERR_MISALIGNED;  // 16-byte row strides for the TMA unit
     if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return BI_ERR_UNSUPPORTED_SHAPE;
-    if (((M + BM - 1) / BM) * ((N + 63) / 64) > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N) > 0x7fffffffLL)
+        return BI_ERR_UNSUPPORTED_SHAPE;
     return BI_OK;
 }
 
@@ -615,14 +630,16 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, void* __res
     }
 }
 
-// The split a batch-size-adaptive library would pick: enough K slices to fill the GPU when
-// the batch alone yields too few output tiles (1, 2, 4 or 8, with K / S a multiple of 64).
+// The split a batch-size-adaptive library would pick: enough K slices to fill the GPU's SM
+// pairs when the batch alone yields too few output tiles (1, 2, 4 or 8, with K / S a multiple
+// of 64).
 int splitk_for(int64_t M, int64_t N, int64_t K) {
-    const int bn = plan_bn(N, K);
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + bn - 1) / bn);
-    const int sms = num_sms() > 0 ? num_sms() : 148;
+    const bool pairs = use_pairs(N, K);
+    const int64_t tm = pairs ? pair::TILE_M : BM, tn = 256;
+    const int64_t tiles = ((M + tm - 1) / tm) * ((N + tn - 1) / tn);
+    const int slots = (num_sms() > 0 ? num_sms() : 148) / (pairs ? 2 : 1);
     int S = 1;
-    while (S < 8 && tiles * S * 2 <= sms && K % ((int64_t)S * 2 * BK) == 0) S *= 2;
+    while (S < 8 && tiles * S * 2 <= slots && K % ((int64_t)S * 2 * BK) == 0) S *= 2;
     return S;
 }
 

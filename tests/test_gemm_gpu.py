@@ -18,6 +18,9 @@ from invariant_deterministic_rmsnorm_b200 import binding, harness, inputs
 pytestmark = pytest.mark.gpu
 
 LLAMA_SHAPES = [(4096, 6144), (4096, 14336), (14336, 4096)]  # (K, N)
+# the decoder's fused gate/up projection and its vocabulary projection: wider than a row of
+# 256-wide CTA-pair tiles can cover on one GPU, so they run on the single-CTA plan
+WIDE_SHAPES = [(4096, 28672), (4096, 32000)]
 
 
 def _gemm(A_np, W_np, out=torch.float32):
@@ -53,7 +56,7 @@ def test_parity_small_config(M):
     assert rel_frobenius(C, oracle.gemm(A, W)) <= 2e-3
 
 
-@pytest.mark.parametrize("K,N", LLAMA_SHAPES)
+@pytest.mark.parametrize("K,N", LLAMA_SHAPES + WIDE_SHAPES)
 @pytest.mark.parametrize("M", [1, 129, 257])
 def test_parity_llama_shapes_sampled_rows(K, N, M):
     A, W = inputs.gemm_case(M, N, K)
@@ -116,7 +119,7 @@ def _device_rows(seed: int, M: int, K: int) -> torch.Tensor:
     return torch.randn((M, K), generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("K,N", LLAMA_SHAPES + [(256, 512)])
+@pytest.mark.parametrize("K,N", LLAMA_SHAPES + [(256, 512)] + WIDE_SHAPES)
 def test_batch_invariance(K, N):
     W = dev(inputs.normal_bf16(inputs.SEED_WEIGHTS, (K, N), 0, 0.02))
     probes = dev(inputs.normal_bf16(inputs.SEED_PROBES, (8, K)))
