@@ -38,6 +38,7 @@ constexpr int SH_KC = 64;           // K per pipeline stage
 constexpr int SH_CWARPS = 8;        // compute warps
 constexpr int SH_THREADS = (SH_CWARPS + 1) * 32;
 constexpr int SH_MAX_STAGES = 6;
+constexpr int SH_MAX_SPLIT = 8;     // the largest cluster the shrink launches (portable cluster size)
 
 template <int R>
 struct ShrinkLayout {
@@ -172,12 +173,20 @@ lora_shrink_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
             for (int i = tid; i < SH_TM * R / 4; i += SH_THREADS) {
                 const uint32_t la = smem_u32(part + 4 * i);
                 float4 v = *reinterpret_cast<const float4*>(part + 4 * i);
-                for (int s = 1; s < split; ++s) {
-                    const float4 p = ld_dsmem_v4(mapa(la, (uint32_t)s));
-                    v.x = __fadd_rn(v.x, p.x);
-                    v.y = __fadd_rn(v.y, p.y);
-                    v.z = __fadd_rn(v.z, p.z);
-                    v.w = __fadd_rn(v.w, p.w);
+                // every peer's piece is requested before the first is used (one round trip, not
+                // split - 1); the adds below still run in slice order
+                float4 p[SH_MAX_SPLIT];
+#pragma unroll
+                for (int s = 1; s < SH_MAX_SPLIT; ++s)
+                    if (s < split) p[s] = ld_dsmem_v4(mapa(la, (uint32_t)s));
+#pragma unroll
+                for (int s = 1; s < SH_MAX_SPLIT; ++s) {
+                    if (s < split) {
+                        v.x = __fadd_rn(v.x, p[s].x);
+                        v.y = __fadd_rn(v.y, p[s].y);
+                        v.z = __fadd_rn(v.z, p[s].z);
+                        v.w = __fadd_rn(v.w, p[s].w);
+                    }
                 }
                 const int row = (4 * i) / R, col = (4 * i) % R;
                 if (m0 + row < M) *reinterpret_cast<float4*>(t + (size_t)(m0 + row) * R + col) = v;
