@@ -25,9 +25,9 @@
 //   t = S_j * scale * log2(e) (masked to -inf past the row's position)
 //   m' = m, or the block max when that exceeds m by more than 8 (then O and l are rescaled
 //        by 2^(m - m'), read from and written back to TMEM)
-//   p = 2^(t - m') (the hardware's approximate exp2);  l += sum p (a fixed summation tree);
-//   P = hi + lo, hi = p cut to bf16, lo = bf16(p - hi)
-// and out = O / l rounded to bf16.  Every decision above is row-local.  Blocks past a row's
+//   p = 2^(t - m') (one fused multiply-add, the hardware's approximate exp2);
+//   l += sum p (a fixed summation tree);  P = hi + lo, hi = p cut to bf16, lo = bf16(p - hi)
+// and out = O * (1 / l) rounded to bf16.  Every decision above is row-local.  Blocks past a row's
 // position contribute exact zeros: masked scores, zeroed values past the tile's last position.
 // So the rows a tile shares with a row never change its bits.
 #include <mutex>
@@ -294,17 +294,18 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 for (int c = 0; c < 32; ++c) sv[c] = __uint_as_float(r0[c]);
             }
             const int kpos0 = j * KB + half * 32;  // position of this thread's first key in the block
-            // scores in base-2 units: t = s * scale * log2(e); keys past the row's position are -inf.
-            // A warp whose rows all sit at or past its last key of the block needs no mask.
+            // scores in base-2 units are t = s * scale * log2(e); keys past the row's position are
+            // -inf.  A warp whose rows all sit at or past its last key of the block needs no mask.
+            // The multiply is monotone, so the block max of t is the scaled max of the raw scores.
             const bool unmasked = __all_sync(0xffffffffu, live && kpos0 + 31 <= qpos);
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                const float v = (unmasked || (live && kpos0 + c <= qpos)) ? __fmul_rn(sv[c], scale_log2) : -INFINITY;
+                const float v = (unmasked || (live && kpos0 + c <= qpos)) ? sv[c] : -INFINITY;
                 sv[c] = v;
                 mx4[c & 3] = fmaxf(mx4[c & 3], v);
             }
-            const float mine = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            const float mine = __fmul_rn(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])), scale_log2);
             bars->xmax[j & 1][half][r] = mine;
             __threadfence_block();
             __syncwarp();
@@ -343,7 +344,8 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             }
             if (need) l = __fmul_rn(l, c_fac);
             m_ref = m_new;
-            // p = 2^(t - m_ref); P = hi + lo with hi = p cut to bf16 (exact top 8 significant bits)
+            // p = 2^(s * scale * log2(e) - m_ref), one fused multiply-add and the hardware exp2;
+            // P = hi + lo with hi = p cut to bf16 (exact top 8 significant bits)
             // and lo = bf16(p - hi) (p - hi is exact in fp32); both go to the 128B-swizzled
             // K-major P tiles.  The partial row sum is four interleaved sums, added in a fixed order.
             const uint32_t row_off = (uint32_t)r * 128u;
@@ -353,8 +355,8 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 uint32_t ph[4], pl[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float p0 = ex2_approx(__fsub_rn(sv[cc * 8 + 2 * e], m_ref));
-                    const float p1 = ex2_approx(__fsub_rn(sv[cc * 8 + 2 * e + 1], m_ref));
+                    const float p0 = ex2_approx(__fmaf_rn(sv[cc * 8 + 2 * e], scale_log2, -m_ref));
+                    const float p1 = ex2_approx(__fmaf_rn(sv[cc * 8 + 2 * e + 1], scale_log2, -m_ref));
                     l4[e] = __fadd_rn(__fadd_rn(l4[e], p0), p1);
                     const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
                     ph[e] = __byte_perm(u0, u1, 0x7632);  // the top halves: bf16(p0) | bf16(p1) << 16, cut
@@ -403,6 +405,7 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
         if (ok) {
             tc_fence_after();
+            const float inv_l = __frcp_rn(l);  // out = O * (1 / l), one reciprocal per row
             __nv_bfloat16* dst = out + (int64_t)(q_row0 + r) * ldo + (int64_t)h * D + half * (D / 2);
 #pragma unroll 1
             for (int c = 0; c < D / 2; c += 32) {
@@ -413,8 +416,8 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        pk[i] = bi::pack_bf16x2(__fdiv_rn(__uint_as_float(o[2 * i]), l),
-                                                __fdiv_rn(__uint_as_float(o[2 * i + 1]), l));
+                        pk[i] = bi::pack_bf16x2(__fmul_rn(__uint_as_float(o[2 * i]), inv_l),
+                                                __fmul_rn(__uint_as_float(o[2 * i + 1]), inv_l));
 #pragma unroll
                     for (int i = 0; i < 16; i += 4)
                         *reinterpret_cast<uint4*>(dst + c + 2 * i) = make_uint4(pk[i], pk[i + 1], pk[i + 2], pk[i + 3]);
