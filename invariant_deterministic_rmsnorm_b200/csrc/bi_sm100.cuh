@@ -200,7 +200,7 @@ __device__ __forceinline__ uint32_t swz(uint32_t addr, uint32_t span_mask) {
 // (by columns) in its own shared memory, and each keeps its rows of D in its own TMEM.
 
 // Tile load into this CTA's shared memory whose completion bytes go to `bar`, a shared::cluster
-// address that may name the pair's leader CTA (no multicast: one destination, one source).
+// address that may name the pair's leader CTA (one destination CTA, one source tile).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, int32_t c0, int32_t c1,
                                                  uint32_t bar) {
     asm volatile(
