@@ -12,14 +12,14 @@
 // position q_pos0[b] + i.  Keys and values of sequence b are rows kv_indptr[b] + p of the packed
 // caches [tokens, Hkv, 128], for positions p = 0 .. position of the query (causal).
 //
-// One CTA per (128-row query tile of a sequence, query head), 6 warps:
+// One CTA per (128-row query tile of a sequence, query head), 18 warps:
 //   warp 0      TMA producer: the Q tile once, then K and V blocks of 64 positions into a
 //               3-stage ring
 //   warp 1      tcgen05.mma issuer (and TMEM owner):
 //                 S_j = Q K_j^T into one of two TMEM score buffers;
 //                 O += P_hi V_j + P_lo V_j into the TMEM output accumulator
-//   warps 2..9  softmax and epilogue, two threads per query row (TMEM lane): one takes the
-//               first 32 keys of each block and output dims 0..63, the other the rest
+//   warps 2..17 softmax and epilogue, four threads per query row (TMEM lane): thread p takes
+//               keys [16p, 16p + 16) of each block and output dims [32p, 32p + 32)
 // KV blocks of 64 positions, starting at position 0, are visited in ascending order.  For
 // block j, each row computes, in base-2 units:
 //   t = S_j * scale * log2(e) (masked to -inf past the row's position)
@@ -45,7 +45,11 @@ constexpr int D = 128;
 constexpr int QT = 128;               // query rows per CTA (the MMA's M)
 constexpr int KB = 64;                // keys per block
 constexpr int NST = 3;                // K/V ring stages
-constexpr int THREADS = 320;          // producer, MMA, 8 softmax warps
+constexpr int PARTS = 4;              // softmax threads per query row
+constexpr int SM_WARPS = 4 * PARTS;   // softmax warps (each TMEM lane quarter is read by PARTS warps)
+constexpr int THREADS = 32 * (2 + SM_WARPS);  // producer, MMA, softmax warps
+constexpr int KEYS_PER = KB / PARTS;  // keys of a block per softmax thread
+constexpr int DIMS_PER = D / PARTS;   // output dims per softmax thread
 constexpr int Q_BOX = 64 * QT * 2;    // 64 dims x 128 rows = 16 KB
 constexpr int KV_BOX = 64 * KB * 2;   // 64 dims x 64 keys = 8 KB
 constexpr int Q_BYTES = 2 * Q_BOX;    // 32 KB
@@ -64,9 +68,9 @@ struct Bars {
     uint64_t p_empty;  // PV_j done: the P tiles are free and O is stable
     uint64_t o_full;   // the last PV is done
     uint64_t drain;    // every MMA this CTA issued has completed
-    uint64_t xchg;     // the 8 softmax warps swapped their partial row maxima (or sums)
-    float xmax[2][2][QT];  // [block parity][half][row]
-    float xsum[2][QT];     // [half][row]
+    uint64_t xchg;     // the softmax warps swapped their partial row maxima (or sums)
+    float xmax[2][PARTS][QT];  // [block parity][part][row]
+    float xsum[PARTS][QT];     // [part][row]
     uint32_t tmem_addr;
     int abort;
 };
@@ -103,6 +107,15 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
            "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
            "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
+}
+// Each thread of the warp reads 16 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -157,11 +170,11 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
         mbar_init(smem_u32(&bars->s_full[0]), 1);
         mbar_init(smem_u32(&bars->s_full[1]), 1);
-        mbar_init(smem_u32(&bars->p_full), 8);
+        mbar_init(smem_u32(&bars->p_full), SM_WARPS);
         mbar_init(smem_u32(&bars->p_empty), 1);
         mbar_init(smem_u32(&bars->o_full), 1);
         mbar_init(smem_u32(&bars->drain), 1);
-        mbar_init(smem_u32(&bars->xchg), 8);
+        mbar_init(smem_u32(&bars->xchg), SM_WARPS);
         bars->abort = 0;
         fence_barrier_init();
         fence_proxy_async_shared();
@@ -266,13 +279,13 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
     } else {
         // ---------------------------------------------------------------- softmax + epilogue
-        // Two threads share a query row: `half` 0 takes keys 0..31 of every block and output
-        // dims 0..63, half 1 keys 32..63 and dims 64..127.  They swap their partial row maxima
-        // (and at the end their partial sums) through shared memory behind an mbarrier.
-        const int sw = warp - 2;             // softmax warp 0..7
-        const int half = sw >> 2;
-        const int quarter = warp & 3;        // this warp reads TMEM lanes 32*quarter .. +31
-        const int r = quarter * 32 + lane;   // query row of the tile
+        // PARTS threads share a query row: `part` p takes keys [16p, 16p + 16) of every block and
+        // output dims [32p, 32p + 32).  They swap their partial row maxima (and at the end their
+        // partial sums) through shared memory behind an mbarrier.
+        const int sw = warp - 2;              // softmax warp 0 .. SM_WARPS - 1
+        const int part = sw >> 2;
+        const int quarter = warp & 3;         // this warp reads TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;    // query row of the tile
         const bool live = r < n_q;
         const int qpos = pos0 + r;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -285,28 +298,28 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 break;
             }
             tc_fence_after();
-            float sv[32];
+            float sv[KEYS_PER];
             {
-                uint32_t r0[32];
-                tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(j & 1) * KB + (uint32_t)half * 32u, r0);
+                uint32_t r0[KEYS_PER];
+                tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(j & 1) * KB + (uint32_t)(part * KEYS_PER), r0);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; ++c) sv[c] = __uint_as_float(r0[c]);
+                for (int c = 0; c < KEYS_PER; ++c) sv[c] = __uint_as_float(r0[c]);
             }
-            const int kpos0 = j * KB + half * 32;  // position of this thread's first key in the block
+            const int kpos0 = j * KB + part * KEYS_PER;  // position of this thread's first key in the block
             // scores in base-2 units are t = s * scale * log2(e); keys past the row's position are
             // -inf.  A warp whose rows all sit at or past its last key of the block needs no mask.
             // The multiply is monotone, so the block max of t is the scaled max of the raw scores.
-            const bool unmasked = __all_sync(0xffffffffu, live && kpos0 + 31 <= qpos);
+            const bool unmasked = __all_sync(0xffffffffu, live && kpos0 + KEYS_PER - 1 <= qpos);
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < KEYS_PER; ++c) {
                 const float v = (unmasked || (live && kpos0 + c <= qpos)) ? sv[c] : -INFINITY;
                 sv[c] = v;
                 mx4[c & 3] = fmaxf(mx4[c & 3], v);
             }
             const float mine = __fmul_rn(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])), scale_log2);
-            bars->xmax[j & 1][half][r] = mine;
+            bars->xmax[j & 1][part][r] = mine;
             __threadfence_block();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->xchg));
@@ -315,7 +328,9 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_CLUSTER);
                 break;
             }
-            const float mx = fmaxf(mine, bars->xmax[j & 1][half ^ 1][r]);
+            float mx = bars->xmax[j & 1][0][r];
+#pragma unroll
+            for (int q = 1; q < PARTS; ++q) mx = fmaxf(mx, bars->xmax[j & 1][q][r]);
             float m_new = m_ref;
             if (m_ref == -INFINITY || mx > m_ref + RESCALE_GAP) m_new = fmaxf(m_ref, mx);
             const bool need = m_new != m_ref && m_ref != -INFINITY;
@@ -330,16 +345,13 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 tc_fence_after();
             }
             if (__any_sync(0xffffffffu, need)) {  // a warp-collective TMEM round trip; c_fac is 1 where not needed
-#pragma unroll 1
-                for (int c = 0; c < D / 2; c += 32) {
-                    const uint32_t col = O_COL + (uint32_t)(half * (D / 2) + c);
-                    uint32_t o[32];
-                    tmem_ld_32x32b_x32(tmem + lane_off + col, o);
-                    tmem_wait_ld();
+                const uint32_t col = O_COL + (uint32_t)(part * DIMS_PER);
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(tmem + lane_off + col, o);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), c_fac));
-                    tmem_st_32x32b_x32(tmem + lane_off + col, o);
-                }
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), c_fac));
+                tmem_st_32x32b_x32(tmem + lane_off + col, o);
                 tmem_wait_st();
             }
             if (need) l = __fmul_rn(l, c_fac);
@@ -351,7 +363,7 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const uint32_t row_off = (uint32_t)r * 128u;
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < KEYS_PER / 8; ++cc) {
                 uint32_t ph[4], pl[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -363,23 +375,23 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     pl[e] = bi::pack_bf16x2(__fsub_rn(p0, __uint_as_float(u0 & 0xFFFF0000u)),
                                             __fsub_rn(p1, __uint_as_float(u1 & 0xFFFF0000u)));
                 }
-                const int ch = half * 4 + cc;  // 16-byte chunk (8 keys) of the row
+                const int ch = part * (KEYS_PER / 8) + cc;  // 16-byte chunk (8 keys) of the row
                 const uint32_t off = row_off + ((uint32_t)(ch ^ (r & 7)) << 4);
                 st_shared_v4(sPh + off, ph[0], ph[1], ph[2], ph[3]);
                 st_shared_v4(sPl + off, pl[0], pl[1], pl[2], pl[3]);
             }
             l = __fadd_rn(l, __fadd_rn(__fadd_rn(l4[0], l4[1]), __fadd_rn(l4[2], l4[3])));
             // values past the tile's last position (another sequence's rows, or never written) are
-            // zeroed, so that a zero P never meets a non-finite V; half h clears box h of the row
-            const int vrow_pos = j * KB + r;
-            if (j * KB + KB - 1 > last_pos && r < KB && vrow_pos > last_pos) {
+            // zeroed, so that a zero P never meets a non-finite V; part p clears 64 of the row's 256 bytes
+            if (j * KB + KB - 1 > last_pos && r < KB && j * KB + r > last_pos) {
                 const int s = j % NST;
                 // the stage's copy completed before S_j was issued; this wait makes its bytes
                 // visible to this thread before they are overwritten
                 if (mbar_wait(smem_u32(&bars->kv_full[s]), (uint32_t)(j / NST) & 1u, abort)) {
-                    const uint32_t v0 = sV + (uint32_t)s * KV_BLOCK + (uint32_t)half * KV_BOX + (uint32_t)r * 128u;
+                    const uint32_t v0 = sV + (uint32_t)s * KV_BLOCK + (uint32_t)(part >> 1) * KV_BOX + (uint32_t)r * 128u +
+                                        (uint32_t)(part & 1) * 64u;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) st_shared_v4(v0 + q * 16, 0u, 0u, 0u, 0u);
+                    for (int q = 0; q < 4; ++q) st_shared_v4(v0 + q * 16, 0u, 0u, 0u, 0u);
                 } else {
                     fail(err, abort, bi::DEVERR_WAIT_FULL);
                 }
@@ -390,14 +402,16 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             if (lane == 0) mbar_arrive(smem_u32(&bars->p_full));
         }
         // ---------------------------------------------------------------- epilogue: out = O / l
-        if (ok) {  // the row sum: half 0's part plus half 1's part, in that order
-            bars->xsum[half][r] = l;
+        if (ok) {  // the row sum: the parts' sums added in part order
+            bars->xsum[part][r] = l;
             __threadfence_block();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars->xchg));
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->xchg), (uint32_t)nb & 1u, abort));
             if (!ok && lane == 0) fail(err, abort, bi::DEVERR_WAIT_CLUSTER);
-            l = __fadd_rn(bars->xsum[0][r], bars->xsum[1][r]);
+            l = bars->xsum[0][r];
+#pragma unroll
+            for (int q = 1; q < PARTS; ++q) l = __fadd_rn(l, bars->xsum[q][r]);
         }
         if (ok) {
             ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars->o_full), 0u, abort));
@@ -406,22 +420,19 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         if (ok) {
             tc_fence_after();
             const float inv_l = __frcp_rn(l);  // out = O * (1 / l), one reciprocal per row
-            __nv_bfloat16* dst = out + (int64_t)(q_row0 + r) * ldo + (int64_t)h * D + half * (D / 2);
-#pragma unroll 1
-            for (int c = 0; c < D / 2; c += 32) {
-                uint32_t o[32];
-                tmem_ld_32x32b_x32(tmem + lane_off + O_COL + (uint32_t)(half * (D / 2) + c), o);
-                tmem_wait_ld();
-                if (live) {
-                    uint32_t pk[16];
+            __nv_bfloat16* dst = out + (int64_t)(q_row0 + r) * ldo + (int64_t)h * D + part * DIMS_PER;
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(tmem + lane_off + O_COL + (uint32_t)(part * DIMS_PER), o);
+            tmem_wait_ld();
+            if (live) {
+                uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        pk[i] = bi::pack_bf16x2(__fmul_rn(__uint_as_float(o[2 * i]), inv_l),
-                                                __fmul_rn(__uint_as_float(o[2 * i + 1]), inv_l));
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = bi::pack_bf16x2(__fmul_rn(__uint_as_float(o[2 * i]), inv_l),
+                                            __fmul_rn(__uint_as_float(o[2 * i + 1]), inv_l));
 #pragma unroll
-                    for (int i = 0; i < 16; i += 4)
-                        *reinterpret_cast<uint4*>(dst + c + 2 * i) = make_uint4(pk[i], pk[i + 1], pk[i + 2], pk[i + 3]);
-                }
+                for (int i = 0; i < 16; i += 4)
+                    *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(pk[i], pk[i + 1], pk[i + 2], pk[i + 3]);
             }
         }
     }

@@ -192,3 +192,26 @@ def test_prefill_attention_layout_error_sets_bit():
     _run_prefill(q, k, v, ql, p0, bad_kb)
     assert binding.bi_get_device_error() & 0x800
     binding.bi_clear_device_error()
+
+
+def test_prefill_attention_ignores_non_finite_spare_rows():
+    """Cache rows outside every sequence's live positions hold NaN: the masked scores and the
+    zeroed value rows keep them out of every output, which must match the zero-filled case bit
+    for bit."""
+    q_lens, pos0 = [70, 129, 5], [0, 30, 200]
+    q, k, v, ql, p0, kb = _prefill_case(q_lens, pos0, seed=60, gap=100)
+    live = np.zeros(k.shape[0], bool)
+    for base, n in zip(kb, p0 + ql):
+        live[base:base + n] = True
+    k_nan, v_nan = k.copy(), v.copy()
+    k_nan[~live] = 0x7FC0
+    v_nan[~live] = 0x7FC0
+    k_zero, v_zero = k.copy(), v.copy()
+    k_zero[~live] = 0
+    v_zero[~live] = 0
+    got = _run_prefill(q, k_nan, v_nan, ql, p0, kb)
+    ref_bits = _run_prefill(q, k_zero, v_zero, ql, p0, kb)
+    assert np.isfinite(bf16_to_f64(got)).all()
+    assert np.array_equal(got, ref_bits)
+    ref = _oracle_prefill(q, k, v, ql, p0, kb)
+    assert rel_frobenius(bf16_to_f64(got), ref) <= 2e-3
