@@ -183,13 +183,15 @@ def build_ops(device, stream, attn_batch=None):
                     launch=lambda k: B.bi_rmsnorm(xs[k % R], w, y=xns[k % R], eps=EPS, stream=stream),
                     desc=f"x bf16 [{M},{H}] -> y bf16, w bf16 [{H}], eps 1e-6"))
 
-    def gemm_op(name, a_of_k, K, N, seed):
+    def gemm_op(name, a_of_k, K, N, seed, n_out=1):
+        """n_out > 1: consecutive steps write alternating output buffers (a step's result can then
+        be copied out while the next step runs)."""
         Wt = _to_dev(inputs.normal_bf16(seed, (K, N), 0.0, 0.02), device)
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        outs = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(n_out)]
         ops.append(dict(name=name, kind="tensor", work=2 * M * N * K, src="bi_gemm.cu",
-                        launch=lambda k: B.bi_gemm(a_of_k(k), Wt, C=out, stream=stream),
+                        launch=lambda k: B.bi_gemm(a_of_k(k), Wt, C=outs[k % n_out], stream=stream),
                         desc=f"A bf16 [{M},{K}] x W bf16 [{K},{N}] -> C bf16, fp32 accumulate"))
-        return out
+        return outs if n_out > 1 else outs[0]
 
     qkv = gemm_op("gemm_qkv", lambda k: xns[k % R], H, 6144, inputs.SEED_WEIGHTS + 10)
 
@@ -207,7 +209,7 @@ def build_ops(device, stream, attn_batch=None):
                     desc=f"q bf16 [{M},{H}] (row stride 6144) += bf16(t) [{M},{r}] x B bf16 [{r},{H}]"))
 
     up = gemm_op("gemm_up", lambda k: xns[k % R], H, 14336, inputs.SEED_WEIGHTS + 11)
-    down = gemm_op("gemm_down", lambda k: up, 14336, H, inputs.SEED_WEIGHTS + 12)
+    downs = gemm_op("gemm_down", lambda k: up, 14336, H, inputs.SEED_WEIGHTS + 12, n_out=2)
 
     # decode attention over a batch of requests with ragged cache lengths
     kv_len = inputs.kv_lengths(attn_batch)
@@ -216,18 +218,21 @@ def build_ops(device, stream, attn_batch=None):
     kc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
     vc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
     q_np = inputs.normal_bf16(inputs.SEED_X + 31, (attn_batch, 32, 128))
-    qa = _to_dev(q_np, device)
+    qas = [_to_dev(q_np, device) for _ in range(2)]  # alternate steps read alternate copies
+    qa = qas[0]
     ip_d = torch.tensor(indptr, dtype=torch.int32, device=device)
     ln_d = torch.tensor(kv_len, dtype=torch.int32, device=device)
     ws = torch.empty(B.bi_decode_attn_workspace_size(T, 32), dtype=torch.uint8, device=device)
-    attn_out = torch.empty((attn_batch, 32, 128), dtype=torch.bfloat16, device=device)
+    attn_outs = [torch.empty((attn_batch, 32, 128), dtype=torch.bfloat16, device=device) for _ in range(2)]
     kv_bytes = int(kv_len.sum()) * 8 * 128 * 2 * 2
     ops.append(dict(name="decode_attn", kind="hbm", work=kv_bytes + attn_batch * 32 * 128 * 4, src="bi_decode_attn.cu",
-                    launch=lambda k: B.bi_decode_attn(qa, kc, vc, ip_d, ln_d, out=attn_out, workspace=ws,
-                                                      stream=stream),
+                    launch=lambda k: B.bi_decode_attn(qas[k % 2], kc, vc, ip_d, ln_d, out=attn_outs[k % 2],
+                                                      workspace=ws, stream=stream),
                     desc=f"B={attn_batch} requests, kv lengths U[512,32768] (sum {int(kv_len.sum())}), 32 q / 8 kv "
                          f"heads, D=128, 256-token chunks", launches=2))
-    io = dict(h2d=[(xs[0], x_np), (qa, q_np)], d2h=[down, attn_out],
+    # per-step host traffic of the end-to-end pass: step k reads xs[k % R] and qas[k % 2] and
+    # writes downs[k % 2] and attn_outs[k % 2]
+    io = dict(h2d=[(xs, x_np), (qas, q_np)], d2h=[downs, attn_outs],
               attn=dict(q=qa, k=kc, v=vc, ip=ip_d, ln=ln_d, kv_len=kv_len, indptr=indptr))
     return ops, io
 
@@ -298,33 +303,58 @@ def run_ours(args, rank, world, local_rank):
     total_ms = t0.elapsed_time(t1)
     op_ms = [sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(K)) for i in range(len(ops))]
 
-    # end-to-end: pinned host inputs -> device, the same launches, device -> pinned host results
-    h_in = [(dst, torch.from_numpy(np.ascontiguousarray(src).view(np.int16) if src.dtype == np.uint16 else src)
-             .pin_memory()) for dst, src in io["h2d"]]
-    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in io["d2h"]]
+    # end-to-end: every step copies its inputs host -> device from pinned memory, runs the same
+    # launches and copies its results device -> host, through the C ABI.  The copies run on their
+    # own streams, one step ahead of (inputs) and one step behind (results) the compute, so that
+    # PCIe traffic overlaps the kernels.
+    def _bits(t):
+        return t.view(torch.int16) if t.dtype == torch.bfloat16 else t
+
+    h_in = [(dsts, torch.from_numpy(np.ascontiguousarray(src).view(np.int16) if src.dtype == np.uint16 else src)
+             .pin_memory()) for dsts, src in io["h2d"]]
+    h_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in srcs] for srcs in io["d2h"]]
     h2d_bytes = sum(t.numel() * t.element_size() for _, t in h_in)
-    d2h_bytes = sum(t.numel() * t.element_size() for t in h_out)
+    d2h_bytes = sum(srcs[0].numel() * srcs[0].element_size() for srcs in io["d2h"])
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
 
-    def e2e_step():
-        for dst, src in h_in:
-            dst.view(torch.int16 if dst.dtype == torch.bfloat16 else dst.dtype).copy_(src, non_blocking=True)
-        step(0)
-        for dst, src in zip(h_out, io["d2h"]):
-            dst.copy_(src, non_blocking=True)
+    def e2e_run(n):
+        """n steps; returns the device events that bracket them."""
+        done, copied = {}, {}
+        e_first = torch.cuda.Event(enable_timing=True)
+        e_last = torch.cuda.Event(enable_timing=True)
+        e_first.record(s_in)
+        for k in range(n):
+            loaded = torch.cuda.Event()
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(done[k - 2])  # the compute that last read these input buffers
+                for dsts, src in h_in:
+                    _bits(dsts[k % len(dsts)]).copy_(src, non_blocking=True)
+                loaded.record(s_in)
+            stream.wait_event(loaded)
+            if k >= 2:
+                stream.wait_event(copied[k - 2])  # the results in these output buffers are on the host
+            with torch.cuda.stream(stream):
+                step(k)
+            done[k] = torch.cuda.Event()
+            done[k].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[k])
+                for srcs, dsts in zip(io["d2h"], h_out):
+                    dsts[k % 2].copy_(srcs[k % 2], non_blocking=True)
+                copied[k] = torch.cuda.Event()
+                copied[k].record(s_out)
+        s_in.wait_stream(s_out)
+        s_in.wait_stream(stream)
+        e_last.record(s_in)
+        return e_first, e_last
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(K):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+    e2e_run(max(1, args.warmup))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = e2e_run(K)
+    torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
     # batch-invariance spot check and the invariance tax, outside the timed region
