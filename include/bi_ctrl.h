@@ -62,6 +62,15 @@ int bi_ctrl_decode_attn_adaptive(const void* q, const void* k, const void* v, co
                                  const int32_t* kv_len, int32_t B, int64_t total_tokens, int32_t Hq, int32_t Hkv,
                                  float scale, void* out, int out_dtype, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * bi_ctrl_wait_timeout_probe -- exercises the failure path that every kernel's bounded waits
+ * share, without a fault.  One CTA waits on an mbarrier that nothing arrives on.  After
+ * limit_ns (1 us .. 2 s) the wait gives up, bit 0x2 is OR-ed into the device error word
+ * (bi_get_device_error), and the kernel returns.  The CUDA context stays usable.  Tests use
+ * it to check the path from a device-side timeout to the host-visible status.
+ */
+int bi_ctrl_wait_timeout_probe(uint64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -65,6 +65,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_ctrl_gemm_splitk": ([P, P, P, I64, I64, I64, C, P, Z, P], C),
         "bi_ctrl_decode_attn_adaptive_workspace_size": ([I64, I32], Z),
         "bi_ctrl_decode_attn_adaptive": ([P, P, P, P, P, I32, I64, I32, I32, F, P, C, P, Z, P], C),
+        "bi_ctrl_wait_timeout_probe": ([ctypes.c_uint64, P], C),
         # include/bi_model.h
         "bi_embed": ([P, P, P, I64, I64, I64, P], C),
         "bi_rope_table": ([P, I64, I32, ctypes.c_double, P], C),
@@ -448,6 +449,11 @@ def bi_ctrl_decode_attn_adaptive(q, k, v, kv_indptr, kv_len, out=None, scale=Non
                                           ws.numel() * ws.element_size(), _stream(stream))
     _check("bi_ctrl_decode_attn_adaptive", st)
     return out
+
+
+def bi_ctrl_wait_timeout_probe(limit_ns: int = 1_000_000, stream=None) -> None:
+    """Launch the one-CTA probe whose bounded wait must run out after limit_ns (sets bit 0x2)."""
+    _check("bi_ctrl_wait_timeout_probe", library().bi_ctrl_wait_timeout_probe(int(limit_ns), _stream(stream)))
 
 
 def bi_get_device_error(stream=None) -> int:

@@ -2,8 +2,24 @@
 #include <atomic>
 
 #include "bi_common.cuh"
+#include "bi_ctrl.h"
+#include "bi_sm100.cuh"
 
 namespace {
+
+// One CTA waits, with the kernels' bounded wait, on an mbarrier that nothing arrives on.  The
+// wait must give up after limit_ns; the kernel then reports it the way every kernel reports a
+// wait that ran out, and returns.
+__global__ void wait_probe_kernel(uint64_t limit_ns, uint32_t* err) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        bi::sm100::mbar_init(bi::sm100::smem_u32(&bar), 1);
+        bi::sm100::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !bi::sm100::mbar_wait_ns(bi::sm100::smem_u32(&bar), 0u, nullptr, limit_ns))
+        atomicOr(err, bi::DEVERR_WAIT_FULL);
+}
 
 // One word per device.  Kernels whose bounded waits run out OR a cause bit into it.
 __device__ uint32_t g_device_error;
@@ -63,4 +79,12 @@ BI_API int bi_clear_device_error(void* stream) {
     uint32_t* word = bi::device_error_word();
     if (!word) return BI_ERR_CUDA;
     return cudaMemsetAsync(word, 0, sizeof(uint32_t), bi::as_stream(stream)) == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+BI_API int bi_ctrl_wait_timeout_probe(uint64_t limit_ns, void* stream) {
+    if (limit_ns < 1000ull || limit_ns > 2000000000ull) return BI_ERR_INVALID_ARG;
+    uint32_t* err = bi::device_error_word();
+    if (!err) return BI_ERR_CUDA;
+    wait_probe_kernel<<<1, 32, 0, bi::as_stream(stream)>>>(limit_ns, err);
+    return bi::launch_status();
 }

@@ -55,17 +55,21 @@ __device__ __forceinline__ bool mbar_test_parity(uint32_t bar, uint32_t parity) 
 }
 
 // Wait until the phase with the given parity has completed.  Gives up (returns false)
-// after kWaitLimitNs, or early once *abort becomes non-zero.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort) {
+// after limit_ns, or early once *abort becomes non-zero.
+__device__ __forceinline__ bool mbar_wait_ns(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                             uint64_t limit_ns) {
     if (mbar_test_parity(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_test_parity(bar, parity)) return true;
         if ((it & 63u) == 0) {
             if (abort != nullptr && *abort) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) return false;
+            if (globaltimer() - t0 > limit_ns) return false;
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort) {
+    return mbar_wait_ns(bar, parity, abort, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- TMA
