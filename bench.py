@@ -54,9 +54,6 @@ ATTN_BATCH = 64
 TRAFFIC = {
     "decode_attn": ("0f1b7b70a1d6d502", 4050480640 + 63069184 + 64504064 + 3840,
                     "decode_attn_chunk_kernel + decode_attn_merge_kernel, B=64 (the step's decode batch)"),
-    "gemm_qkv": ("ea55668dfee15267", 123656704 + 27717120, "bi_gemm_bf16_tc_kernel<256>, M=4096 K=4096 N=6144"),
-    "gemm_up": ("ea55668dfee15267", 269734144 + 91232256, "bi_gemm_bf16_tc_kernel<256>, M=4096 K=4096 N=14336"),
-    "gemm_down": ("ea55668dfee15267", 547947520 + 28950016, "bi_gemm_bf16_tc_kernel<256>, M=4096 K=14336 N=4096"),
 }
 
 
