@@ -731,6 +731,26 @@ def run_sweep(args):
                           "bi_frac_burst": round(fl / (t_bi / 1e3) / peaks["bf16_tflops"], 3)})
             del Ws, As, Cs
         emit({"op": "gemm", "K": K, "N": N, "rows": table})
+    # the GEMM plan's K split: every split count on the narrow projections (QKV, O, down)
+    for K, N in (((4096, 6144), (4096, 4096), (14336, 4096)) if "gemm-split" in only else ()):
+        table = []
+        for M in (8, 64, 256, 512, 1024, 2048, 4096, 8192):
+            R = _copies(2 * (M * K + K * N + M * N))
+            Ws = [rows_dev(50 + j, K, N).mul_(0.02) for j in range(R)]
+            As = [rows_dev(60 + j, M, K) for j in range(R)]
+            Cs = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(R)]
+            ws = torch.zeros(max(lib.bi_ctrl_gemm_split_workspace_size(M, N, K, S) for S in range(1, 5)) + 16,
+                             dtype=torch.uint8, device=device)
+            fl = 2 * M * N * K / 1e12
+            row = {"M": M, "plan": B.gemm_splits(N, K)}
+            for S in range(1, 5):
+                t = _time_graph([lambda j=j, S=S: B.bi_ctrl_gemm_split(As[j], Ws[j], S, C=Cs[j], workspace=ws,
+                                                                       stream=stream) for j in range(R)], stream)
+                row[f"s{S}_us"] = round(t * 1e3, 2)
+                row[f"s{S}_tflops"] = round(fl / (t / 1e3), 1)
+            table.append(row)
+            del Ws, As, Cs, ws
+        emit({"op": "gemm-split", "K": K, "N": N, "rows": table})
     # RMSNorm
     table = []
     w = _to_dev(inputs.rmsnorm_case(1, HIDDEN, "bf16")[1], device)
@@ -1050,7 +1070,7 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="print per-op throughput across batch sizes (one GPU) instead of the benchmark line")
     ap.add_argument("--sweep-ops", nargs="+", default=["gemm", "rmsnorm", "lora", "attn"],
-                    choices=["gemm", "rmsnorm", "lora", "attn"], help="ops the sweep covers")
+                    choices=["gemm", "gemm-split", "rmsnorm", "lora", "attn"], help="ops the sweep covers")
     ap.add_argument("--attn-batch", type=int, default=ATTN_BATCH,
                     help="decode requests in the step (smaller for profiler captures)")
     ap.add_argument("--decoder", action="store_true",

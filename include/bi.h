@@ -66,7 +66,8 @@ int bi_abi_version(void);
  * (0 = no error).  Return value: BI_OK, BI_ERR_TIMEOUT if *code != 0, or
  * BI_ERR_CUDA.  bi_clear_device_error() zeroes the word, ordered on `stream`.
  * Bits: 0x1 a producer's wait for a free stage, 0x2 a wait for a loaded stage,
- * 0x4 a wait for the accumulator, 0x8 a cluster handshake; 0x100 decode-attention
+ * 0x4 a wait for the accumulator, 0x8 a cluster handshake, 0x10 a GEMM's last K slice
+ * waiting for the other slices of its tile; 0x100 decode-attention
  * layout, 0x200 embedding token id, 0x400 KV-append destination row, 0x800
  * prefill-attention layout, 0x1000 RoPE position (the last five are input checks made on
  * the device).
@@ -112,16 +113,36 @@ int bi_rmsnorm(const void* x, const void* w, void* y, int64_t M, int64_t H, int6
  *   C    device, [M, N] row-major, dtype c_dtype (BI_F32: the fp32 accumulator as is;
  *        BI_BF16: the accumulator rounded to nearest even)
  *   M    >= 0 rows.  N, K > 0, multiples of 8 (16-byte rows for the TMA unit).
- *        M <= 65535*128.
- *   ws, ws_bytes  workspace, at least bi_gemm_workspace_size(M, N, K) bytes.  That
- *        size is 0 for every shape this version supports, so ws may be NULL.
+ *   ws, ws_bytes  workspace of at least bi_gemm_workspace_size(M, N, K) bytes, 16-byte
+ *        aligned; NULL is accepted when that size is 0, as it is for every shape in this
+ *        version (the plan does not split K).  A plan that splits K uses it like this:
+ *          - its first bi_gemm_counter_bytes(M, N, K) bytes are counters.  They must be
+ *            zero when the call starts, and a call that completes leaves them zero.
+ *            Zero-fill a new workspace once.  After a call that set a device error bit,
+ *            zero it again before reuse.
+ *          - fp32 partial sums are written to the last bytes of the buffer.
+ *          - several calls may share one workspace when no call's partials can reach
+ *            another call's counters: ws_bytes >= the largest counter bytes plus the
+ *            largest partial bytes among them.  Calls that run concurrently need
+ *            separate workspaces.
+ *        BI_ERR_WORKSPACE if the workspace is missing or too small.
  *
- * Arithmetic: tcgen05.mma 128x256x16, bf16 x bf16 -> fp32 in tensor memory.  The tile
- * is 128 rows x 256 columns and K is walked in ascending 64-wide blocks.  The plan
- * (tile, MMA shape, K order, split count) is a function of (N, K) only.  Rows past M
- * and columns past N or K are zero-filled on load and never stored.  C may not
- * alias A or W.
+ * Arithmetic: bf16 x bf16 -> fp32 in tensor memory, K walked in ascending 64-wide
+ * blocks.  The plan (tile, MMA shape, K order, split count) is a function of (N, K) and
+ * the device only:
+ *   - N <= 256 x (SM pairs): 256 x 256 tiles on 2-CTA clusters,
+ *     tcgen05.mma.cta_group::2 256x256x16.  The kernel can split K into S contiguous
+ *     slices; slice s accumulates its K blocks in fp32, and the output is
+ *     ((P0 + P1) + ...) + P(S-1), summed in that order in fp32.  The plan's
+ *     S = bi_gemm_splits(N, K) is 1 for every shape: a split pays only while M fills one or
+ *     two rows of tiles and costs more than it saves at larger M.  bi_ctrl_gemm_split runs
+ *     other S.
+ *   - wider N: 128 x 256 tiles on one CTA, tcgen05.mma.cta_group::1 128x256x16, no split.
+ * Rows past M and columns past N or K are zero-filled on load and never stored.  C may
+ * not alias A or W.
  */
+int bi_gemm_splits(int64_t N, int64_t K);
+size_t bi_gemm_counter_bytes(int64_t M, int64_t N, int64_t K);
 size_t bi_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype, void* ws,
             size_t ws_bytes, void* stream);

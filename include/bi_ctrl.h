@@ -42,13 +42,27 @@ int bi_ctrl_rmsnorm_split(const void* x, const void* w, void* y, int64_t M, int6
  * bi_ctrl_gemm_splitk -- bi_gemm with a split-K chosen from M, the batch-size-dependent
  * strategy of the "Multiplicación de matrices" section of the same page.  When the batch
  * alone yields too few output tiles to fill the GPU, K is cut into S in {2, 4, 8} slices.
- * Each slice is a bi_gemm into fp32 partials in ws.  The partials are then added in slice
- * order and rounded to c_dtype.  A row's accumulation order therefore depends on M.
+ * Each slice runs bi_gemm's tile kernel unsplit into fp32 partials in ws (S = 1: the whole
+ * product, straight into C).  The partials are then added in slice order and rounded to
+ * c_dtype.  A row's accumulation order therefore depends on M.
  * ws must hold bi_ctrl_gemm_splitk_workspace_size(M, N, K) bytes (0 when S = 1).
  */
 size_t bi_ctrl_gemm_splitk_workspace_size(int64_t M, int64_t N, int64_t K);
 int bi_ctrl_gemm_splitk(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype,
                         void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * bi_ctrl_gemm_split -- bi_gemm with the K split count given by the caller instead of
+ * bi_gemm_splits(N, K): the plan study behind that choice.  For a fixed `splits` it is
+ * batch-invariant like bi_gemm; it is here to time the plan's candidates against each
+ * other at every batch size.  splits in 1 .. 4 and at most ceil(K / 64); a weight too wide
+ * for the CTA-pair tiles takes splits = 1 only (BI_ERR_UNSUPPORTED_SHAPE otherwise).
+ * The workspace follows bi_gemm's rules, with bi_ctrl_gemm_split_workspace_size bytes
+ * (counters first, bi_gemm_counter_bytes' layout).
+ */
+size_t bi_ctrl_gemm_split_workspace_size(int64_t M, int64_t N, int64_t K, int32_t splits);
+int bi_ctrl_gemm_split(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype,
+                       int32_t splits, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * bi_ctrl_decode_attn_adaptive -- bi_decode_attn with the split size chosen from the

@@ -11,10 +11,14 @@
 //   - N up to 256 x (SM pairs) (18944 on a B200): 256 x 256 tiles over a 2-CTA cluster,
 //     tcgen05.mma.cta_group::2 256 x 256 x 16;
 //   - wider N: 128 x 256 tiles on one CTA, tcgen05.mma.cta_group::1 128 x 256 x 16.
-// In both, the K-block order is ascending (64 at a time) and the split count is 1.  A row's
-// tile position and the batch size M change which CTA computes the row.  They never change
-// the instructions that produce its bits.  Rows past M are zero-filled by the TMA unit and
-// are never stored.
+// In both, the K-block order is ascending (64 at a time).  The pair kernel can also split K into
+// S contiguous slices: slice s of a tile accumulates its K blocks in TMEM like an unsplit
+// tile, slices 0 .. S-2 store fp32 partials, and slice S-1 adds them in slice order,
+// ((P0 + P1) + ...) + P(S-1), before the output rounding.  The slices meet through integer
+// counters; no floating-point atomic is used.  The plan's S is 1 (splits_for); other S run
+// through bi_ctrl_gemm_split.  A row's tile position and the batch size M change which CTA
+// computes the row.  They never change the instructions that produce its bits.  Rows past M
+// are zero-filled by the TMA unit and are never stored.
 //
 // CTA structure (192 threads; in the pair kernel two CTAs per cluster):
 //   warp 0      TMA producer.  Pair kernel: 128 rows of A [128 x 64] and 128 columns of W
@@ -70,6 +74,35 @@ struct Bars1 {
 __device__ __forceinline__ void fail(uint32_t* err, volatile int* abort, uint32_t bit) {
     atomicOr(err, bit);
     *abort = 1;
+}
+
+// Split-K meeting point.  Every lane of a writer warp fences its partial-row stores, and after
+// the warp has met, one lane increments the counter.  The last slice waits until the counter
+// holds `target`, then zeroes it for the next call.  Bounded: false after kWaitLimitNs.
+__device__ __forceinline__ void split_signal(uint32_t* cnt, int lane) {
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) atomicAdd(cnt, 1u);
+}
+
+__device__ __forceinline__ bool split_wait(uint32_t* cnt, uint32_t target) {
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        if (v == target) {
+            asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(cnt), "r"(0u) : "memory");
+            return true;
+        }
+        if (globaltimer() - t0 > kWaitLimitNs) return false;
+        __nanosleep(128);
+    }
+}
+
+__device__ __forceinline__ float4 ld_partial(const float* p) {
+    float4 r;
+    asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
+    return r;
 }
 
 // Tile order: groups of `gm` row tiles, walked column by column inside a group, so that the
@@ -294,11 +327,17 @@ struct Bars {
     int abort;
 };
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * ST_BYTES + sizeof(Bars) + 64;
+constexpr int MAX_SPLIT = 4;                 // K slices per tile at most
+constexpr int CNT_PER_TILE = 2 * EPI_WARPS;  // one split counter per (CTA, epilogue warp)
 }  // namespace pair
 
+// SPLIT = false is the unsplit kernel (splits must be 1; cnt and part are unused).
+template <bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
-                         void* __restrict__ C, int M, int N, int K, int c_bf16, int gm, uint32_t* err) {
+                         void* __restrict__ C, int M, int N, int K, int c_bf16, int gm, int splits_arg,
+                         uint32_t* __restrict__ cnt, float* __restrict__ part, uint32_t* err) {
+    const int splits = SPLIT ? splits_arg : 1;
     using pair::ROWS;
     using pair::COLS;
     using pair::TILE_M;
@@ -324,6 +363,9 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     const int tiles_n = (N + TILE_N - 1) / TILE_N;
     const int num_tiles = tiles_m * tiles_n;
     const int num_kb = (K + BK - 1) / BK;
+    // work unit u = (tile u / splits, K slice u % splits); the slices of a tile are adjacent,
+    // so they run side by side on neighbouring pairs
+    const int num_units = num_tiles * splits;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -356,11 +398,13 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     if (warp == 0) {
         if (lane == 0) {
             uint32_t it = 0;  // k-blocks issued by this CTA so far (the ring runs across tiles)
-            for (int t = pair_id; t < num_tiles && !*abort; t += n_pairs) {
+            for (int u = pair_id; u < num_units && !*abort; u += n_pairs) {
+                const int t = u / splits, sl = u - t * splits;
                 int mt, nt;
                 tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
                 const int m0 = mt * TILE_M + (int)rank * ROWS, n0 = nt * TILE_N + (int)rank * COLS;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int kb1 = (int)((int64_t)(sl + 1) * num_kb / splits);
+                for (int kb = (int)((int64_t)sl * num_kb / splits); kb < kb1; ++kb, ++it) {
                     const int s = (int)(it % STAGES);
                     const uint32_t round = it / STAGES;
                     if (!mbar_wait(smem_u32(&bars->empty[s]), (round & 1u) ^ 1u, abort)) {
@@ -394,7 +438,9 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             const uint32_t peer_empty0 = mapa(smem_u32(&bars->empty[0]), 1);
             const uint32_t peer_tfull0 = mapa(smem_u32(&bars->tfull[0]), 1);
             uint32_t it = 0, local = 0;
-            for (int t = pair_id; t < num_tiles && !*abort; t += n_pairs, ++local) {
+            for (int u = pair_id; u < num_units && !*abort; u += n_pairs, ++local) {
+                const int t = u / splits, sl = u - t * splits;
+                const int kb0 = (int)((int64_t)sl * num_kb / splits), kb1 = (int)((int64_t)(sl + 1) * num_kb / splits);
                 const uint32_t acc = local & 1u, use = local >> 1;
                 if (!mbar_wait(smem_u32(&bars->tempty[acc]), (use & 1u) ^ 1u, abort)) {
                     fail(err, abort, bi::DEVERR_WAIT_ACCUM);
@@ -402,7 +448,7 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = (int)(it % STAGES);
                     const uint32_t round = it / STAGES;
                     if (!mbar_wait(smem_u32(&bars->full[s]), round & 1u, abort)) {
@@ -416,7 +462,7 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint64_t adesc = make_smem_desc(a_base + k * UMMA_K * 2, 16, 1024, 2);
                         const uint64_t bdesc = make_smem_desc(b_base + k * UMMA_K * 128, B_BOX, 1024, 2);
-                        mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+                        mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
                     }
                     // stage s of both CTAs is free once these MMAs have read it
                     mma_commit_pair(smem_u32(&bars->empty[s]));
@@ -431,8 +477,10 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     } else {
         const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter .. +31
         const uint32_t tempty0 = rank == 0 ? smem_u32(&bars->tempty[0]) : mapa(smem_u32(&bars->tempty[0]), 0);
+        const int64_t slice_elems = (int64_t)M * N;  // one slice's fp32 partial, [M, N] row-major
         uint32_t local = 0;
-        for (int t = pair_id; t < num_tiles; t += n_pairs, ++local) {
+        for (int u = pair_id; u < num_units; u += n_pairs, ++local) {
+            const int t = u / splits, sl = u - t * splits;
             const uint32_t acc = local & 1u, use = local >> 1;
             const bool ok = mbar_wait(smem_u32(&bars->tfull[acc]), use & 1u, abort);
             if (!ok) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
@@ -441,10 +489,41 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             tc_fence_after();
             int mt, nt;
             tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
-            const int row = mt * TILE_M + (int)rank * ROWS + quarter * 32 + lane;
+            const int row0 = mt * TILE_M + (int)rank * ROWS + quarter * 32;
+            const int row = row0 + lane;
+            // Split K: the S slices' copies of this warp's 32 rows meet through one counter.  A
+            // warp whose rows all lie past M neither stores nor waits, in every slice alike.
+            const bool split = SPLIT && splits > 1 && row0 < M;
+            const bool last = sl == splits - 1;
+            uint32_t* my_cnt = cnt + (int64_t)t * pair::CNT_PER_TILE + (int)rank * EPI_WARPS + quarter;
+            if (split && last) {
+                bool ready = true;
+                if (lane == 0) ready = split_wait(my_cnt, (uint32_t)(splits - 1));
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                __threadfence();  // every lane's partial loads below come after lane 0's acquire
+                if (!ready) {
+                    if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_SPLIT);
+                    break;
+                }
+            }
             const uint32_t lane_addr = tmem_base + acc * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
             for (int c = 0; c < TILE_N; c += 32) {
+                const int col = nt * TILE_N + c;
+                const bool live = row < M && col < N;
+                const int nv = live ? min(32, N - col) : 0;  // a multiple of 8 (N % 8 == 0)
+                // the last slice issues its loads of the earlier partials before reading TMEM
+                float4 pv[(pair::MAX_SPLIT - 1) * 8];
+                if (split && last) {
+#pragma unroll
+                    for (int j = 0; j < pair::MAX_SPLIT - 1; ++j) {
+                        const float* src = part + j * slice_elems + (int64_t)row * N + col;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pv[j * 8 + i] = (j < splits - 1 && 4 * i < nv) ? ld_partial(src + 4 * i)
+                                                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(lane_addr + (uint32_t)c, r);
                 tmem_wait_ld();
@@ -453,37 +532,66 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8u);
                 }
-                const int col = nt * TILE_N + c;
-                if (row < M && col < N) {
-                    if (!c_bf16) {
-                        float* dst = static_cast<float*>(C) + (int64_t)row * N + col;
-                        if (col + 32 <= N) {
+                if (!live) continue;
+                if (split && !last) {  // an earlier slice: store the fp32 partial as it stands
+                    float* dst = part + sl * slice_elems + (int64_t)row * N + col;
 #pragma unroll
-                            for (int i = 0; i < 32; i += 4)
-                                *reinterpret_cast<uint4*>(dst + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
-                        } else {
+                    for (int i = 0; i < 8; ++i)
+                        if (4 * i < nv)
+                            *reinterpret_cast<uint4*>(dst + 4 * i) =
+                                make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+                    continue;
+                }
+                if (split) {  // the last slice: ((P0 + P1) + ...) + this slice's accumulator
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (i < N - col) dst[i] = __uint_as_float(r[i]);
+                    for (int j = 1; j < pair::MAX_SPLIT - 1; ++j) {
+                        if (j < splits - 1) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                pv[i].x = __fadd_rn(pv[i].x, pv[j * 8 + i].x);
+                                pv[i].y = __fadd_rn(pv[i].y, pv[j * 8 + i].y);
+                                pv[i].z = __fadd_rn(pv[i].z, pv[j * 8 + i].z);
+                                pv[i].w = __fadd_rn(pv[i].w, pv[j * 8 + i].w);
+                            }
                         }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        r[4 * i] = __float_as_uint(__fadd_rn(pv[i].x, __uint_as_float(r[4 * i])));
+                        r[4 * i + 1] = __float_as_uint(__fadd_rn(pv[i].y, __uint_as_float(r[4 * i + 1])));
+                        r[4 * i + 2] = __float_as_uint(__fadd_rn(pv[i].z, __uint_as_float(r[4 * i + 2])));
+                        r[4 * i + 3] = __float_as_uint(__fadd_rn(pv[i].w, __uint_as_float(r[4 * i + 3])));
+                    }
+                }
+                if (!c_bf16) {
+                    float* dst = static_cast<float*>(C) + (int64_t)row * N + col;
+                    if (col + 32 <= N) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<uint4*>(dst + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
                     } else {
-                        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(C) + (int64_t)row * N + col;
-                        uint32_t p[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            p[i] = bi::pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                        if (col + 32 <= N) {
+                        for (int i = 0; i < 32; ++i)
+                            if (i < N - col) dst[i] = __uint_as_float(r[i]);
+                    }
+                } else {
+                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(C) + (int64_t)row * N + col;
+                    uint32_t p[16];
 #pragma unroll
-                            for (int i = 0; i < 16; i += 4)
-                                *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(p[i], p[i + 1], p[i + 2], p[i + 3]);
-                        } else {
+                    for (int i = 0; i < 16; ++i)
+                        p[i] = bi::pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                    if (col + 32 <= N) {
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (i < N - col) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
-                        }
+                        for (int i = 0; i < 16; i += 4)
+                            *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(p[i], p[i + 1], p[i + 2], p[i + 3]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i < N - col) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
                     }
                 }
             }
+            if (split && !last) split_signal(my_cnt, lane);  // this warp's partial rows are stored
         }
     }
 
@@ -547,20 +655,80 @@ int launch_gemm_bn(const void* A, int64_t lda, const void* W, int64_t ldw, void*
     return bi::launch_status();
 }
 
-// The CTA-pair kernel: 256 x 256 tiles over 2-CTA clusters, one cluster per SM pair at most.
-int launch_gemm_pair(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N,
-                     int64_t K, bool c_bf16, cudaStream_t stream) {
-    uint32_t* err = bi::device_error_word();
-    if (!err) return BI_ERR_CUDA;
+// Shared-memory attribute of both pair-kernel instantiations (once per device).
+bool pair_smem_attr() {
     static std::once_flag once[64];
-    static bool attr_ok[64];
+    static bool ok[64];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BI_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::call_once(once[dev], [&] {
-        attr_ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)pair::SMEM_BYTES) == cudaSuccess;
+        ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)pair::SMEM_BYTES) == cudaSuccess &&
+                  cudaFuncSetAttribute(bi_gemm_bf16_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)pair::SMEM_BYTES) == cudaSuccess;
     });
-    if (!attr_ok[dev]) return BI_ERR_CUDA;
+    return ok[dev];
+}
+
+// Clusters of the split pair kernel that fit on the device at once (cached per device).  A
+// split grid never exceeds it: the last K slice of a tile waits for the other slices, so
+// every cluster must be resident together.
+int pair_clusters() {
+    static std::once_flag once[64];
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (!pair_smem_attr()) return -1;
+    std::call_once(once[dev], [&] {
+        cached[dev] = -1;
+        const int sms = num_sms();
+        if (sms < 2) return;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(sms & ~1));
+        cfg.blockDim = dim3(THREADS);
+        cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, bi_gemm_bf16_pair_kernel<true>, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return;
+        }
+        if (n <= 0) return;
+        cached[dev] = n < sms / 2 ? n : sms / 2;
+    });
+    return cached[dev];
+}
+
+// Workspace of a pair-kernel call with S > 1 slices: counters at the start (zero between
+// calls), fp32 partials of slices 0 .. S-2 at the end.
+size_t split_counter_bytes(int64_t M, int64_t N) {
+    const int64_t tiles = ((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N);
+    return (size_t)(((tiles * pair::CNT_PER_TILE * 4) + 255) / 256 * 256);
+}
+size_t split_partial_bytes(int64_t M, int64_t N, int S) { return (size_t)(S - 1) * M * N * sizeof(float); }
+
+// The CTA-pair kernel: 256 x 256 tiles over 2-CTA clusters, one cluster per SM pair at most,
+// K split into `splits` slices.
+int launch_gemm_pair(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N,
+                     int64_t K, bool c_bf16, int splits, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    uint32_t* err = bi::device_error_word();
+    if (!err || !pair_smem_attr()) return BI_ERR_CUDA;
+    if (splits < 1 || splits > pair::MAX_SPLIT || splits > (K + BK - 1) / BK) return BI_ERR_INVALID_ARG;
+    const int sms = num_sms();
+    if (sms < 2) return BI_ERR_CUDA;
+    int64_t clusters = sms / 2;
+    if (splits > 1) {
+        const int c = pair_clusters();
+        if (c <= 0) return BI_ERR_CUDA;
+        if (c < clusters) clusters = c;
+    }
+    uint32_t* cnt = nullptr;
+    float* part = nullptr;
+    if (splits > 1) {
+        const size_t cb = split_counter_bytes(M, N), pb = split_partial_bytes(M, N, splits);
+        if (!ws || !bi::aligned16(ws) || ws_bytes < cb + pb) return BI_ERR_WORKSPACE;
+        cnt = static_cast<uint32_t*>(ws);
+        part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + (ws_bytes - pb) / 16 * 16);
+    }
     CUtensorMap tmA, tmW;
     if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK,
                           pair::ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -568,13 +736,18 @@ int launch_gemm_pair(const void* A, int64_t lda, const void* W, int64_t ldw, voi
     if (!bi::make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)N, (uint64_t)K, (uint64_t)ldw * 2, 64,
                           BK, CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
-    const int64_t tiles = ((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N);
-    const int sms = num_sms();
-    if (sms < 2) return BI_ERR_CUDA;
+    const int64_t units =
+        ((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N) * (int64_t)splits;
+    if (units > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
     const int gm = 16;  // row tiles per group of the tile walk (L2 reuse of A and W blocks)
-    const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
-    bi_gemm_bf16_pair_kernel<<<dim3((unsigned)(2 * pairs)), THREADS, pair::SMEM_BYTES, stream>>>(
-        tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, err);
+    const int64_t pairs = units < clusters ? units : clusters;
+    const dim3 grid((unsigned)(2 * pairs));
+    if (splits > 1)
+        bi_gemm_bf16_pair_kernel<true><<<grid, THREADS, pair::SMEM_BYTES, stream>>>(
+            tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, splits, cnt, part, err);
+    else
+        bi_gemm_bf16_pair_kernel<false><<<grid, THREADS, pair::SMEM_BYTES, stream>>>(
+            tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, 1, nullptr, nullptr, err);
     return bi::launch_status();
 }
 
@@ -589,10 +762,27 @@ bool use_pairs(int64_t N, int64_t K) {
     return (N + pair::TILE_N - 1) / pair::TILE_N <= sms / 2;
 }
 
+// The K split of the plan.  The split kernel is built and tested (bi_ctrl_gemm_split runs it
+// with any S), but the plan keeps S = 1 for every shape.  Measured on a B200 for the 4096- and
+// 6144-wide projections: a split fills idle SM pairs and pays while M fits one or two rows of
+// tiles (K = 14336, M = 8: 35 us at S = 4 against 79 us), but its combine of fp32 partials
+// through L2 costs 6 % to 5x once M reaches 1024, and the plan may not depend on M.
+int splits_for(int64_t N, int64_t K) {
+    (void)N;
+    (void)K;
+    return 1;
+}
+
 int launch_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N, int64_t K,
-                bool c_bf16, cudaStream_t stream) {
-    if (use_pairs(N, K)) return launch_gemm_pair(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
+                bool c_bf16, int splits, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (use_pairs(N, K)) return launch_gemm_pair(A, lda, W, ldw, C, M, N, K, c_bf16, splits, ws, ws_bytes, stream);
+    if (splits != 1) return BI_ERR_INVALID_ARG;
     return launch_gemm_bn<256>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
+}
+
+size_t gemm_ws_bytes(int64_t M, int64_t N, int S) {
+    if (M <= 0 || N <= 0 || S <= 1) return 0;
+    return split_counter_bytes(M, N) + split_partial_bytes(M, N, S);
 }
 
 int gemm_shape_checks(const void* A, const void* W, const void* C, int64_t M, int64_t N, int64_t K, int c_dtype) {
@@ -645,18 +835,45 @@ int splitk_for(int64_t M, int64_t N, int64_t K) {
 
 }  // namespace
 
+BI_API int bi_gemm_splits(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0) return 0;
+    return splits_for(N, K);
+}
+
+BI_API size_t bi_gemm_counter_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0 || splits_for(N, K) <= 1) return 0;
+    return split_counter_bytes(M, N);
+}
+
 BI_API size_t bi_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
-    (void)M; (void)N; (void)K;
-    return 0;
+    if (N <= 0 || K <= 0) return 0;
+    return gemm_ws_bytes(M, N, splits_for(N, K));
 }
 
 BI_API int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype, void* ws,
                    size_t ws_bytes, void* stream) {
-    (void)ws; (void)ws_bytes;
     const int c = gemm_shape_checks(A, W, C, M, N, K, c_dtype);
     if (c < 0) return BI_OK;
     if (c != BI_OK) return c;
-    return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, bi::as_stream(stream));
+    const int S = splits_for(N, K);
+    if (S > 1 && (!ws || !bi::aligned16(ws) || ws_bytes < gemm_ws_bytes(M, N, S))) return BI_ERR_WORKSPACE;
+    return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, S, ws, ws_bytes, bi::as_stream(stream));
+}
+
+BI_API size_t bi_ctrl_gemm_split_workspace_size(int64_t M, int64_t N, int64_t K, int32_t splits) {
+    (void)K;
+    return gemm_ws_bytes(M, N, splits);
+}
+
+BI_API int bi_ctrl_gemm_split(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype,
+                              int32_t splits, void* ws, size_t ws_bytes, void* stream) {
+    const int c = gemm_shape_checks(A, W, C, M, N, K, c_dtype);
+    if (c < 0) return BI_OK;
+    if (c != BI_OK) return c;
+    if (!use_pairs(N, K) && splits != 1) return BI_ERR_UNSUPPORTED_SHAPE;
+    if (splits < 1 || splits > pair::MAX_SPLIT || splits > (K + BK - 1) / BK) return BI_ERR_INVALID_ARG;
+    if (splits > 1 && (!ws || !bi::aligned16(ws) || ws_bytes < gemm_ws_bytes(M, N, splits))) return BI_ERR_WORKSPACE;
+    return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, splits, ws, ws_bytes, bi::as_stream(stream));
 }
 
 BI_API size_t bi_ctrl_gemm_splitk_workspace_size(int64_t M, int64_t N, int64_t K) {
@@ -672,7 +889,7 @@ BI_API int bi_ctrl_gemm_splitk(const void* A, const void* W, void* C, int64_t M,
     if (c != BI_OK) return c;
     cudaStream_t s = bi::as_stream(stream);
     const int S = splitk_for(M, N, K);
-    if (S == 1) return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, s);
+    if (S == 1) return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, 1, nullptr, 0, s);
     const size_t need = (size_t)S * M * N * sizeof(float);
     if (!ws || ws_bytes < need || !bi::aligned16(ws)) return BI_ERR_WORKSPACE;
     const int64_t KS = K / S;
@@ -680,7 +897,7 @@ BI_API int bi_ctrl_gemm_splitk(const void* A, const void* W, void* C, int64_t M,
     for (int i = 0; i < S; ++i) {
         const int st = launch_gemm(static_cast<const __nv_bfloat16*>(A) + i * KS, K,
                                    static_cast<const __nv_bfloat16*>(W) + i * KS * N, N, part + (int64_t)i * M * N, M,
-                                   N, KS, false, s);
+                                   N, KS, false, 1, nullptr, 0, s);
         if (st != BI_OK) return st;
     }
     const int64_t MN = M * N;  // N % 8 == 0, so MN is a multiple of 4

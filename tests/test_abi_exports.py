@@ -107,3 +107,30 @@ def test_model_ops_host_checks(lib):
     assert lib.bi_prefill_attn(*args(q=a + 2)) == 3
     assert lib.bi_prefill_attn(*args(ldq=4100)) == 3
     assert lib.bi_prefill_attn(*args(ldo=2048)) == 1
+
+
+def test_gemm_split_plan_host(lib):
+    """The GEMM plan keeps one K slice for every shape (the split was measured to lose at large
+    M, and the plan may not depend on M), so bi_gemm needs no workspace.  The split kernel's
+    workspace arithmetic and argument checks are those of bi_ctrl_gemm_split."""
+    for N, K in ((6144, 4096), (4096, 4096), (4096, 14336), (14336, 4096), (512, 256), (28672, 4096),
+                 (32000, 4096)):
+        assert lib.bi_gemm_splits(N, K) == 1, (N, K)
+        assert lib.bi_gemm_workspace_size(4096, N, K) == 0
+        assert lib.bi_gemm_counter_bytes(4096, N, K) == 0
+    for M in (1, 8, 255, 256, 257, 4096):
+        tiles = -(-M // 256) * 16
+        counters = -(-tiles * 8 * 4 // 256) * 256  # one counter per (tile, CTA, epilogue warp)
+        for S in (2, 3, 4):
+            assert lib.bi_ctrl_gemm_split_workspace_size(M, 4096, 14336, S) == counters + (S - 1) * M * 4096 * 4
+        assert lib.bi_ctrl_gemm_split_workspace_size(M, 4096, 14336, 1) == 0
+    a = 1 << 20
+    P = ctypes.c_void_p
+    # a split without a workspace, with one too small or misaligned: refused before any launch
+    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 2, None, 0, None) == 4
+    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 2, P(a), 64, None) == 4
+    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 2, P(a + 8), 1 << 30, None) == 4
+    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 5, None, 0, None) == 1
+    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 64, 1, 2, None, 0, None) == 1  # 1 K block
+    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 28672, 4096, 1, 2, None, 0, None) == 2
+    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 0, 4096, 4096, 1, 2, None, 0, None) == 0  # empty batch
