@@ -1,10 +1,14 @@
 /*
- * bi_ctrl.h -- comparators of libbi.so.  These are NOT batch-invariant or NOT
- * deterministic, on purpose.
+ * bi_ctrl.h -- comparators and instruments of libbi.so.
  *
- * They exist for two reasons: to measure what invariance costs against the faster
- * schedules it rules out, and to act as positive controls for the invariance harness.
- * Each one must show violations somewhere, or the harness could not see any.
+ * The comparators are NOT batch-invariant or NOT deterministic, on purpose.  They exist for
+ * two reasons: to measure what invariance costs against the faster schedules it rules out,
+ * and to act as positive controls for the invariance harness.  Each one must show
+ * violations somewhere, or the harness could not see any.
+ *
+ * Two instruments sit beside them: bi_ctrl_gemm_split runs bi_gemm's kernel at a split
+ * count the plan does not choose (batch-invariant for a fixed count), and
+ * bi_ctrl_wait_timeout_probe drives the bounded-wait failure path.
  * Conventions are those of bi.h.
  */
 #ifndef BI_CTRL_H
