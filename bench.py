@@ -29,6 +29,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -74,29 +75,93 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling every 200 ms during the timed region."""
+    """SM clock, power and throttle-reason samples during the timed region.
+
+    NVML is polled every millisecond from a thread (read-only queries), so that even a timed
+    region of a few tens of milliseconds holds many samples.  Without NVML, nvidia-smi samples
+    every 200 ms instead."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits, in the order of the last four QUERY fields
+    REASON_BITS = (0x8, 0x40, 0x20, 0x4)  # hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: str):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.rows: list[list[str]] = []
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+
+    def _start_nvml(self) -> bool:
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+        except Exception:
+            return False
+        try:
+            if self.gpu.startswith("GPU-"):
+                try:
+                    h = nv.nvmlDeviceGetHandleByUUID(self.gpu)
+                except Exception:
+                    h = nv.nvmlDeviceGetHandleByUUID(self.gpu.encode())
+            else:
+                h = nv.nvmlDeviceGetHandleByIndex(int(self.gpu))
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def sample():
+                r = int(reasons(h))
+                return [self.gpu, str(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), str(mx),
+                        str(nv.nvmlDeviceGetPowerUsage(h) / 1000.0), hex(r)] + \
+                       ["Active" if r & bit else "Not Active" for bit in self.REASON_BITS]
+
+            self.rows.append(sample())  # fails here, not in the thread, if a query is unsupported
+        except Exception:
+            nv.nvmlShutdown()
+            return False
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.rows.append(sample())
+                except Exception:
+                    return
+                time.sleep(0.001)
+
+        self._nvml = nv
+        self.source = "nvml, every ~1 ms"
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        return True
 
     def __enter__(self):
+        if self._start_nvml():
+            return self
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, every 200 ms"
         except Exception:
             self.proc = None
         time.sleep(0.3)
         return self
 
     def __exit__(self, *a):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.send_signal(signal.SIGTERM)
             try:
@@ -105,20 +170,21 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        rows = []
-        try:
-            with open(self.path) as f:
-                for line in f:
-                    parts = [p.strip() for p in line.split(",")]
-                    if len(parts) >= 9:
-                        rows.append(parts)
-        except Exception:
-            pass
-        finally:
+        rows = list(self.rows)
+        if self.path is not None:
             try:
-                os.unlink(self.path)
+                with open(self.path) as f:
+                    for line in f:
+                        parts = [p.strip() for p in line.split(",")]
+                        if len(parts) >= 9:
+                            rows.append(parts)
             except Exception:
                 pass
+            finally:
+                try:
+                    os.unlink(self.path)
+                except Exception:
+                    pass
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
 
@@ -135,7 +201,8 @@ class ClockSampler:
         top = max(sm) if sm else 0
         loaded = [s for s in sm if s >= 0.5 * top] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None,
+                "source": self.source}
 
 
 def _gpu_id(local_rank: int) -> str:
