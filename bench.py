@@ -364,8 +364,32 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = t0.elapsed_time(t1)
+    total_ev_ms = t0.elapsed_time(t1)
     op_ms = [sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(K)) for i in range(len(ops))]
+    del graph
+    # The same K steps without the per-op events: an event between two launches is a full dependency,
+    # so only this graph lets a kernel's set-up overlap the tail of the kernel before it (programmatic
+    # dependent launch).  Its time is the step time; the per-op times above come from the graph with
+    # events, where no such overlap happens.
+    u0, u1 = mk(), mk()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        u0.record(stream)
+        for k in range(K):
+            step(k)
+        u1.record(stream)
+    graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(_gpu_id(local_rank)) as clk2:
+        graph.replay()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = u0.elapsed_time(u1)
+    del graph
 
     # end-to-end: every step copies its inputs host -> device from pinned memory, runs the same
     # launches and copies its results device -> host, through the C ABI.  The copies run on their
@@ -426,9 +450,13 @@ def run_ours(args, rank, world, local_rank):
     tax = invariance_tax(device, stream, io) if not args.no_tax else None
 
     clocks = clk.summary()
-    (total_ms, e2e_ms, *op_ms), viol = reduce_over_ranks([total_ms, e2e_ms] + op_ms, viol, world, device)
+    clocks_step = clk2.summary()
+    (total_ms, total_ev_ms, e2e_ms, *op_ms), viol = reduce_over_ranks([total_ms, total_ev_ms, e2e_ms] + op_ms, viol,
+                                                                      world, device)
     if rank != 0:
         return None
+    # rank 0 alone, after the last collective: the gate points at every batch size they apply to
+    gates = gate_table(device, stream, load_peaks()[0]) if not args.no_gates else None
 
     peaks, peak_src = load_peaks()
     # A kernel timed inside a long step (a timed region of half a second or more, long enough for
@@ -490,7 +518,8 @@ def run_ours(args, rank, world, local_rank):
     cpu = cpu_baseline(args.cpu_seconds)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4),
+        "ms_per_step_with_op_events": round(total_ev_ms / K, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) activations, "
         "N(0,0.02) weights; no trained weights)",
         "config": {"workload": f"Llama-3-8B-shaped dense ops at M={M_TOKENS} tokens, hidden {HIDDEN}; LoRA r="
@@ -503,7 +532,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": K * sum(op.get("launches", 1) for op in ops),
         "bi_violations": viol,
         "invariance_tax": tax,
-        "clocks": clocks, "cpu_baseline": cpu,
+        "gates": gates,
+        "clocks": clocks, "clocks_step_without_op_events": clocks_step, "cpu_baseline": cpu,
         # what the result was produced with (GPU, driver, CUDA, torch, commit)
         "pin": harness_pin(),
     }
@@ -643,6 +673,89 @@ def invariance_tax(device, stream, io):
                          for r_ in range(min(M, 4)))
             cb[f"K={K2},N={N2}"] = v
         out["cublas_rows_differing_from_solo"] = cb
+    torch.cuda.synchronize()
+    return out
+
+
+def gate_table(device, stream, peaks):
+    """The target fractions measured at the batch sizes they apply to, in the same run (outside the
+    timed region): GEMM >= 60 % of the dense bf16 peak (burst) for M >= 256 on the three Llama-3-8B
+    projections; RMSNorm and the LoRA shrink >= 75 % of HBM from M = 1024 (the shrink's workload
+    stops at M = 4096); decode attention >= 75 % of HBM once the cache holds >= 1 GB of K and V.
+    Each point is the median per-launch time of back-to-back launches in a CUDA graph, inputs
+    rotating through copies that exceed the L2 (one copy when a launch's inputs already do)."""
+    import torch
+    from invariant_deterministic_rmsnorm_b200 import binding as B
+
+    def rows_dev(seed, M, cols):
+        g = torch.Generator(device=device).manual_seed(seed)
+        return torch.randn((M, cols), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+    def point(key, n, work, ms, peak, gate, unit):
+        ach = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
+        return {key: n, "us": round(ms * 1e3, 2), "achieved": round(ach, 1), "frac": round(ach / peak, 4),
+                "gate": gate, "met": bool(ach / peak >= gate)}
+
+    out = {"peaks": {"bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"]}}
+    with torch.cuda.stream(stream):
+        for K, N in GEMM_SHAPES:
+            rows = []
+            for M in (256, 512, 1024, 4096, 8192):
+                R = _copies(2 * (M * K + K * N + M * N))
+                Ws = [rows_dev(50 + j, K, N).mul_(0.02) for j in range(R)]
+                As = [rows_dev(60 + j, M, K) for j in range(R)]
+                Cs = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(R)]
+                ms = _time_graph([lambda j=j: B.bi_gemm(As[j], Ws[j], C=Cs[j], stream=stream) for j in range(R)],
+                                 stream)
+                rows.append(point("M", M, 2 * M * N * K, ms, peaks["bf16_tflops"], 0.60, "TFLOP/s"))
+                del Ws, As, Cs
+            out[f"gemm_K{K}_N{N}"] = {"unit": "TFLOP/s", "rows": rows}
+        w = _to_dev(inputs.rmsnorm_case(1, HIDDEN, "bf16")[1], device)
+        rows = []
+        for M in (1024, 4096, 8192):
+            R = _copies(2 * 2 * HIDDEN * M)
+            xs = [rows_dev(70 + j, M, HIDDEN) for j in range(R)]
+            ys = [torch.empty_like(xs[0]) for _ in range(R)]
+            ms = _time_graph([lambda j=j: B.bi_rmsnorm(xs[j], w, y=ys[j], eps=EPS, stream=stream)
+                              for j in range(R)], stream)
+            rows.append(point("M", M, 2 * 2 * HIDDEN * M + 2 * HIDDEN, ms, peaks["hbm_gbs"], 0.75, "GB/s"))
+            del xs, ys
+        out["rmsnorm_H4096"] = {"unit": "GB/s", "rows": rows}
+        for r in (8, 16, 64):
+            A_l = rows_dev(80, HIDDEN, r).mul_(0.02)
+            rows = []
+            for M in (1024, 4096):
+                R = _copies(2 * HIDDEN * M)
+                xs = [rows_dev(90 + j, M, HIDDEN) for j in range(R)]
+                t = torch.empty((M, r), dtype=torch.float32, device=device)
+                ms = _time_graph([lambda j=j: B.bi_lora_shrink(xs[j], A_l, t=t, split_k=8, stream=stream)
+                                  for j in range(R)], stream)
+                rows.append(point("M", M, 2 * HIDDEN * M + 2 * HIDDEN * r + 4 * M * r, ms, peaks["hbm_gbs"], 0.75,
+                                  "GB/s"))
+                del xs
+            out[f"lora_shrink_r{r}"] = {"unit": "GB/s", "rows": rows}
+        kv_len = inputs.kv_lengths(256)
+        indptr, T = inputs.kv_layout(kv_len, 256)
+        g = torch.Generator(device=device).manual_seed(5)
+        kc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        vc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        qa = torch.randn((256, 32, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        ip_d = torch.tensor(indptr, dtype=torch.int32, device=device)
+        ln_d = torch.tensor(kv_len, dtype=torch.int32, device=device)
+        rows = []
+        for Bn in (32, 64, 128, 256):
+            Tn = int(indptr[Bn])
+            o = torch.empty((Bn, 32, 128), dtype=torch.bfloat16, device=device)
+            ws = torch.empty(B.bi_decode_attn_workspace_size(Tn, 32), dtype=torch.uint8, device=device)
+            q = qa[:Bn].contiguous()
+            kv = int(kv_len[:Bn].sum()) * 8 * 128 * 2 * 2
+            ms = _time_graph([lambda: B.bi_decode_attn(q, kc[:Tn], vc[:Tn], ip_d[:Bn + 1], ln_d[:Bn], out=o,
+                                                       workspace=ws, stream=stream)], stream)
+            pt = point("B", Bn, kv + Bn * 32 * 128 * 4, ms, peaks["hbm_gbs"], 0.75, "GB/s")
+            pt["kv_gb"] = round(kv / 1e9, 3)
+            rows.append(pt)
+        del kc, vc
+        out["decode_attn"] = {"unit": "GB/s", "rows": rows}
     torch.cuda.synchronize()
     return out
 
@@ -1028,6 +1141,61 @@ class FastOps:
         return B.bi_ctrl_decode_attn_adaptive(q, k, v, kv_indptr, kv_len, out=out)
 
 
+def _contrast_fill(d, slots, contents, isolated):
+    """Prefill; returns the greedy next token of every listed slot.  isolated: one prefill call per
+    request (the fixed-shape alternative never batches prefill)."""
+    from invariant_deterministic_rmsnorm_b200 import binding as B
+    d.reset()
+    if isolated:
+        return [int(B.bi_argmax(d.forward([s], [c]))[0]) for s, c in zip(slots, contents)]
+    return B.bi_argmax(d.forward(slots, contents)).cpu().tolist()
+
+
+def contrast_composition(dec_bi, dec_fast, prompts, filler, BF=128, probe_steps=16):
+    """Bit for bit, does a probe request's (prompts[0]) logits over `probe_steps` greedy decode
+    steps after its prefill stay the same when its co-residents or its slot change?
+
+    Three ways of running the same decoder (the position-invariant scheduling alternative of the
+    CoRun comment thread, "thecolony.si" page, against batch-invariant kernels):
+      - fast kernels at a fixed BF-slot shape, every request prefilled alone, decode replayed from
+        one graph: alone (filler elsewhere) vs among real co-residents vs in another slot;
+      - fast kernels at the true batch (dynamic shapes): alone vs in a batch of 37;
+      - batch-invariant kernels: alone vs in a batch of 37 vs in a batched BF-request prefill.
+    Returns the findings as a dict of booleans and largest differences."""
+    probe = prompts[0]
+    others = list(prompts[1:BF])
+
+    def probe_logits(d, slots, contents, at, isolated):
+        first = _contrast_fill(d, slots, contents, isolated)
+        g = d.decode_graph(slots)
+        g.set_tokens(first)
+        got = []
+        for _ in range(probe_steps):
+            got.append(g.replay()[at].cpu().numpy().copy())
+        del g
+        return np.stack(got)
+
+    def same(a, b):
+        return bool(np.array_equal(a.view(np.uint32), b.view(np.uint32)))
+
+    fixed_alone = probe_logits(dec_fast, list(range(BF)), [filler] * 5 + [probe] + [filler] * (BF - 6), 5, True)
+    fixed_busy = probe_logits(dec_fast, list(range(BF)), others[:5] + [probe] + others[5:BF - 1], 5, True)
+    fixed_moved = probe_logits(dec_fast, list(range(BF)), [filler] * 77 + [probe] + [filler] * (BF - 78), 77, True)
+    dyn_alone = probe_logits(dec_fast, [0], [probe], 0, False)
+    dyn_busy = probe_logits(dec_fast, list(range(37)), others[:5] + [probe] + others[5:36], 5, False)
+    bi_alone = probe_logits(dec_bi, [0], [probe], 0, False)
+    bi_busy = probe_logits(dec_bi, list(range(37)), others[:5] + [probe] + others[5:36], 5, False)
+    bi_fixed = probe_logits(dec_bi, list(range(BF)), others[:5] + [probe] + others[5:BF - 1], 5, False)
+    return {"contrast": "composition", "probe_len": len(probe), "decode_steps": probe_steps,
+            "fast_fixed128_alone_vs_busy_same_slot": same(fixed_alone, fixed_busy),
+            "fast_fixed128_slot5_vs_slot77": same(fixed_alone, fixed_moved),
+            "fast_dynamic_alone_vs_batch37": same(dyn_alone, dyn_busy),
+            "fast_dynamic_max_abs_diff": float(np.abs(dyn_alone - dyn_busy).max()),
+            "bi_alone_vs_batch37": same(bi_alone, bi_busy),
+            "bi_alone_vs_batch128_batched_prefill": same(bi_alone, bi_fixed),
+            "fast_vs_bi_max_abs_diff": float(np.abs(fixed_alone - bi_alone).max())}
+
+
 def run_contrast(args):
     """Position-invariant scheduling against batch-invariant kernels, on the same synthetic decoder.
 
@@ -1039,7 +1207,6 @@ def run_contrast(args):
     then, bit for bit, whether a probe request's logits over prefill + 16 greedy steps stay the
     same when its co-residents or its slot change."""
     import torch
-    from invariant_deterministic_rmsnorm_b200 import binding as B
     from invariant_deterministic_rmsnorm_b200.decoder import Decoder
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
@@ -1053,12 +1220,7 @@ def run_contrast(args):
     filler = inputs.prompt(inputs.SEED_FILLER_BASE, 16, shape.vocab)
     dec = {"bi": Decoder(shape, w, BF, max_len), "fast": Decoder(shape, w, BF, max_len, ops=FastOps)}
 
-    def fill(d, slots, contents, isolated):
-        """Prefill; returns the greedy next token of every listed slot."""
-        d.reset()
-        if isolated:
-            return [int(B.bi_argmax(d.forward([s], [c]))[0]) for s, c in zip(slots, contents)]
-        return B.bi_argmax(d.forward(slots, contents)).cpu().tolist()
+    fill = _contrast_fill
 
     def step_ms(d, slots):
         g = d.decode_graph(slots)
@@ -1088,39 +1250,7 @@ def run_contrast(args):
                      "fast_fixed128_ms": round(t_fix, 4), "fast_fixed128_tokens_per_s": round(b / t_fix * 1e3)})
     print(json.dumps({"contrast": "decode_throughput", "fixed_slots": BF, "steps": steps, "rows": rows}), flush=True)
 
-    probe = prompts[0]
-
-    def probe_logits(d, slots, contents, at, isolated):
-        """The probe's (contents[at]) logits at each of probe_steps greedy decode steps after the prefill."""
-        first = fill(d, slots, contents, isolated)
-        g = d.decode_graph(slots)
-        g.set_tokens(first)
-        got = []
-        for _ in range(probe_steps):
-            got.append(g.replay()[at].cpu().numpy().copy())
-        del g
-        return np.stack(got)
-
-    def same(a, b):
-        return bool(np.array_equal(a.view(np.uint32), b.view(np.uint32)))
-
-    others = prompts[1:BF]
-    fixed_alone = probe_logits(dec["fast"], list(range(BF)), [filler] * 5 + [probe] + [filler] * (BF - 6), 5, True)
-    fixed_busy = probe_logits(dec["fast"], list(range(BF)), others[:5] + [probe] + others[5:BF - 1], 5, True)
-    fixed_moved = probe_logits(dec["fast"], list(range(BF)), [filler] * 77 + [probe] + [filler] * (BF - 78), 77, True)
-    dyn_alone = probe_logits(dec["fast"], [0], [probe], 0, False)
-    dyn_busy = probe_logits(dec["fast"], list(range(37)), others[:5] + [probe] + others[5:36], 5, False)
-    bi_alone = probe_logits(dec["bi"], [0], [probe], 0, False)
-    bi_busy = probe_logits(dec["bi"], list(range(37)), others[:5] + [probe] + others[5:36], 5, False)
-    bi_fixed = probe_logits(dec["bi"], list(range(BF)), others[:5] + [probe] + others[5:BF - 1], 5, False)
-    print(json.dumps({"contrast": "composition", "probe_len": len(probe), "decode_steps": probe_steps,
-                      "fast_fixed128_alone_vs_busy_same_slot": same(fixed_alone, fixed_busy),
-                      "fast_fixed128_slot5_vs_slot77": same(fixed_alone, fixed_moved),
-                      "fast_dynamic_alone_vs_batch37": same(dyn_alone, dyn_busy),
-                      "fast_dynamic_max_abs_diff": float(np.abs(dyn_alone - dyn_busy).max()),
-                      "bi_alone_vs_batch37": same(bi_alone, bi_busy),
-                      "bi_alone_vs_batch128_batched_prefill": same(bi_alone, bi_fixed),
-                      "fast_vs_bi_max_abs_diff": float(np.abs(fixed_alone - bi_alone).max())}), flush=True)
+    print(json.dumps(contrast_composition(dec["bi"], dec["fast"], prompts, filler, BF, probe_steps)), flush=True)
 
 
 def main():
@@ -1131,6 +1261,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-tax", action="store_true", help="skip the invariance-tax comparison")
+    ap.add_argument("--no-gates", action="store_true", help="skip the per-batch-size gate table")
     ap.add_argument("--replay-study", action="store_true",
                     help="identical-input replay study of the atomic vs ordered split-K shrink (one GPU)")
     ap.add_argument("--replays", type=int, default=200)

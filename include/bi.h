@@ -223,8 +223,8 @@ int bi_lora_expand(const float* t, const void* B, void* y, int64_t M, int32_t r,
  * merged in order c = 0, 1, ... with an fp32 log-sum-exp rescale, and out = o / l.
  *
  * Layout violations that only the device can see (kv_indptr not chunk-aligned, kv_len
- * out of range) set bit 0x100 of the device error word.  The affected rows of out are
- * then left unwritten.
+ * out of range, kv_indptr[b + 1] > total_tokens) set bit 0x100 of the device error word.
+ * The affected rows of out are then left unwritten; the other rows are computed as usual.
  */
 size_t bi_decode_attn_workspace_size(int64_t total_tokens, int32_t Hq, int32_t head_dim, int32_t chunk);
 int bi_decode_attn(const void* q, const void* k, const void* v, const int32_t* kv_indptr, const int32_t* kv_len,
@@ -250,7 +250,11 @@ int bi_decode_attn(const void* q, const void* k, const void* v, const int32_t* k
  *     bytes.  Beyond 16 MiB the call returns BI_ERR_WORKSPACE and launches nothing.
  *     At Hq = 32 that is about 258,000 cache tokens; use bi_decode_attn for larger caches.
  *   - The first call on each device looks up the array's device address with that
- *     device current, then caches it.  Make that first call before any stream capture.
+ *     device current, then caches it.  Make that first call before any stream capture.  A
+ *     lookup that fails returns BI_ERR_CUDA and is tried again by the next call.
+ *   - A sequence whose kv_indptr[b + 1] exceeds total_tokens is a layout error (bit 0x100,
+ *     row left unwritten), as in bi_decode_attn: the call never reads partials it did not
+ *     write in this call.
  *   - Every call on a device shares the one array, which keeps whatever the last call
  *     left there.  Nothing in it needs to start at zero.  Calls whose work overlaps on
  *     the GPU (on different streams, or from different host threads without ordering)

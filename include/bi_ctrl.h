@@ -89,6 +89,16 @@ int bi_ctrl_decode_attn_adaptive(const void* q, const void* k, const void* v, co
  */
 int bi_ctrl_wait_timeout_probe(uint64_t limit_ns, void* stream);
 
+/*
+ * bi_ctrl_set_pdl -- turn programmatic dependent launch on (enable != 0, the default) or off for
+ * the library's later launches; returns the previous setting.  With it on, a kernel may begin
+ * its set-up (barriers, tensor memory, descriptor prefetch) while the kernel before it on the
+ * stream finishes, and waits for that kernel before it touches global memory.  It changes when
+ * work starts, never what is computed: outputs are bitwise the same either way.  Here to
+ * measure what the overlap gains.  Process-wide; not synchronised with launches in flight.
+ */
+int bi_ctrl_set_pdl(int enable);
+
 #ifdef __cplusplus
 }
 #endif

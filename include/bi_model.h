@@ -105,6 +105,15 @@ int bi_swiglu(const void* gu, int64_t ld_gu, void* out, int64_t ld_out, int64_t 
 int bi_argmax(const float* x, int64_t ld, int64_t T, int64_t N, int32_t* out, void* stream);
 
 /*
+ * bi_advance -- v[i] += step for i < n (int32, wrapping as two's complement).
+ *
+ * The bookkeeping of a replayed greedy decode step: the positions, cache rows and KV lengths
+ * of every sequence move on by one token.  Kept in the library so that a captured decode
+ * step runs no device work outside it.  v int32 [n], device; n >= 0 (0 is a no-op).
+ */
+int bi_advance(int32_t* v, int64_t n, int32_t step, void* stream);
+
+/*
  * bi_prefill_attn -- batch-invariant causal attention for prefill (grouped-query, variable length).
  *
  * Source: "Defeating Nondeterminism in LLM Inference" (Spanish summary), section "Attention".

@@ -70,6 +70,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_ctrl_decode_attn_adaptive_workspace_size": ([I64, I32], Z),
         "bi_ctrl_decode_attn_adaptive": ([P, P, P, P, P, I32, I64, I32, I32, F, P, C, P, Z, P], C),
         "bi_ctrl_wait_timeout_probe": ([ctypes.c_uint64, P], C),
+        "bi_ctrl_set_pdl": ([C], C),
         # include/bi_model.h
         "bi_embed": ([P, P, P, I64, I64, I64, P], C),
         "bi_rope_table": ([P, I64, I32, ctypes.c_double, P], C),
@@ -78,6 +79,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_add": ([P, I64, P, I64, I64, I64, P], C),
         "bi_swiglu": ([P, I64, P, I64, I64, I64, P], C),
         "bi_argmax": ([P, I64, I64, I64, P, P], C),
+        "bi_advance": ([P, I64, I32, P], C),
         "bi_prefill_attn": ([P, I64, I64, P, P, I64, P, P, I32, P, P, I32, I32, I32, I32, F, P, I64, P], C),
     }
     for name, (args, res) in sig.items():
@@ -419,6 +421,13 @@ def bi_argmax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> 
     _i32(out, "out")
     _check("bi_argmax", library().bi_argmax(_ptr(x), x.stride(0), T, N, _ptr(out), _stream(stream)))
     return out
+
+
+def bi_advance(v: torch.Tensor, step: int = 1, stream=None) -> torch.Tensor:
+    """v += step, in place (int32, on the device)."""
+    _i32(v, "v")
+    _check("bi_advance", library().bi_advance(_ptr(v), v.numel(), int(step), _stream(stream)))
+    return v
 
 
 PREFILL_TILE_ROWS = 128

@@ -26,10 +26,13 @@ __device__ uint32_t g_device_error;
 
 constexpr int kMaxDevices = 64;
 std::atomic<uintptr_t> g_word_addr[kMaxDevices];
+std::atomic<int> g_pdl{1};
 
 }  // namespace
 
 namespace bi {
+
+bool pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
 
 // Device address of the error word on the current device.  The address is looked
 // up once per device and cached.  Returns nullptr on a CUDA error.
@@ -87,4 +90,9 @@ BI_API int bi_ctrl_wait_timeout_probe(uint64_t limit_ns, void* stream) {
     if (!err) return BI_ERR_CUDA;
     wait_probe_kernel<<<1, 32, 0, bi::as_stream(stream)>>>(limit_ns, err);
     return bi::launch_status();
+}
+
+BI_API int bi_ctrl_set_pdl(int enable) {
+    const int old = g_pdl.exchange(enable ? 1 : 0);
+    return old;
 }

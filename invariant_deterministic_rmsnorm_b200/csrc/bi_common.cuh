@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "bi.h"
 
 #define BI_API extern "C" __attribute__((visibility("default")))
@@ -22,6 +24,40 @@ inline int launch_status() {
 
 // Device address of the library's error word on the current device (bi_abi.cu).
 uint32_t* device_error_word();
+
+// Whether launches may use programmatic dependent launch (bi_abi.cu; on unless
+// bi_ctrl_set_pdl(0) turned it off).
+bool pdl_enabled();
+
+// Launch `kernel` on `s`.  With programmatic dependent launch on, it may begin while the kernel
+// before it on the stream finishes; every kernel launched this way calls pdl_wait() (bi_sm100.cuh)
+// before it reads or writes global memory.  cluster: CTAs per cluster along y (1 = no cluster).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              unsigned cluster_y, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_y > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = 1;
+        attr[n].val.clusterDim.y = cluster_y;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = n ? attr : nullptr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 inline int elem_size(int dtype) { return dtype == BI_F32 ? 4 : (dtype == BI_BF16 ? 2 : 0); }
 

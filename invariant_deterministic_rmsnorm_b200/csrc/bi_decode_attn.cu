@@ -87,7 +87,8 @@ struct SeqCache {
 // The (sequence, chunk) that owns CH-token slot `slot` of the packed cache.
 template <int CH>
 __device__ __forceinline__ Item item_of(int slot, const int32_t* __restrict__ kv_indptr,
-                                        const int32_t* __restrict__ kv_len, int B, bool& bad, SeqCache& sc) {
+                                        const int32_t* __restrict__ kv_len, int B, int64_t T, bool& bad,
+                                        SeqCache& sc) {
     Item it{0, 0, 0, (int64_t)slot * CH};
     bad = false;
     int lo;
@@ -109,7 +110,9 @@ __device__ __forceinline__ Item item_of(int slot, const int32_t* __restrict__ kv
     const int64_t sbase = sc.lo_tok;
     const int len = sc.len;
     const int64_t cap = sc.hi_tok - sbase;
-    if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap) {
+    // a sequence whose capacity reaches past the cache's T tokens is refused whole, so that the
+    // merge never reads a slot this phase did not write
+    if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap || sc.hi_tok > T) {
         bad = (it.tok0 - sbase) < CH;  // report once per sequence
         return it;
     }
@@ -127,8 +130,8 @@ template <int G, int CH>
 __global__ void __launch_bounds__(THREADS, 2)
 decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ kv_indptr,
-                         const int32_t* __restrict__ kv_len, int B, int Hq, int Hkv, int n_items, float scale,
-                         float* __restrict__ o_part, float* __restrict__ ml_part, uint32_t* err) {
+                         const int32_t* __restrict__ kv_len, int B, int64_t T, int Hq, int Hkv, int n_items,
+                         float scale, float* __restrict__ o_part, float* __restrict__ ml_part, uint32_t* err) {
     using L = AttnLayout<G>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -157,6 +160,8 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         fence_proxy_async_shared();
     }
     __syncthreads();
+    pdl_wait();  // q, the cache and the index arrays may come from the kernels just before this one
+    pdl_trigger();
 
     if (warp == CWARPS) {
         // ------------------------------------------------ producer
@@ -168,7 +173,7 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             for (int w = w_begin; w < w_end && !*abort; ++w) {
                 const int slot = w / Hkv, g = w % Hkv;
                 bool bad;
-                const Item itm = item_of<CH>(slot, kv_indptr, kv_len, B, bad, sc);
+                const Item itm = item_of<CH>(slot, kv_indptr, kv_len, B, T, bad, sc);
                 if (bad && g == 0) atomicOr(err, DEVERR_BAD_LAYOUT);
                 if (itm.n_tok == 0) continue;
                 const int nsub = (itm.n_tok + SUB - 1) / SUB;
@@ -211,7 +216,7 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     for (int w = w_begin; w < w_end; ++w) {
         const int slot = w / Hkv, g = w % Hkv;
         bool bad;
-        const Item itm = item_of<CH>(slot, kv_indptr, kv_len, B, bad, sc);
+        const Item itm = item_of<CH>(slot, kv_indptr, kv_len, B, T, bad, sc);
         if (itm.n_tok == 0) continue;
         const int n_tok = itm.n_tok;
         const int nsub = (n_tok + SUB - 1) / SUB;
@@ -390,16 +395,19 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 template <bool OUT_BF16, int CH>
 __global__ void __launch_bounds__(128)
 decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restrict__ ml_part,
-                         const int32_t* __restrict__ kv_indptr, const int32_t* __restrict__ kv_len, int Hq,
-                         void* __restrict__ out, uint32_t* err) {
+                         const int32_t* __restrict__ kv_indptr, const int32_t* __restrict__ kv_len, int64_t T,
+                         int Hq, void* __restrict__ out, uint32_t* err) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x * 4 + warp;
     const int b = blockIdx.y;
+    pdl_wait();  // the partials come from phase 1, launched just before
+    pdl_trigger();
     if (h >= Hq) return;
     const int64_t sbase = kv_indptr[b];
     const int len = kv_len[b];
     const int64_t cap = (int64_t)kv_indptr[b + 1] - sbase;
-    if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap) {
+    // the same checks as phase 1: a sequence past the cache's T tokens has no partials to merge
+    if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap || (int64_t)kv_indptr[b + 1] > T) {
         if (lane == 0) atomicOr(err, DEVERR_BAD_LAYOUT);  // out row left unwritten
         return;
     }
@@ -443,6 +451,12 @@ decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restri
     } else {
         *reinterpret_cast<float4*>(static_cast<float*>(out) + off) = make_float4(r0, r1, r2, r3);
     }
+}
+
+// Phase 2 on `s`, allowed to start while phase 1 finishes (it waits for phase 1 before it reads).
+template <typename K, typename... Args>
+void launch_merge(K kernel, dim3 grid, cudaStream_t s, Args... args) {
+    (void)bi::launch_pdl(kernel, grid, dim3(128), 0, s, 1u, args...);
 }
 
 template <typename F>
@@ -503,8 +517,9 @@ int launch_chunks(const void* q, const void* k, const void* v, const int32_t* kv
     if (sms <= 0) return BI_ERR_CUDA;
     const int64_t ctas = 2LL * sms;  // two persistent CTAs per SM: one computes while the other waits
     dim3 grid((unsigned)(items < ctas ? items : ctas));
-    kern<<<grid, THREADS, L::BYTES, s>>>(tmK, tmV, static_cast<const __nv_bfloat16*>(q), kv_indptr, kv_len, B, Hq,
-                                         Hkv, (int)items, scale, o_part, ml_part, err);
+    if (bi::launch_pdl(kern, grid, dim3(THREADS), L::BYTES, s, 1u, tmK, tmV, static_cast<const __nv_bfloat16*>(q),
+                       kv_indptr, kv_len, B, T, Hq, Hkv, (int)items, scale, o_part, ml_part, err) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -545,9 +560,11 @@ BI_API int bi_decode_attn(const void* q, const void* k, const void* v, const int
     dim3 grid((unsigned)((Hq + 3) / 4), (unsigned)B);
     uint32_t* err = bi::device_error_word();
     if (out_dtype == BI_BF16)
-        decode_attn_merge_kernel<true, CHUNK><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        launch_merge(decode_attn_merge_kernel<true, CHUNK>, grid, s, o_part, ml_part, kv_indptr, kv_len,
+                     total_tokens, Hq, out, err);
     else
-        decode_attn_merge_kernel<false, CHUNK><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        launch_merge(decode_attn_merge_kernel<false, CHUNK>, grid, s, o_part, ml_part, kv_indptr, kv_len,
+                     total_tokens, Hq, out, err);
     return bi::launch_status();
 }
 
@@ -569,19 +586,22 @@ constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;  // 16 MiB; mirrored i
 static __device__ __align__(256) unsigned char g_decode_attn_scratch[kNoAllocScratchBytes];
 
 constexpr int kNoAllocMaxDevices = 64;
-std::once_flag g_scratch_once[kNoAllocMaxDevices];
+std::mutex g_scratch_mu;
 void* g_scratch_ptr[kNoAllocMaxDevices];
 
-// Device address of the scratch array on the current device.  It is looked up on the
-// first call made with that device current, then cached.  Returns nullptr if the
-// lookup fails.
+// Device address of the scratch array on the current device.  It is looked up with that
+// device current and cached once the lookup has succeeded; a failed lookup (for instance one
+// attempted inside a stream capture) caches nothing, so the next call tries again.  Returns
+// nullptr if the lookup fails.
 void* noalloc_scratch() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
-    std::call_once(g_scratch_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
         void* p = nullptr;
-        g_scratch_ptr[dev] = (cudaGetSymbolAddress(&p, g_decode_attn_scratch) == cudaSuccess) ? p : nullptr;
-    });
+        if (cudaGetSymbolAddress(&p, g_decode_attn_scratch) == cudaSuccess) g_scratch_ptr[dev] = p;
+        else (void)cudaGetLastError();  // the failed lookup must not surface as a later launch's error
+    }
     return g_scratch_ptr[dev];
 }
 
@@ -622,9 +642,11 @@ BI_API int bi_decode_attn_noalloc(const void* q, const void* k, const void* v, c
     uint32_t* err = bi::device_error_word();
     dim3 grid((unsigned)((Hq + 3) / 4), (unsigned)B);
     if (out_dtype == BI_BF16)
-        decode_attn_merge_kernel<true, CHUNK><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        launch_merge(decode_attn_merge_kernel<true, CHUNK>, grid, s, o_part, ml_part, kv_indptr, kv_len,
+                     total_tokens, Hq, out, err);
     else
-        decode_attn_merge_kernel<false, CHUNK><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        launch_merge(decode_attn_merge_kernel<false, CHUNK>, grid, s, o_part, ml_part, kv_indptr, kv_len,
+                     total_tokens, Hq, out, err);
     return bi::launch_status();
 }
 
@@ -653,9 +675,11 @@ int run_adaptive(const void* q, const void* k, const void* v, const int32_t* kv_
     uint32_t* err = bi::device_error_word();
     dim3 grid((unsigned)((Hq + 3) / 4), (unsigned)B);
     if (out_dtype == BI_BF16)
-        decode_attn_merge_kernel<true, CH><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        launch_merge(decode_attn_merge_kernel<true, CH>, grid, s, o_part, ml_part, kv_indptr, kv_len, T, Hq,
+                     out, err);
     else
-        decode_attn_merge_kernel<false, CH><<<grid, 128, 0, s>>>(o_part, ml_part, kv_indptr, kv_len, Hq, out, err);
+        launch_merge(decode_attn_merge_kernel<false, CH>, grid, s, o_part, ml_part, kv_indptr, kv_len, T, Hq,
+                     out, err);
     return bi::launch_status();
 }
 

@@ -168,6 +168,10 @@ bi_gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_addr;
+    // everything above overlaps the previous kernel's tail; A and W may come from it, and it may
+    // still read C
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -394,6 +398,10 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_addr;
+    // everything above overlaps the previous kernel's tail; A and W may come from it, and it may
+    // still read C or the split workspace
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -650,8 +658,9 @@ int launch_gemm_bn(const void* A, int64_t lda, const void* W, int64_t ldw, void*
     if (sms <= 0) return BI_ERR_CUDA;
     const int gm = 16;  // ~16 row tiles x ~9 column tiles in flight: A and W blocks balanced within L2
     dim3 grid((unsigned)(tiles < sms ? tiles : sms));
-    bi_gemm_bf16_tc_kernel<BN><<<grid, THREADS, Tile<BN>::SMEM_BYTES, stream>>>(tmA, tmW, C, (int)M, (int)N, (int)K,
-                                                                                 c_bf16 ? 1 : 0, gm, err);
+    if (bi::launch_pdl(bi_gemm_bf16_tc_kernel<BN>, grid, dim3(THREADS), Tile<BN>::SMEM_BYTES, stream, 1u, tmA, tmW, C,
+                       (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, err) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -742,12 +751,14 @@ int launch_gemm_pair(const void* A, int64_t lda, const void* W, int64_t ldw, voi
     const int gm = 16;  // row tiles per group of the tile walk (L2 reuse of A and W blocks)
     const int64_t pairs = units < clusters ? units : clusters;
     const dim3 grid((unsigned)(2 * pairs));
-    if (splits > 1)
-        bi_gemm_bf16_pair_kernel<true><<<grid, THREADS, pair::SMEM_BYTES, stream>>>(
-            tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, splits, cnt, part, err);
-    else
-        bi_gemm_bf16_pair_kernel<false><<<grid, THREADS, pair::SMEM_BYTES, stream>>>(
-            tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, 1, nullptr, nullptr, err);
+    // the pair kernel's cluster shape is compiled in (__cluster_dims__)
+    const cudaError_t e =
+        splits > 1 ? bi::launch_pdl(bi_gemm_bf16_pair_kernel<true>, grid, dim3(THREADS), pair::SMEM_BYTES, stream, 1u,
+                                    tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, splits, cnt, part, err)
+                   : bi::launch_pdl(bi_gemm_bf16_pair_kernel<false>, grid, dim3(THREADS), pair::SMEM_BYTES, stream,
+                                    1u, tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, 1,
+                                    static_cast<uint32_t*>(nullptr), static_cast<float*>(nullptr), err);
+    if (e != cudaSuccess) return BI_ERR_CUDA;
     return bi::launch_status();
 }
 

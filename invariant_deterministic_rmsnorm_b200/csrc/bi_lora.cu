@@ -7,21 +7,21 @@
 // is identical under replay.
 //
 // Shrink, t[M, r] = x[M, K] . A[K, r]:
-//   One thread-block cluster of `split` CTAs per 64-row tile.  CTA s of the cluster computes
-//   the partial P_s over its contiguous K slice [s*K/split, (s+1)*K/split).  A producer warp
-//   streams 64-wide K chunks of x and A into a 6-stage shared-memory ring with TMA.  Four
-//   warps accumulate with mma.sync m16n8k16 (bf16 in, fp32 accumulate), K ascending.  The
-//   partial lands in the CTA's shared memory.  After a cluster barrier, CTA 0 reads the
-//   partials of CTAs 1..split-1 over distributed shared memory and adds them in slice order:
-//   t = ((P_0 + P_1) + P_2) + ... + P_{split-1}, every add rounded to nearest.  There is no
-//   workspace, no atomic and no extra HBM traffic.  The split count and slice size depend
-//   only on (K, split), never on M.
+//   The partial P_s of slice s covers the contiguous K slice [s*K/split, (s+1)*K/split).  It is
+//   accumulated with mma.sync m16n8k16 (bf16 in, fp32 accumulate), 16-deep K steps in ascending
+//   order, starting from zero.  The output is t = ((P_0 + P_1) + P_2) + ... + P_{split-1}, every
+//   add rounded to nearest.  There is no atomic, and the split count and slice size depend only
+//   on (K, split), never on M.  A thread-block cluster of `split` CTAs computes 128-row tiles:
+//   CTA s streams x and A of its slice through a TMA ring, eight compute warps own 16 rows each,
+//   and the partials meet on chip (distributed shared memory), never in HBM.  The ordered kernel
+//   (lora_shrink_ordered_kernel) is persistent and spreads the combine over every CTA of the
+//   cluster; the atomic comparator (lora_shrink_kernel) adds the partials into t with
+//   floating-point atomics instead.
 //
 // Expand, y[M, N] += scale * bf16(t)[M, r] . B[r, N]:
 //   64 x 128 tiles of y per CTA.  t is rounded to bf16 (nearest even) into shared memory,
-//   zero-padded to 16 when r = 8.  The product comes from mma.sync into fp32 and is staged
-//   in shared memory.  Then y is read and written with coalesced 128-bit accesses:
-//   y = round(fma(scale, delta, y)).
+//   zero-padded to 16 when r = 8.  The product comes from mma.sync into fp32 registers and goes
+//   straight to y in 16-byte pieces: y = round(fma(scale, delta, y)).
 #include <mutex>
 
 #include "bi_common.cuh"
@@ -54,10 +54,12 @@ struct ShrinkLayout {
     static constexpr uint32_t A_MASK = R == 64 ? 7u : (R == 32 ? 3u : (R == 16 ? 1u : 0u));
 };
 
-template <int R, bool ATOMIC>
+// The comparator: one CTA per (128-row tile, K slice), partials added into t by floating-point
+// atomics in whatever order the CTAs finish.
+template <int R>
 __global__ void __launch_bounds__(SH_THREADS, 1)
-lora_shrink_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
-                   float* __restrict__ t, int M, int KS, int split, uint32_t* err) {
+lora_shrink_atomic_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
+                          float* __restrict__ t, int M, int KS, uint32_t* err) {
     using L = ShrinkLayout<R>;
     extern __shared__ uint8_t smem_raw[];
     constexpr int SH_STAGES = L::STAGES;
@@ -70,7 +72,7 @@ lora_shrink_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const uint32_t slice = ATOMIC ? blockIdx.y : cluster_ctarank();
+    const uint32_t slice = blockIdx.y;
     const int m0 = blockIdx.x * SH_TM;
     const int kbase = (int)slice * KS;
     const int nchunks = KS / SH_KC;
@@ -159,44 +161,231 @@ lora_shrink_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
         }
     }
 
-    __syncwarp();  // reconverge each warp before the block / cluster barriers below
-    if constexpr (ATOMIC) {
-        // Comparator only: partials are added to t in whatever order the CTAs arrive.
-        __syncthreads();
-        for (int i = tid; i < SH_TM * R; i += SH_THREADS) {
-            const int row = i / R, col = i % R;
-            if (m0 + row < M) atomicAdd(t + (size_t)(m0 + row) * R + col, part[i]);
-        }
-    } else {
-        cluster_sync();  // every partial of the cluster is complete and visible
-        if (slice == 0) {
-            for (int i = tid; i < SH_TM * R / 4; i += SH_THREADS) {
-                const uint32_t la = smem_u32(part + 4 * i);
-                float4 v = *reinterpret_cast<const float4*>(part + 4 * i);
-                // every peer's piece is requested before the first is used (one round trip, not
-                // split - 1); the adds below still run in slice order
-                float4 p[SH_MAX_SPLIT];
-#pragma unroll
-                for (int s = 1; s < SH_MAX_SPLIT; ++s)
-                    if (s < split) p[s] = ld_dsmem_v4(mapa(la, (uint32_t)s));
-#pragma unroll
-                for (int s = 1; s < SH_MAX_SPLIT; ++s) {
-                    if (s < split) {
-                        v.x = __fadd_rn(v.x, p[s].x);
-                        v.y = __fadd_rn(v.y, p[s].y);
-                        v.z = __fadd_rn(v.z, p[s].z);
-                        v.w = __fadd_rn(v.w, p[s].w);
-                    }
-                }
-                const int row = (4 * i) / R, col = (4 * i) % R;
-                if (m0 + row < M) *reinterpret_cast<float4*>(t + (size_t)(m0 + row) * R + col) = v;
-            }
-        }
-        cluster_sync();  // peers keep their shared memory until the leader has read it
+    __syncwarp();
+    __syncthreads();
+    for (int i = tid; i < SH_TM * R; i += SH_THREADS) {
+        const int row = i / R, col = i % R;
+        if (m0 + row < M) atomicAdd(t + (size_t)(m0 + row) * R + col, part[i]);
     }
 }
 
+// ------------------------------------------------------------------ shrink, ordered combine
+// The batch-invariant shrink.  Each output element is computed exactly as described at the top
+// of this file: slice s's partial is one mma.sync chain over its K slice, and the partials are
+// added in slice order.  What this kernel changes is where and when that happens:
+//   - Persistent clusters.  A cluster of `split` CTAs (CTA s = slice s) walks 128-row tiles
+//     c, c + clusters, ...; its producer warp keeps one TMA ring streaming across tiles, so a
+//     cluster's second tile loads while its first is being combined.
+//   - Distributed, pushed combine.  Compute warp w owns rows [16w, 16w + 16) of the tile.  When
+//     its chain ends, it stores its fragment of the partial (st.async) straight into the shared
+//     memory of the CTA that combines those rows: CTA d = w * split / 8 combines rows
+//     [128 d / split, 128 (d + 1) / split).  The stores complete bytes on d's receive barrier.
+//     A combiner warp in every CTA then adds its rows' split partials from its own shared memory,
+//     in slice order, and writes t.  Every CTA combines; no CTA reads a peer's shared memory.
+//   - Receive buffers rotate (two for r <= 16, one above), and a combiner hands a buffer back to
+//     the senders with a remote arrive once it has read it.
+// Every wait is bounded.  A cluster barrier at the end keeps each CTA's shared memory alive until
+// no peer can still write into it.
+constexpr int SO_CWARPS = 8;
+constexpr int SO_THREADS = (SO_CWARPS + 2) * 32;  // compute warps, a producer warp, a combiner warp
+
+template <int R>
+struct OrderedLayout {
+    static constexpr int X_STAGE = SH_TM * SH_KC * 2;  // 16 KB, 128B-swizzled rows of 64 K
+    static constexpr int A_STAGE = SH_KC * R * 2;
+    static constexpr int STAGE = X_STAGE + A_STAGE;
+    static constexpr int NB = R >= 32 ? 1 : 2;         // receive buffers
+    static constexpr int RECV = SH_TM * R * 4;         // one buffer: [slice][rows this CTA combines][R] fp32
+    // two CTAs per SM: at most 112 KB each, including the 1 KB alignment pad and the barriers
+    static constexpr int BUDGET = 112 * 1024 - 1024 - 256;
+    static constexpr int STAGES_FIT = (BUDGET - NB * RECV) / STAGE;
+    static constexpr int STAGES = STAGES_FIT > SH_MAX_STAGES ? SH_MAX_STAGES : STAGES_FIT;
+    static_assert(STAGES >= 3, "the ring needs at least three stages");
+    static constexpr int RECV_OFF = STAGES * STAGE;
+    static constexpr int BAR_OFF = RECV_OFF + NB * RECV;
+    // full[STAGES], empty[STAGES], rfull[NB], rfree[NB][SH_MAX_SPLIT], then the abort flag
+    static constexpr int NBARS = 2 * STAGES + NB + NB * SH_MAX_SPLIT;
+    static constexpr size_t BYTES = 1024 + (size_t)BAR_OFF + NBARS * 8 + 16;
+    static constexpr uint32_t A_MASK = R == 64 ? 7u : (R == 32 ? 3u : (R == 16 ? 1u : 0u));
+};
+
+template <int R>
+__global__ void __launch_bounds__(SO_THREADS, 2)
+lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
+                           float* __restrict__ t, int M, int KS, int split, int n_tiles, uint32_t* err) {
+    using L = OrderedLayout<R>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* recv = reinterpret_cast<float*>(base + L::RECV_OFF);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::BAR_OFF);
+    uint64_t* empty = full + L::STAGES;
+    uint64_t* rfull = empty + L::STAGES;        // [NB]: every slice's partial of this CTA's rows has landed
+    uint64_t* rfree = rfull + L::NB;            // [NB][8]: CTA d's receive buffer b may be written again
+    volatile int* abort = reinterpret_cast<volatile int*>(rfree + L::NB * SH_MAX_SPLIT);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const uint32_t slice = cluster_ctarank();
+    const int kbase = (int)slice * KS;
+    const int nchunks = KS / SH_KC;
+    const int rows_per = SH_TM / split;  // rows of a tile that each CTA combines
+    constexpr uint32_t RECV_TX = (uint32_t)L::RECV;  // bytes a combiner receives per tile
+
+    if (tid == 0) {
+        for (int i = 0; i < L::STAGES; ++i) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), SO_CWARPS);
+        }
+        for (int b = 0; b < L::NB; ++b) {
+            mbar_init(smem_u32(&rfull[b]), 1);
+            for (int d = 0; d < SH_MAX_SPLIT; ++d) mbar_init(smem_u32(&rfree[b * SH_MAX_SPLIT + d]), 1);
+        }
+        *abort = 0;
+        fence_barrier_init();
+        fence_proxy_async_shared();
+    }
+    __syncthreads();
+    cluster_sync();  // every CTA's barriers exist before any signal crosses the cluster
+    pdl_wait();      // x and A may come from the kernel before this one; it may still read t
+    pdl_trigger();
+
+    if (warp == SO_CWARPS) {
+        // ------------------------------------------------ producer: one ring across all tiles
+        if (lane == 0) {
+            prefetch_tmap(&tmX);
+            prefetch_tmap(&tmA);
+            uint32_t it = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
+                for (int c = 0; c < nchunks; ++c, ++it) {
+                    const int st = (int)(it % L::STAGES);
+                    const uint32_t round = it / L::STAGES;
+                    if (!mbar_wait(smem_u32(&empty[st]), (round & 1u) ^ 1u, abort)) {
+                        atomicOr(err, bi::DEVERR_WAIT_TMA);
+                        *abort = 1;
+                        break;
+                    }
+                    uint8_t* sx = base + st * L::STAGE;
+                    const uint32_t fb = smem_u32(&full[st]);
+                    mbar_arrive_expect_tx(fb, L::STAGE);
+                    tma_load_2d(smem_u32(sx), &tmX, kbase + c * SH_KC, tile * SH_TM, fb);
+                    tma_load_2d(smem_u32(sx + L::X_STAGE), &tmA, 0, kbase + c * SH_KC, fb);
+                }
+            }
+            if (*abort) {  // let loads already in flight land before the shared memory is released
+                for (uint32_t i = it > (uint32_t)L::STAGES ? it - L::STAGES : 0u; i < it; ++i)
+                    (void)mbar_wait(smem_u32(&full[i % L::STAGES]), (i / L::STAGES) & 1u, nullptr);
+            }
+        }
+    } else if (warp == SO_CWARPS + 1) {
+        // ------------------------------------------------ combiner: this CTA's rows of every tile
+        int j = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
+            const int b = j % L::NB;
+            const uint32_t par = (uint32_t)(j / L::NB) & 1u;
+            if (lane == 0) mbar_arrive_expect_tx(smem_u32(&rfull[b]), RECV_TX);
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&rfull[b]), par, abort));
+            if (!ok) {
+                if (lane == 0) atomicOr(err, bi::DEVERR_WAIT_CLUSTER);
+                *abort = 1;
+                break;
+            }
+            const float* rb = recv + b * (SH_TM * R);  // [slice][rows_per][R]
+            const int row0 = tile * SH_TM + (int)slice * rows_per;
+            for (int i = lane; i < rows_per * R / 4; i += 32) {
+                const int row = (4 * i) / R, col = (4 * i) % R;
+                float4 v = *reinterpret_cast<const float4*>(rb + row * R + col);
+                for (int sl = 1; sl < split; ++sl) {  // ((P0 + P1) + P2) + ...: slice order
+                    const float4 p = *reinterpret_cast<const float4*>(rb + (sl * rows_per + row) * R + col);
+                    v.x = __fadd_rn(v.x, p.x);
+                    v.y = __fadd_rn(v.y, p.y);
+                    v.z = __fadd_rn(v.z, p.z);
+                    v.w = __fadd_rn(v.w, p.w);
+                }
+                if (row0 + row < M) *reinterpret_cast<float4*>(t + (size_t)(row0 + row) * R + col) = v;
+            }
+            __syncwarp();
+            // buffer b of this CTA has been read: every sender in the cluster may refill it
+            if (lane < split) mbar_arrive_cluster(mapa(smem_u32(&rfree[b * SH_MAX_SPLIT + slice]), (uint32_t)lane));
+        }
+    } else {
+        // ------------------------------------------------ compute warps
+        const int d = warp * split / SO_CWARPS;            // the CTA that combines this warp's rows
+        const int lrow0 = warp * 16 - d * rows_per;        // first of them inside d's share
+        const uint32_t peer_recv = mapa(smem_u32(recv), (uint32_t)d);
+        const uint32_t peer_rfull = mapa(smem_u32(rfull), (uint32_t)d);
+        const int g = lane >> 2, q = lane & 3;
+        uint32_t it = 0;
+        int j = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
+            float acc[R / 8][4];
+#pragma unroll
+            for (int nt = 0; nt < R / 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+            bool ok = true;
+            for (int c = 0; c < nchunks; ++c, ++it) {
+                const int st = (int)(it % L::STAGES);
+                const uint32_t round = it / L::STAGES;
+                // ldmatrix / mma.sync are warp-collective: the whole warp leaves together on a timeout
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), round & 1u, abort));
+                if (!ok) {
+                    if (lane == 0) atomicOr(err, bi::DEVERR_WAIT_FULL);
+                    *abort = 1;
+                    break;
+                }
+                const uint32_t xs = smem_u32(base + st * L::STAGE);
+                const uint32_t as = xs + L::X_STAGE;
+#pragma unroll
+                for (int kk = 0; kk < SH_KC / 16; ++kk) {
+                    uint32_t a[4];
+                    const int row = warp * 16 + (lane & 15);
+                    const int kb = (kk * 16 + (lane >> 4) * 8) * 2;
+                    ldmatrix_x4(swz(xs + row * 128 + kb, 7u), a);
+#pragma unroll
+                    for (int nt = 0; nt < R / 8; ++nt) {
+                        uint32_t bf[2];
+                        const int krow = kk * 16 + (lane & 15);
+                        ldmatrix_x2_trans(swz(as + krow * (2 * R) + nt * 16, L::A_MASK), bf);
+                        mma_m16n8k16_bf16(acc[nt], a, bf);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+            }
+            if (!ok) break;
+            const int b = j % L::NB;
+            const uint32_t par = (uint32_t)(j / L::NB) & 1u;
+            // d has read what this warp pushed into buffer b for tile j - NB
+            ok = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&rfree[b * SH_MAX_SPLIT + d]), par ^ 1u, abort));
+            if (!ok) {
+                if (lane == 0) atomicOr(err, bi::DEVERR_WAIT_CLUSTER);
+                *abort = 1;
+                break;
+            }
+            // rows lrow0 + g and lrow0 + g + 8 of this slice's block in d's buffer b
+            const uint32_t dst = peer_recv + (uint32_t)((b * SH_TM * R + ((int)slice * rows_per + lrow0 + g) * R) * 4);
+            const uint32_t bar = peer_rfull + (uint32_t)b * 8u;
+#pragma unroll
+            for (int nt = 0; nt < R / 8; ++nt) {
+                const uint32_t col = (uint32_t)(nt * 8 + q * 2) * 4u;
+                st_async_v2(dst + col, acc[nt][0], acc[nt][1], bar);
+                st_async_v2(dst + (uint32_t)(8 * R * 4) + col, acc[nt][2], acc[nt][3], bar);
+            }
+        }
+    }
+    // no CTA leaves while a peer may still store into its shared memory or signal its barriers
+    __syncwarp();
+    cluster_sync();
+}
+
 // ------------------------------------------------------------------ expand
+// A CTA owns a 64 x 128 tile of y; warp (wr, wc) owns rows [16 wr, 16 wr + 16) and columns
+// [64 wc, 64 wc + 64) of it.  The B tile is staged with its columns permuted inside each group
+// of 32, so that the mma.sync accumulator of lane (g, q) holds, for rows g and g + 8, the 8
+// CONSECUTIVE output columns [8q, 8q + 8) of every group: the product goes straight from the
+// accumulator registers to y in 16-byte pieces, with no trip through shared memory.  Column
+// L = 8p + 2q + e of a group in shared memory (p, e: the MMA's n-tile and pair element) holds
+// the weights of output column 8q + 2p + e.  Each output element is still one MMA chain over
+// r, so the permutation moves work between lanes and changes no arithmetic.
 constexpr int EX_TM = 64;
 constexpr int EX_TN = 128;
 constexpr int EX_THREADS = 256;
@@ -205,11 +394,10 @@ template <int R>
 struct ExpandLayout {
     static constexpr int RP = R < 16 ? 16 : R;       // K of the MMA, padded with zeros
     static constexpr int T_PITCH = RP * 2 + 16;       // bytes per row of bf16(t); +16 avoids bank conflicts
-    static constexpr int B_PITCH = EX_TN * 2 + 16;    // bytes per K-row of the B tile
-    static constexpr int D_PITCH = EX_TN + 8;         // floats per row of the staged product (conflict-free)
+    static constexpr int B_PITCH = EX_TN * 2 + 16;    // bytes per K-row of the permuted B tile
     static constexpr int T_BYTES = EX_TM * T_PITCH;
     static constexpr int B_BYTES = RP * B_PITCH;
-    static constexpr size_t BYTES = (size_t)T_BYTES + B_BYTES + EX_TM * D_PITCH * 4;
+    static constexpr size_t BYTES = (size_t)T_BYTES + B_BYTES;
 };
 
 template <int R, bool YBF16>
@@ -220,34 +408,41 @@ lora_expand_kernel(const float* __restrict__ t, const __nv_bfloat16* __restrict_
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* sT = smem;
     uint8_t* sB = smem + L::T_BYTES;
-    float* sD = reinterpret_cast<float*>(smem + L::T_BYTES + L::B_BYTES);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
+    const int wr = warp >> 1, wc = warp & 1;
+    const int g = lane >> 2, q = lane & 3;
     const int m0 = blockIdx.y * EX_TM;
     const int n0 = blockIdx.x * EX_TN;
 
-    // 0. Issue this thread's loads of the y tile first: their HBM latency overlaps steps 1-3.
-    //    A chunk is 4 consecutive elements of a row (8 bytes of bf16 or 16 of fp32), so that the
-    //    matching 16 bytes of the staged product are read without bank conflicts.
-    constexpr int CPR = EX_TN / 4;                              // chunks per tile row
-    constexpr int NCH = EX_TM * CPR / EX_THREADS;               // chunks per thread (8)
-    uint4 yv[NCH];
+    pdl_wait();  // t and y may come from the kernels just before this one
+
+    // 0. This lane's pieces of y: rows g and g + 8 of the warp's strip, columns [8q, 8q + 8) of
+    //    each of the warp's two 32-column groups.  Issued first: their HBM latency overlaps 1-3.
+    //    A piece is 8 elements: one 16-byte load in bf16, two in fp32.
+    constexpr int W = YBF16 ? 1 : 2;  // 16-byte words per piece
+    uint4 yv[2][2][W];                // [row half][group][word]
+    bool live[2][2];
 #pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        const int i = tid + k * EX_THREADS;
-        const int row = i / CPR, cc = i % CPR;
-        const int col = n0 + cc * 4;
-        yv[k] = make_uint4(0u, 0u, 0u, 0u);
-        if (m0 + row < M && col < N) {
-            if constexpr (YBF16) {
-                const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(y) +
-                                                                 (size_t)(m0 + row) * ldy + col);
-                yv[k].x = u.x;
-                yv[k].y = u.y;
-            } else {
-                yv[k] = *reinterpret_cast<const uint4*>(static_cast<const float*>(y) + (size_t)(m0 + row) * ldy + col);
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int G = 0; G < 2; ++G) {
+            const int row = m0 + wr * 16 + g + 8 * h;
+            const int col = n0 + wc * 64 + G * 32 + 8 * q;
+            live[h][G] = row < M && col < N;  // N % 8 == 0: a piece is wholly inside or outside
+#pragma unroll
+            for (int w = 0; w < W; ++w) yv[h][G][w] = make_uint4(0u, 0u, 0u, 0u);
+            if (live[h][G]) {
+                if constexpr (YBF16) {
+                    yv[h][G][0] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(y) +
+                                                                  (size_t)row * ldy + col);
+                } else {
+                    const float* p = static_cast<const float*>(y) + (size_t)row * ldy + col;
+                    yv[h][G][0] = *reinterpret_cast<const uint4*>(p);
+                    yv[h][G][1] = *reinterpret_cast<const uint4*>(p + 4);
+                }
             }
         }
     }
@@ -260,18 +455,24 @@ lora_expand_kernel(const float* __restrict__ t, const __nv_bfloat16* __restrict_
         uint2 p = make_uint2(bi::pack_bf16x2(v.x, v.y), bi::pack_bf16x2(v.z, v.w));
         *reinterpret_cast<uint2*>(sT + row * L::T_PITCH + k * 2) = p;
     }
-    // 2. The B tile [R, 128] (columns past N and rows past R are zero).
+    // 2. The B tile [R, 128], permuted: the 8 weights of output columns [8c, 8c + 8) (c = 4 gg + qq)
+    //    go, two at a time, to shared-memory columns 32 gg + 8 p + 2 qq, p = 0..3.  Columns past N
+    //    and rows past R are zero.
     for (int i = tid; i < L::RP * (EX_TN / 8); i += EX_THREADS) {
-        const int k = i / (EX_TN / 8), cc = i % (EX_TN / 8);
-        const int col = n0 + cc * 8;
+        const int k = i / (EX_TN / 8), c = i % (EX_TN / 8);
+        const int col = n0 + c * 8;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (k < R && col < N) v = bi::ld_cached_v4(B + (size_t)k * N + col);
-        *reinterpret_cast<uint4*>(sB + k * L::B_PITCH + cc * 16) = v;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(sB + k * L::B_PITCH) + 16 * (c >> 2) + (c & 3);
+        dst[0] = v.x;
+        dst[4] = v.y;
+        dst[8] = v.z;
+        dst[12] = v.w;
     }
     __syncthreads();
+    pdl_trigger();
 
-    // 3. delta[16 rows x 64 cols] per warp with mma.sync.
-    const int wr = warp >> 1, wc = warp & 1;
+    // 3. delta[16 rows x 64 cols] per warp with mma.sync (shared-memory column order).
     float acc[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
@@ -287,39 +488,42 @@ lora_expand_kernel(const float* __restrict__ t, const __nv_bfloat16* __restrict_
             mma_m16n8k16_bf16(acc[nt], a, b);
         }
     }
-    const int g = lane >> 2, q = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-        const int col = wc * 64 + nt * 8 + q * 2;
-        *reinterpret_cast<float2*>(sD + (wr * 16 + g) * L::D_PITCH + col) = make_float2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<float2*>(sD + (wr * 16 + g + 8) * L::D_PITCH + col) = make_float2(acc[nt][2], acc[nt][3]);
-    }
-    __syncthreads();
 
-    // 4. y = round(fma(scale, delta, y)) with coalesced 128-bit accesses.
+    // 4. y = round(fma(scale, delta, y)).  In group G, n-tile p = 0..3 of the accumulator holds
+    //    output columns 8q + 2p + {0, 1} of row g (elements 0, 1) and row g + 8 (elements 2, 3).
 #pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        const int i = tid + k * EX_THREADS;
-        const int row = i / CPR, cc = i % CPR;
-        const int col = n0 + cc * 4;
-        if (m0 + row >= M || col >= N) continue;
-        const float4 d = *reinterpret_cast<const float4*>(sD + row * L::D_PITCH + cc * 4);
-        if constexpr (YBF16) {
-            const float a0 = __fmaf_rn(scale, d.x, bi::bf16_lo(yv[k].x));
-            const float a1 = __fmaf_rn(scale, d.y, bi::bf16_hi(yv[k].x));
-            const float a2 = __fmaf_rn(scale, d.z, bi::bf16_lo(yv[k].y));
-            const float a3 = __fmaf_rn(scale, d.w, bi::bf16_hi(yv[k].y));
-            __nv_bfloat16* p = static_cast<__nv_bfloat16*>(y) + (size_t)(m0 + row) * ldy + col;
-            *reinterpret_cast<uint2*>(p) = make_uint2(bi::pack_bf16x2(a0, a1), bi::pack_bf16x2(a2, a3));
-        } else {
-            float4 v = make_float4(__uint_as_float(yv[k].x), __uint_as_float(yv[k].y), __uint_as_float(yv[k].z),
-                                   __uint_as_float(yv[k].w));
-            v.x = __fmaf_rn(scale, d.x, v.x);
-            v.y = __fmaf_rn(scale, d.y, v.y);
-            v.z = __fmaf_rn(scale, d.z, v.z);
-            v.w = __fmaf_rn(scale, d.w, v.w);
-            float* p = static_cast<float*>(y) + (size_t)(m0 + row) * ldy + col;
-            *reinterpret_cast<float4*>(p) = v;
+    for (int h = 0; h < 2; ++h) {
+        const int row = m0 + wr * 16 + g + 8 * h;
+#pragma unroll
+        for (int G = 0; G < 2; ++G) {
+            if (!live[h][G]) continue;
+            const int col = n0 + wc * 64 + G * 32 + 8 * q;
+            float d[8];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                d[2 * p] = acc[G * 4 + p][2 * h];
+                d[2 * p + 1] = acc[G * 4 + p][2 * h + 1];
+            }
+            if constexpr (YBF16) {
+                const uint4 u = yv[h][G][0];
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    o[j] = bi::pack_bf16x2(__fmaf_rn(scale, d[2 * j], bi::bf16_lo(w4[j])),
+                                           __fmaf_rn(scale, d[2 * j + 1], bi::bf16_hi(w4[j])));
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + (size_t)row * ldy + col) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
+            } else {
+                float* p = static_cast<float*>(y) + (size_t)row * ldy + col;
+                const uint4 u0 = yv[h][G][0], u1 = yv[h][G][1];
+                *reinterpret_cast<float4*>(p) = make_float4(
+                    __fmaf_rn(scale, d[0], __uint_as_float(u0.x)), __fmaf_rn(scale, d[1], __uint_as_float(u0.y)),
+                    __fmaf_rn(scale, d[2], __uint_as_float(u0.z)), __fmaf_rn(scale, d[3], __uint_as_float(u0.w)));
+                *reinterpret_cast<float4*>(p + 4) = make_float4(
+                    __fmaf_rn(scale, d[4], __uint_as_float(u1.x)), __fmaf_rn(scale, d[5], __uint_as_float(u1.y)),
+                    __fmaf_rn(scale, d[6], __uint_as_float(u1.z)), __fmaf_rn(scale, d[7], __uint_as_float(u1.w)));
+            }
         }
     }
 }
@@ -347,11 +551,11 @@ bool set_smem_once(F kernel, size_t bytes) {
     return true;
 }
 
-template <int R, bool ATOMIC>
-int launch_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K, int split, cudaStream_t s) {
+template <int R>
+int launch_shrink_atomic(const void* x, const void* A, float* t, int64_t M, int64_t K, int split, cudaStream_t s) {
     using L = ShrinkLayout<R>;
     uint32_t* err = bi::device_error_word();
-    auto kern = lora_shrink_kernel<R, ATOMIC>;
+    auto kern = lora_shrink_atomic_kernel<R>;
     if (!err || !set_smem_once(kern, L::BYTES)) return BI_ERR_CUDA;
     CUtensorMap tmX, tmA;
     if (!bi::make_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2,
@@ -360,34 +564,94 @@ int launch_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K, 
     if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)R, (uint64_t)K, (uint64_t)R * 2, R,
                           SH_KC, bi::swizzle_for(R * 2)))
         return BI_ERR_CUDA;
-    const int KS = (int)(K / split);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((M + SH_TM - 1) / SH_TM), (unsigned)split, 1);
-    cfg.blockDim = dim3(SH_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = L::BYTES;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    if (!ATOMIC) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 1;
-        attr[0].val.clusterDim.y = (unsigned)split;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+    dim3 grid((unsigned)((M + SH_TM - 1) / SH_TM), (unsigned)split, 1);
+    kern<<<grid, SH_THREADS, L::BYTES, s>>>(tmX, tmA, t, (int)M, (int)(K / split), err);
+    return bi::launch_status();
+}
+
+// Clusters of the ordered kernel that fit on the device at once, per (R, split); queried once per
+// device.  The grid never exceeds it, so every cluster is resident and walks its tiles; a larger
+// grid would only queue clusters behind the first wave.
+template <int R>
+int ordered_clusters(int split) {
+    static std::mutex mu;
+    static int cached[64][4];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    const int si = split == 1 ? 0 : (split == 2 ? 1 : (split == 4 ? 2 : 3));
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev][si] == 0) {
+        using L = OrderedLayout<R>;
+        int n = 0;
+        if (split == 1) {
+            int per_sm = 0, sms = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lora_shrink_ordered_kernel<R>, SO_THREADS,
+                                                              L::BYTES) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return -1;
+            n = per_sm * sms;
+        } else {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(1, (unsigned)split, 1);
+            cfg.blockDim = dim3(SO_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = L::BYTES;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1;
+            attr[0].val.clusterDim.y = (unsigned)split;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, lora_shrink_ordered_kernel<R>, &cfg) != cudaSuccess) return -1;
+        }
+        cached[dev][si] = n > 0 ? n : 1;
     }
-    if (cudaLaunchKernelEx(&cfg, kern, tmX, tmA, t, (int)M, KS, split, err) != cudaSuccess) return BI_ERR_CUDA;
+    return cached[dev][si];
+}
+
+template <int R>
+int launch_shrink_ordered(const void* x, const void* A, float* t, int64_t M, int64_t K, int split, cudaStream_t s) {
+    using L = OrderedLayout<R>;
+    uint32_t* err = bi::device_error_word();
+    auto kern = lora_shrink_ordered_kernel<R>;
+    if (!err || !set_smem_once(kern, L::BYTES)) return BI_ERR_CUDA;
+    const int fit = ordered_clusters<R>(split);
+    if (fit <= 0) return BI_ERR_CUDA;
+    CUtensorMap tmX, tmA;
+    if (!bi::make_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2,
+                          SH_KC, SH_TM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)R, (uint64_t)K, (uint64_t)R * 2, R,
+                          SH_KC, bi::swizzle_for(R * 2)))
+        return BI_ERR_CUDA;
+    const int n_tiles = (int)((M + SH_TM - 1) / SH_TM);
+    const int clusters = n_tiles < fit ? n_tiles : fit;
+    if (bi::launch_pdl(kern, dim3((unsigned)clusters, (unsigned)split), dim3(SO_THREADS), L::BYTES, s,
+                       (unsigned)split, tmX, tmA, t, (int)M, (int)(K / split), (int)split, n_tiles,
+                       err) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
 template <bool ATOMIC>
 int shrink_dispatch(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r, int32_t split,
                     cudaStream_t s) {
-    switch (r) {
-        case 8: return launch_shrink<8, ATOMIC>(x, A, t, M, K, split, s);
-        case 16: return launch_shrink<16, ATOMIC>(x, A, t, M, K, split, s);
-        case 32: return launch_shrink<32, ATOMIC>(x, A, t, M, K, split, s);
-        case 64: return launch_shrink<64, ATOMIC>(x, A, t, M, K, split, s);
-        default: return BI_ERR_UNSUPPORTED_SHAPE;
+    if constexpr (!ATOMIC) {
+        switch (r) {
+            case 8: return launch_shrink_ordered<8>(x, A, t, M, K, split, s);
+            case 16: return launch_shrink_ordered<16>(x, A, t, M, K, split, s);
+            case 32: return launch_shrink_ordered<32>(x, A, t, M, K, split, s);
+            case 64: return launch_shrink_ordered<64>(x, A, t, M, K, split, s);
+            default: return BI_ERR_UNSUPPORTED_SHAPE;
+        }
+    } else {
+        switch (r) {
+            case 8: return launch_shrink_atomic<8>(x, A, t, M, K, split, s);
+            case 16: return launch_shrink_atomic<16>(x, A, t, M, K, split, s);
+            case 32: return launch_shrink_atomic<32>(x, A, t, M, K, split, s);
+            case 64: return launch_shrink_atomic<64>(x, A, t, M, K, split, s);
+            default: return BI_ERR_UNSUPPORTED_SHAPE;
+        }
     }
 }
 
@@ -408,15 +672,11 @@ int launch_expand(const float* t, const void* B, void* y, int64_t M, int64_t N, 
                   cudaStream_t s) {
     using L = ExpandLayout<R>;
     dim3 grid((unsigned)((N + EX_TN - 1) / EX_TN), (unsigned)((M + EX_TM - 1) / EX_TM));
-    if (ybf16) {
-        auto k = lora_expand_kernel<R, true>;
-        if (!set_smem_once(k, L::BYTES)) return BI_ERR_CUDA;
-        k<<<grid, EX_THREADS, L::BYTES, s>>>(t, static_cast<const __nv_bfloat16*>(B), y, (int)M, (int)N, ldy, scale);
-    } else {
-        auto k = lora_expand_kernel<R, false>;
-        if (!set_smem_once(k, L::BYTES)) return BI_ERR_CUDA;
-        k<<<grid, EX_THREADS, L::BYTES, s>>>(t, static_cast<const __nv_bfloat16*>(B), y, (int)M, (int)N, ldy, scale);
-    }
+    auto k = ybf16 ? lora_expand_kernel<R, true> : lora_expand_kernel<R, false>;
+    if (!set_smem_once(k, L::BYTES)) return BI_ERR_CUDA;
+    if (bi::launch_pdl(k, grid, dim3(EX_THREADS), L::BYTES, s, 1u, t, static_cast<const __nv_bfloat16*>(B), y,
+                       (int)M, (int)N, ldy, scale) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 

@@ -11,12 +11,18 @@
 
 #include "bi_common.cuh"
 #include "bi_model.h"
+#include "bi_sm100.cuh"
+
+using bi::sm100::pdl_trigger;
+using bi::sm100::pdl_wait;
 
 namespace {
 
 // ------------------------------------------------------------------ embedding gather
 __global__ void embed_kernel(const int32_t* __restrict__ tokens, const __nv_bfloat16* __restrict__ table,
                              __nv_bfloat16* __restrict__ out, int64_t H, int64_t vocab, uint32_t* err) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
     const int64_t t = blockIdx.x;
     const int32_t id = tokens[t];
     if (id < 0 || id >= vocab) {
@@ -32,6 +38,8 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const __nv_bflo
 // table[p][i] = (cos, sin) of the angle p * theta^(-2i/D) for pair i < D/2, formed in double
 // precision and rounded once to fp32.  Built once per (theta, D, positions); every rotation reads it.
 __global__ void rope_table_kernel(float2* __restrict__ table, int64_t rows, int half, double log_theta, int D) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
     const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= rows * half) return;
     const int64_t p = k / half;
@@ -47,6 +55,8 @@ __global__ void rope_table_kernel(float2* __restrict__ table, int64_t rows, int 
 __global__ void rope_kernel(__nv_bfloat16* __restrict__ x, int64_t ld_row, int heads, int D,
                             const int32_t* __restrict__ pos, const float4* __restrict__ table, int64_t table_rows,
                             uint32_t* err) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
     const int64_t t = blockIdx.x;
     const int half = D / 2, quads = half / 2;  // pairs per head, two at a time
     const int j = blockIdx.y * blockDim.x + threadIdx.x;
@@ -73,6 +83,8 @@ __global__ void rope_kernel(__nv_bfloat16* __restrict__ x, int64_t ld_row, int h
 __global__ void kv_append_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src,
                                  const int32_t* __restrict__ dst_row, __nv_bfloat16* __restrict__ dst,
                                  int64_t row_elems, int64_t dst_rows, uint32_t* err) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
     const int64_t t = blockIdx.x;
     const int64_t r = dst_row[t];
     if (r < 0 || r >= dst_rows) {
@@ -87,6 +99,8 @@ __global__ void kv_append_kernel(const __nv_bfloat16* __restrict__ src, int64_t 
 // ------------------------------------------------------------------ residual add (in place)
 __global__ void add_kernel(__nv_bfloat16* __restrict__ h, int64_t ldh, const __nv_bfloat16* __restrict__ d,
                            int64_t ldd, int64_t N) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
     const int64_t t = blockIdx.x;
     const int64_t i = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;  // 8-element vector of the row
     if (i < N / 8) {
@@ -106,6 +120,8 @@ __global__ void add_kernel(__nv_bfloat16* __restrict__ h, int64_t ldh, const __n
 // out[t, j] = silu(gu[t, j]) * gu[t, N + j] with silu(g) = g / (1 + e^-g), fp32, rounded once.
 __global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ gu, int64_t ld_gu, __nv_bfloat16* __restrict__ out,
                               int64_t ld_out, int64_t N) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
     const int64_t t = blockIdx.x;
     const int64_t i = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;  // 8-element vector of the row
     if (i < N / 8) {
@@ -129,6 +145,8 @@ __global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ gu, int64_t ld_g
 constexpr int ARGMAX_THREADS = 1024;
 __global__ void __launch_bounds__(ARGMAX_THREADS) argmax_kernel(const float* __restrict__ x, int64_t ld, int64_t N,
                                                                 int32_t* __restrict__ out) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
     __shared__ float sv[ARGMAX_THREADS];
     __shared__ int32_t si[ARGMAX_THREADS];
     const int64_t t = blockIdx.x;
@@ -160,6 +178,15 @@ __global__ void __launch_bounds__(ARGMAX_THREADS) argmax_kernel(const float* __r
 
 int rows_ok(int64_t rows) { return rows >= 0 && rows <= 0x7fffffffLL; }
 
+// v[i] += step: the per-step bookkeeping of a replayed decode step (positions, cache rows, KV
+// lengths), so that no device work in the decoder runs outside this library.
+__global__ void advance_kernel(int32_t* __restrict__ v, int64_t n, int32_t step) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) v[i] += step;
+}
+
 }  // namespace
 
 BI_API int bi_embed(const int32_t* tokens, const void* table, void* out, int64_t T, int64_t H, int64_t vocab,
@@ -170,8 +197,10 @@ BI_API int bi_embed(const int32_t* tokens, const void* table, void* out, int64_t
     if (H % 8 != 0 || !bi::aligned16(table) || !bi::aligned16(out)) return BI_ERR_MISALIGNED;
     uint32_t* err = bi::device_error_word();
     if (!err) return BI_ERR_CUDA;
-    embed_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(tokens, static_cast<const __nv_bfloat16*>(table),
-                                                                 static_cast<__nv_bfloat16*>(out), H, vocab, err);
+    if (bi::launch_pdl(embed_kernel, dim3((unsigned)T), dim3(256), 0, bi::as_stream(stream), 1u,
+                       tokens, static_cast<const __nv_bfloat16*>(table), static_cast<__nv_bfloat16*>(out), H, vocab,
+                       err) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -183,8 +212,9 @@ BI_API int bi_rope_table(void* table, int64_t positions, int32_t head_dim, doubl
     const int half = head_dim / 2;
     if (positions > ((int64_t)1 << 38) / half) return BI_ERR_UNSUPPORTED_SHAPE;
     const int64_t n = positions * half;
-    rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, bi::as_stream(stream)>>>(
-        static_cast<float2*>(table), positions, half, log(theta), head_dim);
+    if (bi::launch_pdl(rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, bi::as_stream(stream), 1u,
+                       static_cast<float2*>(table), positions, half, log(theta), head_dim) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -201,8 +231,10 @@ BI_API int bi_rope(void* x, int64_t T, int64_t ld_row, int32_t heads, int32_t he
     const int work = heads * (head_dim / 4);
     if ((work + 127) / 128 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
     dim3 grid((unsigned)T, (unsigned)((work + 127) / 128));
-    rope_kernel<<<grid, 128, 0, bi::as_stream(stream)>>>(static_cast<__nv_bfloat16*>(x), ld_row, heads, head_dim, pos,
-                                                          static_cast<const float4*>(table), table_rows, err);
+    if (bi::launch_pdl(rope_kernel, dim3(grid), dim3(128), 0, bi::as_stream(stream), 1u,
+                       static_cast<__nv_bfloat16*>(x), ld_row, heads, head_dim, pos,
+                       static_cast<const float4*>(table), table_rows, err) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -214,9 +246,10 @@ BI_API int bi_kv_append(const void* src, int64_t ld_src, const int32_t* dst_row,
     if (row_elems % 8 != 0 || ld_src % 8 != 0 || !bi::aligned16(src) || !bi::aligned16(dst)) return BI_ERR_MISALIGNED;
     uint32_t* err = bi::device_error_word();
     if (!err) return BI_ERR_CUDA;
-    kv_append_kernel<<<(unsigned)T, 256, 0, bi::as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(src), ld_src,
-                                                                     dst_row, static_cast<__nv_bfloat16*>(dst),
-                                                                     row_elems, dst_rows, err);
+    if (bi::launch_pdl(kv_append_kernel, dim3((unsigned)T), dim3(256), 0, bi::as_stream(stream), 1u,
+                       static_cast<const __nv_bfloat16*>(src), ld_src, dst_row, static_cast<__nv_bfloat16*>(dst),
+                       row_elems, dst_rows, err) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -226,9 +259,11 @@ BI_API int bi_add(void* h, int64_t ldh, const void* d, int64_t ldd, int64_t T, i
     if (!h || !d) return BI_ERR_INVALID_ARG;
     if (N % 8 != 0 || ldh % 8 != 0 || ldd % 8 != 0 || !bi::aligned16(h) || !bi::aligned16(d)) return BI_ERR_MISALIGNED;
     if ((N / 8 + 255) / 256 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
-    add_kernel<<<dim3((unsigned)T, (unsigned)((N / 8 + 255) / 256)), 256, 0, bi::as_stream(stream)>>>(
-        static_cast<__nv_bfloat16*>(h), ldh,
-                                                                static_cast<const __nv_bfloat16*>(d), ldd, N);
+    if (bi::launch_pdl(add_kernel, dim3((unsigned)T, (unsigned)((N / 8 + 255) / 256)), dim3(256), 0,
+                       bi::as_stream(stream), 1u,
+                       static_cast<__nv_bfloat16*>(h), ldh, static_cast<const __nv_bfloat16*>(d), ldd,
+                       N) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -239,9 +274,11 @@ BI_API int bi_swiglu(const void* gu, int64_t ld_gu, void* out, int64_t ld_out, i
     if (N % 8 != 0 || ld_gu % 8 != 0 || ld_out % 8 != 0 || !bi::aligned16(gu) || !bi::aligned16(out))
         return BI_ERR_MISALIGNED;
     if ((N / 8 + 255) / 256 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
-    swiglu_kernel<<<dim3((unsigned)T, (unsigned)((N / 8 + 255) / 256)), 256, 0, bi::as_stream(stream)>>>(
-        static_cast<const __nv_bfloat16*>(gu), ld_gu,
-                                                                   static_cast<__nv_bfloat16*>(out), ld_out, N);
+    if (bi::launch_pdl(swiglu_kernel, dim3((unsigned)T, (unsigned)((N / 8 + 255) / 256)), dim3(256), 0,
+                       bi::as_stream(stream), 1u,
+                       static_cast<const __nv_bfloat16*>(gu), ld_gu, static_cast<__nv_bfloat16*>(out), ld_out,
+                       N) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -249,6 +286,18 @@ BI_API int bi_argmax(const float* x, int64_t ld, int64_t T, int64_t N, int32_t* 
     if (T < 0 || N <= 0 || ld < N || !rows_ok(T) || N > 0x7fffffffLL) return BI_ERR_INVALID_ARG;
     if (T == 0) return BI_OK;
     if (!x || !out) return BI_ERR_INVALID_ARG;
-    argmax_kernel<<<(unsigned)T, ARGMAX_THREADS, 0, bi::as_stream(stream)>>>(x, ld, N, out);
+    if (bi::launch_pdl(argmax_kernel, dim3((unsigned)T), dim3(ARGMAX_THREADS), 0, bi::as_stream(stream), 1u,
+                       x, ld, N, out) != cudaSuccess)
+        return BI_ERR_CUDA;
+    return bi::launch_status();
+}
+
+BI_API int bi_advance(int32_t* v, int64_t n, int32_t step, void* stream) {
+    if (n < 0 || n > ((int64_t)1 << 40)) return BI_ERR_INVALID_ARG;
+    if (n == 0) return BI_OK;
+    if (!v) return BI_ERR_INVALID_ARG;
+    if (bi::launch_pdl(advance_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, bi::as_stream(stream), 1u,
+                       v, n, step) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }

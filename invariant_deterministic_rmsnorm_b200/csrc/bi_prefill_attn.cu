@@ -136,6 +136,8 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     volatile int* abort = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();  // q, the cache and the index arrays may come from the kernels just before this one
+    pdl_trigger();
     const int tile = n_tiles - 1 - (int)blockIdx.x;  // the longer tiles of a sequence start first
     const int h = blockIdx.y;
     const int g = h / (Hq / Hkv);
@@ -486,8 +488,10 @@ BI_API int bi_prefill_attn(const void* q, int64_t ldq, int64_t q_rows, const voi
                           64, KB, CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
     dim3 grid((unsigned)n_tiles, (unsigned)Hq);
-    prefill_attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, bi::as_stream(stream)>>>(
-        tmQ, tmK, tmV, q_indptr, q_tile_indptr, kv_indptr, q_pos0, B, Hq, Hkv, (int)q_rows, (int)cache_tokens,
-        n_tiles, (float)((double)scale * 1.4426950408889634), static_cast<__nv_bfloat16*>(out), ldo, err);
+    if (bi::launch_pdl(prefill_attn_tc_kernel, grid, dim3(THREADS), SMEM_BYTES, bi::as_stream(stream), 1u, tmQ, tmK,
+                       tmV, q_indptr, q_tile_indptr, kv_indptr, q_pos0, B, Hq, Hkv, (int)q_rows, (int)cache_tokens,
+                       n_tiles, (float)((double)scale * 1.4426950408889634), static_cast<__nv_bfloat16*>(out), ldo,
+                       err) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }

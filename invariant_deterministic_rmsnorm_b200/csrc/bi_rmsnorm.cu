@@ -19,6 +19,9 @@
 #include "bi_common.cuh"
 #include "bi_sm100.cuh"
 
+using bi::sm100::pdl_trigger;
+using bi::sm100::pdl_wait;
+
 namespace {
 
 constexpr int kMaxThreads = 256;
@@ -96,6 +99,10 @@ rmsnorm_rows_kernel(const TIO* __restrict__ x, const TW* __restrict__ w, TIO* __
 
     uint4 xv[VPT], xn[VPT];
     int64_t row = blockIdx.x;
+    // Every CTA waits for the kernel before it (x and w may come from it) before anything else,
+    // so this grid never completes ahead of that one: a later kernel's wait then covers both.
+    pdl_wait();
+    pdl_trigger();  // the next kernel may start its set-up; it waits for this grid before it reads y
     if (row >= M) return;
     // the weights are the same for every row: when a thread's share is small, keep their raw
     // bits in registers for the CTA's lifetime (widened per use); otherwise re-read them per row
@@ -206,7 +213,9 @@ int launch_rows(const TIO* x, const TW* w, TIO* y, int64_t M, int nvec, int thre
         per_sm = (n > 0 ? n : 1) * sms;
     }
     const int64_t grid = M < per_sm ? M : per_sm;
-    rmsnorm_rows_kernel<TIO, TW, VPT><<<(unsigned)grid, threads, 0, s>>>(x, w, y, M, nvec, ldx, ldy, hf, eps);
+    if (bi::launch_pdl(rmsnorm_rows_kernel<TIO, TW, VPT>, dim3((unsigned)grid), dim3(threads), 0, s, 1u, x, w, y, M,
+                       nvec, ldx, ldy, hf, eps) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 

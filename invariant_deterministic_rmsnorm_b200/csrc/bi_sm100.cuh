@@ -266,3 +266,57 @@ __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
 
 }  // namespace sm100
 }  // namespace bi
+
+namespace bi {
+namespace sm100 {
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with the programmatic-stream-serialization attribute may start while the
+// kernel before it on the stream is still finishing.  It must call pdl_wait() before it touches
+// global memory that the earlier kernel may write or read; what comes before (barrier set-up,
+// TMEM allocation, tensor-map prefetch) overlaps the earlier kernel's tail.  pdl_wait() returns
+// once the earlier grid has completed and its memory operations are visible; without the
+// attribute it returns at once.  pdl_trigger() lets the next kernel on the stream begin its own
+// set-up early; it changes no result, only when the next launch may start.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace sm100
+}  // namespace bi
+
+namespace bi {
+namespace sm100 {
+
+// ---------------------------------------------------------------- cluster signalling
+// Wait on one of this CTA's mbarriers whose phase other CTAs of the cluster complete (remote
+// arrives, st.async bytes): acquire at cluster scope, so that what they wrote before signalling is
+// visible.  Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_test_parity_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const volatile int* abort) {
+    if (mbar_test_parity_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_test_parity_cluster(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (abort != nullptr && *abort) return false;
+            if (globaltimer() - t0 > kWaitLimitNs) return false;
+        }
+    }
+}
+// 8-byte store into the shared memory of a CTA of this cluster (`addr` from mapa); its bytes count
+// as completed transactions on that CTA's mbarrier `bar` (also a mapa address) once they land.
+__device__ __forceinline__ void st_async_v2(uint32_t addr, float a, float b, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+                 :: "r"(addr), "f"(a), "f"(b), "r"(bar) : "memory");
+}
+
+}  // namespace sm100
+}  // namespace bi

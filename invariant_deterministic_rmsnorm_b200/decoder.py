@@ -91,6 +91,25 @@ class Decoder:
         else:
             self.length[np.asarray(slots)] = 0
 
+    def share_prefix(self, src: int, dst: int, n: int) -> None:
+        """A prefix-cache hit: sequence `dst` starts from the first n cached tokens of sequence `src`.
+
+        The K and V rows of positions 0 .. n-1 are copied from src's cache slot into dst's in every
+        layer (bi_kv_append, a row scatter), and dst's length becomes n.  Its next prefill then
+        appends after them.  Because a cached row depends only on the tokens up to its position,
+        dst's logits are bitwise those of prefilling its whole prompt from scratch."""
+        src, dst, n = int(src), int(dst), int(n)
+        if not (0 <= src < self.max_seqs and 0 <= dst < self.max_seqs) or src == dst:
+            raise ValueError("src and dst must be two different slots")
+        if not 0 < n <= self.length[src]:
+            raise ValueError("the shared prefix must be cached in src")
+        rows = _dev_i32(dst * self.cap + np.arange(n), self.device)
+        width = self.s.kv_heads * self.s.head_dim
+        for cache in self.k_cache + self.v_cache:
+            rows_src = cache[src * self.cap:src * self.cap + n].view(n, width)
+            bi.bi_kv_append(rows_src, rows, cache)
+        self.length[dst] = n
+
     # ------------------------------------------------------------------ one step
     def _plan(self, slots, tokens, phase):
         """Check a step and build its host-side index arrays."""
@@ -208,7 +227,8 @@ class DecodeGraph:
     The graph reads the current tokens from a device buffer, appends them at each sequence's
     next position, writes the logits to a static fp32 buffer, and writes the greedy next tokens
     back into the token buffer.  It then advances the device copies of the positions, cache
-    rows and KV lengths (or, with prefill attention, the first query positions) by one.  Consecutive replays thus decode greedily with no host work.
+    rows and KV lengths (or, with prefill attention, the first query positions) by one, with a
+    library launch like every other step of the graph.  Consecutive replays thus decode greedily with no host work.
     The host mirrors the lengths in Decoder.length.
 
     Every launch in the graph is the same launch as in Decoder.forward(..., "decode").  The graph
@@ -223,9 +243,10 @@ class DecodeGraph:
         plan = dec._plan(self.slots, [[0]] * B, "decode")
         self.d = dec._upload(plan)
         # positions, cache rows and KV lengths move together; keep them in one buffer so that one
-        # device add advances them all
-        adv = torch.stack([self.d["pos"], self.d["rows"]] + ([self.d["kv_len"]] if plan["split"] else []))
-        self.adv = adv.contiguous()
+        # library launch (bi_advance) advances them all
+        adv = np.stack([np.asarray(plan[k], np.int32) for k in (["pos", "rows", "kv_len"] if plan["split"]
+                                                                   else ["pos", "rows"])])
+        self.adv = _dev_i32(adv, dec.device)
         self.d["pos"], self.d["rows"] = self.adv[0], self.adv[1]
         if plan["split"]:
             self.d["kv_len"] = self.adv[2]
@@ -243,7 +264,7 @@ class DecodeGraph:
         with torch.cuda.graph(self.graph, stream=stream):
             self.logits = dec._run(B, self.split, n_tiles, self.d)
             bi.bi_argmax(self.logits, out=self.d["tok"])
-            self.adv.add_(1)
+            bi.bi_advance(self.adv, 1)
 
     def set_tokens(self, tokens) -> None:
         """Tokens for the next replay (otherwise the previous replay's greedy tokens are used)."""

@@ -118,6 +118,32 @@ def test_chunked_prefill_gives_the_same_bits(llama, cuts):
     assert np.array_equal(got_dec.view(np.uint32), ref_dec.view(np.uint32))
 
 
+def test_prefix_cache_hit_gives_the_same_bits(llama):
+    """Prefix caching across requests ("Defeating Nondeterminism in LLM Inference", section
+    Attention: cached and new keys share one layout).  Request A's prefill writes the K and V
+    rows of a shared 700-token prefix; request B starts from those rows (a cache hit) and
+    prefills only its own 123-token suffix, inside a batch with another request.  B's logits,
+    and its next decode step, must be bitwise those of B prefilled from scratch."""
+    shape, w = llama
+    prefix = inputs.prompt(9, 700, shape.vocab)
+    a_tail = inputs.prompt(10, 300, shape.vocab)
+    b_tail = inputs.prompt(11, 123, shape.vocab)
+    other = inputs.prompt(12, 200, shape.vocab)
+    dec = Decoder(shape, w, max_seqs=4, max_len=1100)
+    ref = dec.forward([3], [np.concatenate([prefix, b_tail])]).cpu().numpy()
+    ref_dec = dec.forward([3], [[5]], "decode").cpu().numpy()
+    dec.forward([0], [np.concatenate([prefix, a_tail])])  # A fills slot 0's cache
+    dec.share_prefix(0, 1, len(prefix))                   # B's cache hit: slot 1 starts at 700
+    got = dec.forward([1, 2], [b_tail, other]).cpu().numpy()[0]
+    assert dec.length[1] == len(prefix) + len(b_tail)
+    assert np.array_equal(got.view(np.uint32), ref[0].view(np.uint32))
+    got_dec = dec.forward([1], [[5]], "decode").cpu().numpy()
+    assert np.array_equal(got_dec.view(np.uint32), ref_dec.view(np.uint32))
+    # a miss would have shown: A's own continuation differs from B's
+    a_next = dec.forward([0], [[5]], "decode").cpu().numpy()
+    assert not np.array_equal(a_next.view(np.uint32), ref_dec.view(np.uint32))
+
+
 def test_decode_through_prefill_attention_equals_prefill(llama):
     """With decode_attention='prefill', a decode step is bitwise the last row of a longer prefill."""
     shape, w = llama

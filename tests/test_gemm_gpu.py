@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import bf16_to_f64, dev, host, rel_frobenius
+from gpu_util import bf16_to_f64, dev, host, oracle_rows, rel_frobenius
 from invariant_deterministic_rmsnorm_b200 import binding, harness, inputs
 
 pytestmark = pytest.mark.gpu
@@ -94,15 +94,40 @@ def test_bf16_output():
     assert np.all(np.abs(g - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-4 * rms)
 
 
-def test_full_size_sampled_rows():
-    """The bench's launch configuration: M = 4096 through the three Llama-shaped weights."""
+@pytest.mark.parametrize("K,N", LLAMA_SHAPES + WIDE_SHAPES)
+def test_full_size_every_row_on_a_column_slice(K, N):
+    """The bench's launch configuration, M = 4096, on both plans (CTA pairs for the three
+    Llama-shaped projections, single CTAs for the two wide ones).  Every one of the 4096 rows
+    is compared with the oracle on 256 columns that straddle a tile boundary, so a slip in any
+    row tile, in either CTA of a pair, or across a column-tile edge shows.  The bf16 output the
+    bench uses must be the nearest-even rounding of the fp32 accumulator at every element."""
     M = 4096
-    for K, N in LLAMA_SHAPES:
-        A, W = inputs.gemm_case(M, N, K)
-        C = _gemm(A, W, torch.bfloat16)
-        rows = [0, 1, 2047, 4095]
-        ref = oracle.gemm(A[rows], W)
-        assert rel_frobenius(bf16_to_f64(C[rows]), ref) <= 2e-3
+    A, W = inputs.gemm_case(M, N, K)
+    C32 = _gemm(A, W, torch.float32)
+    c0 = N - 384
+    ref = oracle_rows(oracle.gemm, A, np.ascontiguousarray(W[:, c0:c0 + 256]))
+    g = C32[:, c0:c0 + 256].astype(np.float64)
+    rms = np.sqrt((ref ** 2).mean(axis=1, keepdims=True))
+    row_err = np.linalg.norm(g - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert row_err.max() <= 2e-3 and row_err.max() <= 1e-4, (int(row_err.argmax()), float(row_err.max()))
+    assert np.all(np.abs(g - ref) <= 1e-3 * rms)
+    Cb = _gemm(A, W, torch.bfloat16)
+    assert np.array_equal(Cb, inputs.f32_to_bf16_bits(C32))
+
+
+@pytest.mark.parametrize("K,N", WIDE_SHAPES)
+@pytest.mark.parametrize("M", [1, 129, 300])
+def test_small_int_exact_wide_plan(K, N, M):
+    """Small-integer operands through the single-CTA plan of the wide weights: every partial sum
+    is an exact integer in fp32, so every element must equal the oracle bit for bit.  K = 264
+    ends in a ragged K block; M = 129 and 300 end in ragged row tiles; 32000 = 125 x 256 exactly,
+    28672 = 112 x 256."""
+    Ks = 264
+    A = inputs.small_int_bf16(55, (M, Ks))
+    W = inputs.small_int_bf16(56, (Ks, N))
+    C = _gemm(A, W)
+    ref = oracle_rows(oracle.gemm, A, W, block=16)
+    assert np.array_equal(C.astype(np.float64), ref), int((C != ref).sum())
 
 
 def test_empty_and_bad_args():

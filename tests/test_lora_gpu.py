@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import bf16_to_f64, dev, host, rel_frobenius
+from gpu_util import bf16_to_f64, dev, host, oracle_rows, rel_frobenius
 from invariant_deterministic_rmsnorm_b200 import binding, harness, inputs
 
 pytestmark = pytest.mark.gpu
@@ -47,6 +47,19 @@ def test_shrink_parity(r, M):
     err = rel_frobenius(t, ref)
     assert err <= 2e-3, err
     assert err <= 1e-4, err
+
+
+@pytest.mark.parametrize("r", [8, 16, 64])
+def test_shrink_parity_full_size(r):
+    """The bench's launch configuration, M = 4096 (32 tiles of 128 rows, every one a full
+    cluster of 8 K slices): every row against the oracle's split-8 sum."""
+    M = 4096
+    x, A, _, _ = inputs.lora_case(M, r)
+    t = _shrink(x, A)
+    ref = oracle_rows(oracle.lora_shrink_split, x, A, 8)
+    row_err = np.linalg.norm(t - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert rel_frobenius(t, ref) <= 2e-3
+    assert row_err.max() <= 1e-4, (int(row_err.argmax()), float(row_err.max()))
 
 
 def test_shrink_other_k_and_splits():
