@@ -919,17 +919,15 @@ def run_sweep(args):
             Ws = [rows_dev(50 + j, K, N).mul_(0.02) for j in range(R)]
             As = [rows_dev(60 + j, M, K) for j in range(R)]
             Cs = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(R)]
-            ws = torch.zeros(max(lib.bi_ctrl_gemm_split_workspace_size(M, N, K, S) for S in range(1, 5)) + 16,
-                             dtype=torch.uint8, device=device)
             fl = 2 * M * N * K / 1e12
             row = {"M": M, "plan": B.gemm_splits(N, K)}
             for S in range(1, 5):
-                t = _time_graph([lambda j=j, S=S: B.bi_ctrl_gemm_split(As[j], Ws[j], S, C=Cs[j], workspace=ws,
+                t = _time_graph([lambda j=j, S=S: B.bi_ctrl_gemm_split(As[j], Ws[j], S, C=Cs[j],
                                                                        stream=stream) for j in range(R)], stream)
                 row[f"s{S}_us"] = round(t * 1e3, 2)
                 row[f"s{S}_tflops"] = round(fl / (t / 1e3), 1)
             table.append(row)
-            del Ws, As, Cs, ws
+            del Ws, As, Cs
         emit({"op": "gemm-split", "K": K, "N": N, "rows": table})
     # RMSNorm
     table = []

@@ -137,72 +137,15 @@ def bi_rmsnorm(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, 
     return y
 
 
-class _SplitWorkspace:
-    """The zero-filled split-K workspace that bi_gemm calls share on one device, one call at a
-    time (the library's counters return to zero after every call).  It is sized for the
-    largest counter region plus the largest partial region seen, so that no call's partials
-    reach another call's counters.  It grows only outside CUDA graph capture; a replaced buffer
-    is kept alive, because a graph captured earlier may still point at it."""
-
-    def __init__(self) -> None:
-        self.buf: torch.Tensor | None = None
-        self.counters = 0
-        self.partials = 0
-        self.retired: list[torch.Tensor] = []
-
-    def get(self, device: torch.device, counters: int, partials: int) -> torch.Tensor:
-        if self.buf is not None and counters <= self.counters and partials <= self.partials:
-            return self.buf
-        if torch.cuda.is_current_stream_capturing():
-            raise BIError("the GEMM split workspace must grow, which cannot happen during graph capture: "
-                          "call reserve_gemm_workspace before capturing")
-        self.counters, self.partials = max(counters, self.counters), max(partials, self.partials)
-        if self.buf is not None:
-            self.retired.append(self.buf)
-        self.buf = torch.zeros(self.counters + self.partials, dtype=torch.uint8, device=device)
-        torch.cuda.synchronize(device)  # zeroed before any stream uses it
-        return self.buf
-
-    def reset(self) -> None:
-        """Zero the buffer again, after a call that set a device error bit."""
-        if self.buf is not None:
-            self.buf.zero_()
-            torch.cuda.synchronize(self.buf.device)
-
-
-_split_ws: dict[int, _SplitWorkspace] = {}
-
-
-def _split_workspace(device: torch.device) -> _SplitWorkspace:
-    idx = device.index if device.index is not None else torch.cuda.current_device()
-    return _split_ws.setdefault(idx, _SplitWorkspace())
-
-
 def gemm_splits(N: int, K: int) -> int:
     """The K split count of bi_gemm's plan for a [K, N] weight on the current device."""
     return int(library().bi_gemm_splits(N, K))
 
 
-def reserve_gemm_workspace(M: int, N: int, K: int, device=None) -> None:
-    """Grow the shared split workspace for a [M, K] x [K, N] GEMM ahead of graph capture."""
-    lib = library()
-    need = lib.bi_gemm_workspace_size(M, N, K)
-    if need:
-        cb = lib.bi_gemm_counter_bytes(M, N, K)
-        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-        _split_workspace(dev).get(dev, cb, need - cb)
-
-
-def reset_gemm_workspace() -> None:
-    for w in _split_ws.values():
-        w.reset()
-
-
 def bi_gemm(A: torch.Tensor, W: torch.Tensor, C: torch.Tensor | None = None, out_dtype=torch.float32,
-            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+            stream=None) -> torch.Tensor:
     """C = A @ W with A [M, K] bf16, W [K, N] bf16 (both row-major contiguous); C fp32 or bf16 [M, N].
-    A split plan needs a workspace: the shared zero-filled one unless `workspace` is given (which
-    then follows bi_gemm's rules: counters zero between calls)."""
+    The library needs no workspace for any plan (bi_gemm_workspace_size is 0)."""
     for t, n in ((A, "A"), (W, "W")):
         if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 2 or not t.is_cuda:
             raise ValueError(f"{n} must be a contiguous 2-D bf16 CUDA tensor")
@@ -214,15 +157,8 @@ def bi_gemm(A: torch.Tensor, W: torch.Tensor, C: torch.Tensor | None = None, out
         C = torch.empty((M, N), dtype=out_dtype, device=A.device)
     if tuple(C.shape) != (M, N) or not C.is_contiguous():
         raise ValueError("C must be a contiguous [M, N] tensor")
-    lib = library()
-    need = lib.bi_gemm_workspace_size(M, N, K)
-    ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
-    if need:
-        if workspace is None:
-            cb = lib.bi_gemm_counter_bytes(M, N, K)
-            workspace = _split_workspace(A.device).get(A.device, cb, need - cb)
-        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
-    st = lib.bi_gemm(_ptr(A), _ptr(W), _ptr(C), M, N, K, _dtype_code(C), ws_ptr, ws_bytes, _stream(stream))
+    st = library().bi_gemm(_ptr(A), _ptr(W), _ptr(C), M, N, K, _dtype_code(C), ctypes.c_void_p(0), 0,
+                           _stream(stream))
     _check("bi_gemm", st)
     return C
 
@@ -508,22 +444,17 @@ def bi_ctrl_gemm_splitk(A: torch.Tensor, W: torch.Tensor, C: torch.Tensor | None
 
 
 def bi_ctrl_gemm_split(A: torch.Tensor, W: torch.Tensor, splits: int, C: torch.Tensor | None = None,
-                       out_dtype=torch.float32, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """bi_gemm with the K split count given (the plan study).  `workspace`, when given, must be
-    zero-filled and at least bi_ctrl_gemm_split_workspace_size bytes; by default a fresh zeroed
-    one is allocated."""
+                       out_dtype=torch.float32, stream=None) -> torch.Tensor:
+    """bi_gemm with the K split count given (the plan study): S > 1 runs the cluster-split kernel,
+    whose partials meet on chip."""
     _bf16_2d(A, "A")
     _bf16_2d(W, "W")
     M, K = A.shape
     N = W.shape[1]
     if C is None:
         C = torch.empty((M, N), dtype=out_dtype, device=A.device)
-    lib = library()
-    need = lib.bi_ctrl_gemm_split_workspace_size(M, N, K, splits)
-    if workspace is None:
-        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=A.device)
-    st = lib.bi_ctrl_gemm_split(_ptr(A), _ptr(W), _ptr(C), M, N, K, _dtype_code(C), int(splits), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _stream(stream))
+    st = library().bi_ctrl_gemm_split(_ptr(A), _ptr(W), _ptr(C), M, N, K, _dtype_code(C), int(splits),
+                                      ctypes.c_void_p(0), 0, _stream(stream))
     _check("bi_ctrl_gemm_split", st)
     return C
 

@@ -31,7 +31,9 @@ bool pdl_enabled();
 
 // Launch `kernel` on `s`.  With programmatic dependent launch on, it may begin while the kernel
 // before it on the stream finishes; every kernel launched this way calls pdl_wait() (bi_sm100.cuh)
-// before it reads or writes global memory.  cluster: CTAs per cluster along y (1 = no cluster).
+// before it reads or writes global memory.  cluster_y: CTAs per cluster along y; 0 = launched
+// without a cluster shape.  A kernel that uses cluster-scope instructions (mapa, st.async,
+// barrier.cluster) is always given one, even a cluster of a single CTA.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                               unsigned cluster_y, Args&&... args) {
@@ -47,7 +49,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
         attr[n].val.programmaticStreamSerializationAllowed = 1;
         ++n;
     }
-    if (cluster_y > 1) {
+    if (cluster_y >= 1) {
         attr[n].id = cudaLaunchAttributeClusterDimension;
         attr[n].val.clusterDim.x = 1;
         attr[n].val.clusterDim.y = cluster_y;

@@ -456,7 +456,7 @@ decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restri
 // Phase 2 on `s`, allowed to start while phase 1 finishes (it waits for phase 1 before it reads).
 template <typename K, typename... Args>
 void launch_merge(K kernel, dim3 grid, cudaStream_t s, Args... args) {
-    (void)bi::launch_pdl(kernel, grid, dim3(128), 0, s, 1u, args...);
+    (void)bi::launch_pdl(kernel, grid, dim3(128), 0, s, 0u, args...);
 }
 
 template <typename F>
@@ -517,7 +517,7 @@ int launch_chunks(const void* q, const void* k, const void* v, const int32_t* kv
     if (sms <= 0) return BI_ERR_CUDA;
     const int64_t ctas = 2LL * sms;  // two persistent CTAs per SM: one computes while the other waits
     dim3 grid((unsigned)(items < ctas ? items : ctas));
-    if (bi::launch_pdl(kern, grid, dim3(THREADS), L::BYTES, s, 1u, tmK, tmV, static_cast<const __nv_bfloat16*>(q),
+    if (bi::launch_pdl(kern, grid, dim3(THREADS), L::BYTES, s, 0u, tmK, tmV, static_cast<const __nv_bfloat16*>(q),
                        kv_indptr, kv_len, B, T, Hq, Hkv, (int)items, scale, o_part, ml_part, err) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();

@@ -76,35 +76,6 @@ __device__ __forceinline__ void fail(uint32_t* err, volatile int* abort, uint32_
     *abort = 1;
 }
 
-// Split-K meeting point.  Every lane of a writer warp fences its partial-row stores, and after
-// the warp has met, one lane increments the counter.  The last slice waits until the counter
-// holds `target`, then zeroes it for the next call.  Bounded: false after kWaitLimitNs.
-__device__ __forceinline__ void split_signal(uint32_t* cnt, int lane) {
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) atomicAdd(cnt, 1u);
-}
-
-__device__ __forceinline__ bool split_wait(uint32_t* cnt, uint32_t target) {
-    const uint64_t t0 = globaltimer();
-    while (true) {
-        uint32_t v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-        if (v == target) {
-            asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(cnt), "r"(0u) : "memory");
-            return true;
-        }
-        if (globaltimer() - t0 > kWaitLimitNs) return false;
-        __nanosleep(128);
-    }
-}
-
-__device__ __forceinline__ float4 ld_partial(const float* p) {
-    float4 r;
-    asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
-    return r;
-}
-
 // Tile order: groups of `gm` row tiles, walked column by column inside a group, so that the
 // tiles in flight at any moment share a few W column blocks and a few A row blocks in L2.
 // The order decides only which CTA computes a tile, never how.
@@ -331,17 +302,11 @@ struct Bars {
     int abort;
 };
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * ST_BYTES + sizeof(Bars) + 64;
-constexpr int MAX_SPLIT = 4;                 // K slices per tile at most
-constexpr int CNT_PER_TILE = 2 * EPI_WARPS;  // one split counter per (CTA, epilogue warp)
 }  // namespace pair
 
-// SPLIT = false is the unsplit kernel (splits must be 1; cnt and part are unused).
-template <bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
-                         void* __restrict__ C, int M, int N, int K, int c_bf16, int gm, int splits_arg,
-                         uint32_t* __restrict__ cnt, float* __restrict__ part, uint32_t* err) {
-    const int splits = SPLIT ? splits_arg : 1;
+                         void* __restrict__ C, int M, int N, int K, int c_bf16, int gm, uint32_t* err) {
     using pair::ROWS;
     using pair::COLS;
     using pair::TILE_M;
@@ -367,9 +332,6 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     const int tiles_n = (N + TILE_N - 1) / TILE_N;
     const int num_tiles = tiles_m * tiles_n;
     const int num_kb = (K + BK - 1) / BK;
-    // work unit u = (tile u / splits, K slice u % splits); the slices of a tile are adjacent,
-    // so they run side by side on neighbouring pairs
-    const int num_units = num_tiles * splits;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -399,20 +361,18 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     tc_fence_after();
     const uint32_t tmem_base = bars->tmem_addr;
     // everything above overlaps the previous kernel's tail; A and W may come from it, and it may
-    // still read C or the split workspace
+    // still read C
     pdl_wait();
     pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
             uint32_t it = 0;  // k-blocks issued by this CTA so far (the ring runs across tiles)
-            for (int u = pair_id; u < num_units && !*abort; u += n_pairs) {
-                const int t = u / splits, sl = u - t * splits;
+            for (int t = pair_id; t < num_tiles && !*abort; t += n_pairs) {
                 int mt, nt;
                 tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
                 const int m0 = mt * TILE_M + (int)rank * ROWS, n0 = nt * TILE_N + (int)rank * COLS;
-                const int kb1 = (int)((int64_t)(sl + 1) * num_kb / splits);
-                for (int kb = (int)((int64_t)sl * num_kb / splits); kb < kb1; ++kb, ++it) {
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = (int)(it % STAGES);
                     const uint32_t round = it / STAGES;
                     if (!mbar_wait(smem_u32(&bars->empty[s]), (round & 1u) ^ 1u, abort)) {
@@ -446,9 +406,7 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             const uint32_t peer_empty0 = mapa(smem_u32(&bars->empty[0]), 1);
             const uint32_t peer_tfull0 = mapa(smem_u32(&bars->tfull[0]), 1);
             uint32_t it = 0, local = 0;
-            for (int u = pair_id; u < num_units && !*abort; u += n_pairs, ++local) {
-                const int t = u / splits, sl = u - t * splits;
-                const int kb0 = (int)((int64_t)sl * num_kb / splits), kb1 = (int)((int64_t)(sl + 1) * num_kb / splits);
+            for (int t = pair_id; t < num_tiles && !*abort; t += n_pairs, ++local) {
                 const uint32_t acc = local & 1u, use = local >> 1;
                 if (!mbar_wait(smem_u32(&bars->tempty[acc]), (use & 1u) ^ 1u, abort)) {
                     fail(err, abort, bi::DEVERR_WAIT_ACCUM);
@@ -456,7 +414,7 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = (int)(it % STAGES);
                     const uint32_t round = it / STAGES;
                     if (!mbar_wait(smem_u32(&bars->full[s]), round & 1u, abort)) {
@@ -470,7 +428,7 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint64_t adesc = make_smem_desc(a_base + k * UMMA_K * 2, 16, 1024, 2);
                         const uint64_t bdesc = make_smem_desc(b_base + k * UMMA_K * 128, B_BOX, 1024, 2);
-                        mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+                        mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
                     }
                     // stage s of both CTAs is free once these MMAs have read it
                     mma_commit_pair(smem_u32(&bars->empty[s]));
@@ -485,10 +443,8 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     } else {
         const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter .. +31
         const uint32_t tempty0 = rank == 0 ? smem_u32(&bars->tempty[0]) : mapa(smem_u32(&bars->tempty[0]), 0);
-        const int64_t slice_elems = (int64_t)M * N;  // one slice's fp32 partial, [M, N] row-major
         uint32_t local = 0;
-        for (int u = pair_id; u < num_units; u += n_pairs, ++local) {
-            const int t = u / splits, sl = u - t * splits;
+        for (int t = pair_id; t < num_tiles; t += n_pairs, ++local) {
             const uint32_t acc = local & 1u, use = local >> 1;
             const bool ok = mbar_wait(smem_u32(&bars->tfull[acc]), use & 1u, abort);
             if (!ok) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
@@ -497,41 +453,11 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             tc_fence_after();
             int mt, nt;
             tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
-            const int row0 = mt * TILE_M + (int)rank * ROWS + quarter * 32;
-            const int row = row0 + lane;
-            // Split K: the S slices' copies of this warp's 32 rows meet through one counter.  A
-            // warp whose rows all lie past M neither stores nor waits, in every slice alike.
-            const bool split = SPLIT && splits > 1 && row0 < M;
-            const bool last = sl == splits - 1;
-            uint32_t* my_cnt = cnt + (int64_t)t * pair::CNT_PER_TILE + (int)rank * EPI_WARPS + quarter;
-            if (split && last) {
-                bool ready = true;
-                if (lane == 0) ready = split_wait(my_cnt, (uint32_t)(splits - 1));
-                ready = __shfl_sync(0xffffffffu, ready, 0);
-                __threadfence();  // every lane's partial loads below come after lane 0's acquire
-                if (!ready) {
-                    if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_SPLIT);
-                    break;
-                }
-            }
+            const int row = mt * TILE_M + (int)rank * ROWS + quarter * 32 + lane;
             const uint32_t lane_addr = tmem_base + acc * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
             for (int c = 0; c < TILE_N; c += 32) {
                 const int col = nt * TILE_N + c;
-                const bool live = row < M && col < N;
-                const int nv = live ? min(32, N - col) : 0;  // a multiple of 8 (N % 8 == 0)
-                // the last slice issues its loads of the earlier partials before reading TMEM
-                float4 pv[(pair::MAX_SPLIT - 1) * 8];
-                if (split && last) {
-#pragma unroll
-                    for (int j = 0; j < pair::MAX_SPLIT - 1; ++j) {
-                        const float* src = part + j * slice_elems + (int64_t)row * N + col;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            pv[j * 8 + i] = (j < splits - 1 && 4 * i < nv) ? ld_partial(src + 4 * i)
-                                                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                }
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(lane_addr + (uint32_t)c, r);
                 tmem_wait_ld();
@@ -540,37 +466,7 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8u);
                 }
-                if (!live) continue;
-                if (split && !last) {  // an earlier slice: store the fp32 partial as it stands
-                    float* dst = part + sl * slice_elems + (int64_t)row * N + col;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        if (4 * i < nv)
-                            *reinterpret_cast<uint4*>(dst + 4 * i) =
-                                make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-                    continue;
-                }
-                if (split) {  // the last slice: ((P0 + P1) + ...) + this slice's accumulator
-#pragma unroll
-                    for (int j = 1; j < pair::MAX_SPLIT - 1; ++j) {
-                        if (j < splits - 1) {
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                pv[i].x = __fadd_rn(pv[i].x, pv[j * 8 + i].x);
-                                pv[i].y = __fadd_rn(pv[i].y, pv[j * 8 + i].y);
-                                pv[i].z = __fadd_rn(pv[i].z, pv[j * 8 + i].z);
-                                pv[i].w = __fadd_rn(pv[i].w, pv[j * 8 + i].w);
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        r[4 * i] = __float_as_uint(__fadd_rn(pv[i].x, __uint_as_float(r[4 * i])));
-                        r[4 * i + 1] = __float_as_uint(__fadd_rn(pv[i].y, __uint_as_float(r[4 * i + 1])));
-                        r[4 * i + 2] = __float_as_uint(__fadd_rn(pv[i].z, __uint_as_float(r[4 * i + 2])));
-                        r[4 * i + 3] = __float_as_uint(__fadd_rn(pv[i].w, __uint_as_float(r[4 * i + 3])));
-                    }
-                }
+                if (row >= M || col >= N) continue;
                 if (!c_bf16) {
                     float* dst = static_cast<float*>(C) + (int64_t)row * N + col;
                     if (col + 32 <= N) {
@@ -599,11 +495,308 @@ bi_gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                     }
                 }
             }
-            if (split && !last) split_signal(my_cnt, lane);  // this warp's partial rows are stored
         }
     }
 
     // no CTA of the pair leaves (or frees TMEM) while the other may still signal it
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ the cluster-split kernel
+// K cut into S contiguous slices whose partials meet on chip.  A cluster of 2S CTAs is S CTA
+// pairs; pair p (ranks 2p, 2p + 1) computes slice p of the cluster's current 256 x 256 tile
+// exactly as the pair kernel computes a whole tile: cta_group::2 MMAs, its K blocks in ascending
+// order, into one of two TMEM accumulators.  The epilogue then combines the S accumulators
+// through distributed shared memory.  The tile's 256 columns are cut into 16 chunks of 16;
+// chunk c belongs to slice c % S.  For each chunk, the CTA of the owning slice that holds the
+// same 128 rows adds ((P0 + P1) + ...) + P(S-1), element by element in fp32, rounds once and
+// stores C; each other CTA pushes its piece of the chunk (st.async) into a two-slot receive
+// ring of the owner, whose remote arrive hands the slot back once it has been read.  The
+// partials never touch HBM, and no floating-point atomic is used.  A cluster walks tiles
+// c, c + clusters, ...; the accumulator double buffer lets the exchange of one tile overlap the
+// MMAs of the next.
+namespace cs {
+constexpr int STAGES = 5;
+constexpr int CW = 16;                          // columns per exchanged chunk
+constexpr int NCH = pair::TILE_N / CW;          // chunks per tile
+constexpr int RING = 2;                         // receive slots per epilogue warp
+constexpr int MAX_S = 4;
+constexpr int PIECE = 32 * CW * 4;              // one sender's piece for one warp: 32 rows x 16 fp32
+constexpr int SLOT = (MAX_S - 1) * PIECE;       // every other slice's piece
+constexpr int RECV_BYTES = EPI_WARPS * RING * SLOT;
+struct Bars {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint64_t rfull[EPI_WARPS][RING];         // owner: every other slice's piece of this slot has landed
+    uint64_t rfree[EPI_WARPS][RING][MAX_S];  // sender: slot r of warp w in slice o's CTA may be refilled
+    uint32_t tmem_addr;
+    int abort;
+};
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * pair::ST_BYTES + RECV_BYTES + sizeof(Bars) + 64;
+static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
+}  // namespace cs
+
+__global__ void __launch_bounds__(THREADS, 1)
+bi_gemm_bf16_cluster_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                            void* __restrict__ C, int M, int N, int K, int c_bf16, int gm, int S, uint32_t* err) {
+    using pair::ROWS;
+    using pair::COLS;
+    using pair::TILE_M;
+    using pair::TILE_N;
+    using pair::A_ST;
+    using pair::B_ST;
+    using pair::ST_BYTES;
+    using pair::ACC_COLS;
+    using pair::TMEM_COLS;
+    constexpr int STAGES = cs::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * A_ST;
+    uint8_t* recv = sB + STAGES * B_ST;
+    cs::Bars* bars = reinterpret_cast<cs::Bars*>(recv + cs::RECV_BYTES);
+    volatile int* abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int slice = (int)(rank >> 1);
+    const uint32_t rp = rank & 1u;            // 0: the pair's leader, which issues the MMAs
+    const uint32_t leader = rank & ~1u;
+    const int csize = 2 * S;
+    const int cluster_id = (int)blockIdx.x / csize, n_clusters = (int)gridDim.x / csize;
+    const int tiles_m = (M + TILE_M - 1) / TILE_M;
+    const int tiles_n = (N + TILE_N - 1) / TILE_N;
+    const int num_tiles = tiles_m * tiles_n;
+    const int num_kb = (K + BK - 1) / BK;
+    const int kb0 = (int)((int64_t)slice * num_kb / S), kb1 = (int)((int64_t)(slice + 1) * num_kb / S);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&bars->full[s]), 1);
+            mbar_init(smem_u32(&bars->empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&bars->tfull[b]), 1);
+            mbar_init(smem_u32(&bars->tempty[b]), 2 * EPI_WARPS);
+        }
+        mbar_init(smem_u32(&bars->drain), 1);
+        for (int w = 0; w < EPI_WARPS; ++w)
+            for (int r = 0; r < cs::RING; ++r) {
+                mbar_init(smem_u32(&bars->rfull[w][r]), 1);
+                for (int o = 0; o < cs::MAX_S; ++o) mbar_init(smem_u32(&bars->rfree[w][r][o]), 1);
+            }
+        bars->abort = 0;
+        fence_barrier_init();
+        fence_proxy_async_shared();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmW);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(&bars->tmem_addr), TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    // every CTA's barriers are initialised and its TMEM allocated before any signal crosses the cluster
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = bars->tmem_addr;
+    pdl_wait();  // A and W may come from the kernel before this one, and it may still read C
+    pdl_trigger();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;  // k-blocks issued by this CTA so far (the ring runs across tiles)
+            for (int t = cluster_id; t < num_tiles && !*abort; t += n_clusters) {
+                int mt, nt;
+                tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
+                const int m0 = mt * TILE_M + (int)rp * ROWS, n0 = nt * TILE_N + (int)rp * COLS;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = (int)(it % STAGES);
+                    const uint32_t round = it / STAGES;
+                    if (!mbar_wait(smem_u32(&bars->empty[s]), (round & 1u) ^ 1u, abort)) {
+                        fail(err, abort, bi::DEVERR_WAIT_TMA);
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&bars->full[s]);
+                    if (rp == 0) mbar_arrive_expect_tx(fb, 2 * ST_BYTES);  // this stage of both CTAs
+                    const uint32_t fb_leader = mapa(fb, leader);
+                    tma_load_2d_pair(smem_u32(sA + s * A_ST), &tmA, kb * BK, m0, fb_leader);
+                    tma_load_2d_pair(smem_u32(sB + s * B_ST), &tmW, n0, kb * BK, fb_leader);
+                    tma_load_2d_pair(smem_u32(sB + s * B_ST + B_BOX), &tmW, n0 + 64, kb * BK, fb_leader);
+                }
+            }
+            if (*abort) {  // let loads in flight land before the shared memory is released
+                if (rp == 0) {
+                    for (uint32_t i = it > (uint32_t)STAGES ? it - STAGES : 0u; i < it; ++i)
+                        (void)mbar_wait(smem_u32(&bars->full[i % STAGES]), (i / STAGES) & 1u, nullptr);
+                } else {
+                    const uint64_t t0 = globaltimer();
+                    while (globaltimer() - t0 < 200000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rp == 0) {
+            constexpr uint32_t idesc = make_idesc_bf16_f32(TILE_M, TILE_N, 0, 1);
+            const uint32_t peer_empty0 = mapa(smem_u32(&bars->empty[0]), rank | 1u);
+            const uint32_t peer_tfull0 = mapa(smem_u32(&bars->tfull[0]), rank | 1u);
+            uint32_t it = 0, local = 0;
+            for (int t = cluster_id; t < num_tiles && !*abort; t += n_clusters, ++local) {
+                const uint32_t acc = local & 1u, use = local >> 1;
+                if (!mbar_wait(smem_u32(&bars->tempty[acc]), (use & 1u) ^ 1u, abort)) {
+                    fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    const int s = (int)(it % STAGES);
+                    const uint32_t round = it / STAGES;
+                    if (!mbar_wait(smem_u32(&bars->full[s]), round & 1u, abort)) {
+                        fail(err, abort, bi::DEVERR_WAIT_FULL);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA + s * A_ST);
+                    const uint32_t b_base = smem_u32(sB + s * B_ST);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        const uint64_t adesc = make_smem_desc(a_base + k * UMMA_K * 2, 16, 1024, 2);
+                        const uint64_t bdesc = make_smem_desc(b_base + k * UMMA_K * 128, B_BOX, 1024, 2);
+                        mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+                    }
+                    mma_commit_pair(smem_u32(&bars->empty[s]));
+                    mma_commit_pair(peer_empty0 + (uint32_t)s * 8u);
+                }
+                mma_commit_pair(smem_u32(&bars->tfull[acc]));
+                mma_commit_pair(peer_tfull0 + acc * 8u);
+            }
+            mma_commit_pair(smem_u32(&bars->drain));  // TMEM is released only after every MMA completed
+            (void)mbar_wait(smem_u32(&bars->drain), 0u, nullptr);
+        }
+    } else {
+        const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter .. +31
+        const uint32_t tempty0 = rp == 0 ? smem_u32(&bars->tempty[0]) : mapa(smem_u32(&bars->tempty[0]), leader);
+        const uint32_t ring = smem_u32(recv) + (uint32_t)(quarter * cs::RING * cs::SLOT);  // this warp's slots
+        const uint32_t rfull0 = smem_u32(&bars->rfull[quarter][0]);
+        bool alive = true;
+        uint32_t local = 0;
+        for (int t = cluster_id; t < num_tiles && alive; t += n_clusters, ++local) {
+            const uint32_t acc = local & 1u, use = local >> 1;
+            const bool ok = mbar_wait(smem_u32(&bars->tfull[acc]), use & 1u, abort);
+            if (!ok) fail(err, abort, bi::DEVERR_WAIT_ACCUM);
+            // tcgen05.ld is warp-collective: the whole warp takes the same branch
+            if (!__all_sync(0xffffffffu, ok && !*abort)) break;
+            tc_fence_after();
+            int mt, nt;
+            tile_coords(t, tiles_m, tiles_n, gm, mt, nt);
+            const int row = mt * TILE_M + (int)rp * ROWS + quarter * 32 + lane;
+            const uint32_t lane_addr = tmem_base + acc * ACC_COLS + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < cs::NCH; ++c) {
+                uint32_t r[16];
+                tmem_ld16(lane_addr + (uint32_t)(c * cs::CW), r);
+                tmem_wait_ld();
+                if (c == cs::NCH - 1) {  // every column of this accumulator is in registers: hand it back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8u);
+                }
+                const int o = c % S;                                 // the slice that owns chunk c
+                const int nown_o = (cs::NCH - o + S - 1) / S;
+                const uint32_t n = local * (uint32_t)nown_o + (uint32_t)(c / S);  // o's running chunk count
+                const int slot = (int)(n % cs::RING);
+                const uint32_t par = (n / cs::RING) & 1u;
+                if (o != slice) {
+                    // push this piece into o's slot once o has read what was there before
+                    const bool free_ok = __all_sync(
+                        0xffffffffu, mbar_wait_cluster(smem_u32(&bars->rfree[quarter][slot][o]), par ^ 1u, abort));
+                    if (!free_ok) {
+                        if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_CLUSTER);
+                        alive = false;
+                        break;
+                    }
+                    const uint32_t owner = (uint32_t)(2 * o) + rp;
+                    const int idx = slice < o ? slice : slice - 1;
+                    const uint32_t dst =
+                        mapa(ring + (uint32_t)(slot * cs::SLOT + idx * cs::PIECE + lane * cs::CW * 4), owner);
+                    const uint32_t bar = mapa(rfull0 + (uint32_t)slot * 8u, owner);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        st_async_v4(dst + 16u * i, r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3], bar);
+                    continue;
+                }
+                // this slice owns chunk c: wait for the other slices' pieces, add in slice order
+                if (lane == 0) mbar_arrive_expect_tx(rfull0 + (uint32_t)slot * 8u, (uint32_t)((S - 1) * cs::PIECE));
+                const bool full_ok = __all_sync(0xffffffffu, mbar_wait_cluster(rfull0 + (uint32_t)slot * 8u, par, abort));
+                if (!full_ok) {
+                    if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_CLUSTER);
+                    alive = false;
+                    break;
+                }
+                float v[16];
+                for (int q = 0; q < S; ++q) {
+                    float p[16];
+                    if (q == slice) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) p[i] = __uint_as_float(r[i]);
+                    } else {
+                        const int idx = q < slice ? q : q - 1;
+                        const uint32_t src = ring + (uint32_t)(slot * cs::SLOT + idx * cs::PIECE + lane * cs::CW * 4);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                                         : "=f"(p[4 * i]), "=f"(p[4 * i + 1]), "=f"(p[4 * i + 2]), "=f"(p[4 * i + 3])
+                                         : "r"(src + 16u * i));
+                    }
+                    if (q == 0) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = p[i];
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(v[i], p[i]);
+                    }
+                }
+                __syncwarp();
+                // the slot has been read: every sender may refill it
+                if (lane < S && lane != slice)
+                    mbar_arrive_cluster(mapa(smem_u32(&bars->rfree[quarter][slot][slice]), (uint32_t)(2 * lane) + rp));
+                const int col = nt * TILE_N + c * cs::CW;
+                if (row >= M || col >= N) continue;
+                if (!c_bf16) {
+                    float* dst = static_cast<float*>(C) + (int64_t)row * N + col;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (col + 4 * i + 4 <= N)
+                            *reinterpret_cast<float4*>(dst + 4 * i) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2],
+                                                                                  v[4 * i + 3]);
+                } else {
+                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(C) + (int64_t)row * N + col;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        if (col + 8 * h + 8 <= N)
+                            *reinterpret_cast<uint4*>(dst + 8 * h) = make_uint4(
+                                bi::pack_bf16x2(v[8 * h], v[8 * h + 1]), bi::pack_bf16x2(v[8 * h + 2], v[8 * h + 3]),
+                                bi::pack_bf16x2(v[8 * h + 4], v[8 * h + 5]), bi::pack_bf16x2(v[8 * h + 6], v[8 * h + 7]));
+                }
+            }
+        }
+    }
+
+    // no CTA leaves (or frees TMEM) while a peer may still store into it or signal it
     tc_fence_before();
     __syncthreads();
     cluster_sync();
@@ -658,86 +851,33 @@ int launch_gemm_bn(const void* A, int64_t lda, const void* W, int64_t ldw, void*
     if (sms <= 0) return BI_ERR_CUDA;
     const int gm = 16;  // ~16 row tiles x ~9 column tiles in flight: A and W blocks balanced within L2
     dim3 grid((unsigned)(tiles < sms ? tiles : sms));
-    if (bi::launch_pdl(bi_gemm_bf16_tc_kernel<BN>, grid, dim3(THREADS), Tile<BN>::SMEM_BYTES, stream, 1u, tmA, tmW, C,
+    if (bi::launch_pdl(bi_gemm_bf16_tc_kernel<BN>, grid, dim3(THREADS), Tile<BN>::SMEM_BYTES, stream, 0u, tmA, tmW, C,
                        (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, err) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
-// Shared-memory attribute of both pair-kernel instantiations (once per device).
+// Shared-memory attribute of the pair kernel (once per device).
 bool pair_smem_attr() {
     static std::once_flag once[64];
     static bool ok[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::call_once(once[dev], [&] {
-        ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)pair::SMEM_BYTES) == cudaSuccess &&
-                  cudaFuncSetAttribute(bi_gemm_bf16_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)pair::SMEM_BYTES) == cudaSuccess;
     });
     return ok[dev];
 }
 
-// Clusters of the split pair kernel that fit on the device at once (cached per device).  A
-// split grid never exceeds it: the last K slice of a tile waits for the other slices, so
-// every cluster must be resident together.
-int pair_clusters() {
-    static std::once_flag once[64];
-    static int cached[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-    if (!pair_smem_attr()) return -1;
-    std::call_once(once[dev], [&] {
-        cached[dev] = -1;
-        const int sms = num_sms();
-        if (sms < 2) return;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(sms & ~1));
-        cfg.blockDim = dim3(THREADS);
-        cfg.dynamicSmemBytes = pair::SMEM_BYTES;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, bi_gemm_bf16_pair_kernel<true>, &cfg) != cudaSuccess) {
-            (void)cudaGetLastError();
-            return;
-        }
-        if (n <= 0) return;
-        cached[dev] = n < sms / 2 ? n : sms / 2;
-    });
-    return cached[dev];
-}
-
-// Workspace of a pair-kernel call with S > 1 slices: counters at the start (zero between
-// calls), fp32 partials of slices 0 .. S-2 at the end.
-size_t split_counter_bytes(int64_t M, int64_t N) {
-    const int64_t tiles = ((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N);
-    return (size_t)(((tiles * pair::CNT_PER_TILE * 4) + 255) / 256 * 256);
-}
-size_t split_partial_bytes(int64_t M, int64_t N, int S) { return (size_t)(S - 1) * M * N * sizeof(float); }
-
-// The CTA-pair kernel: 256 x 256 tiles over 2-CTA clusters, one cluster per SM pair at most,
-// K split into `splits` slices.
+// The CTA-pair kernel: 256 x 256 tiles over 2-CTA clusters, one cluster per SM pair at most.
 int launch_gemm_pair(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N,
-                     int64_t K, bool c_bf16, int splits, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                     int64_t K, bool c_bf16, cudaStream_t stream) {
     uint32_t* err = bi::device_error_word();
     if (!err || !pair_smem_attr()) return BI_ERR_CUDA;
-    if (splits < 1 || splits > pair::MAX_SPLIT || splits > (K + BK - 1) / BK) return BI_ERR_INVALID_ARG;
     const int sms = num_sms();
     if (sms < 2) return BI_ERR_CUDA;
-    int64_t clusters = sms / 2;
-    if (splits > 1) {
-        const int c = pair_clusters();
-        if (c <= 0) return BI_ERR_CUDA;
-        if (c < clusters) clusters = c;
-    }
-    uint32_t* cnt = nullptr;
-    float* part = nullptr;
-    if (splits > 1) {
-        const size_t cb = split_counter_bytes(M, N), pb = split_partial_bytes(M, N, splits);
-        if (!ws || !bi::aligned16(ws) || ws_bytes < cb + pb) return BI_ERR_WORKSPACE;
-        cnt = static_cast<uint32_t*>(ws);
-        part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + (ws_bytes - pb) / 16 * 16);
-    }
+    const int64_t clusters = sms / 2;
     CUtensorMap tmA, tmW;
     if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK,
                           pair::ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -745,20 +885,101 @@ int launch_gemm_pair(const void* A, int64_t lda, const void* W, int64_t ldw, voi
     if (!bi::make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)N, (uint64_t)K, (uint64_t)ldw * 2, 64,
                           BK, CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
-    const int64_t units =
-        ((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N) * (int64_t)splits;
-    if (units > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
+    const int64_t tiles = ((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N);
     const int gm = 16;  // row tiles per group of the tile walk (L2 reuse of A and W blocks)
-    const int64_t pairs = units < clusters ? units : clusters;
-    const dim3 grid((unsigned)(2 * pairs));
+    const int64_t pairs = tiles < clusters ? tiles : clusters;
     // the pair kernel's cluster shape is compiled in (__cluster_dims__)
-    const cudaError_t e =
-        splits > 1 ? bi::launch_pdl(bi_gemm_bf16_pair_kernel<true>, grid, dim3(THREADS), pair::SMEM_BYTES, stream, 1u,
-                                    tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, splits, cnt, part, err)
-                   : bi::launch_pdl(bi_gemm_bf16_pair_kernel<false>, grid, dim3(THREADS), pair::SMEM_BYTES, stream,
-                                    1u, tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, 1,
-                                    static_cast<uint32_t*>(nullptr), static_cast<float*>(nullptr), err);
-    if (e != cudaSuccess) return BI_ERR_CUDA;
+    if (bi::launch_pdl(bi_gemm_bf16_pair_kernel, dim3((unsigned)(2 * pairs)), dim3(THREADS), pair::SMEM_BYTES, stream,
+                       0u, tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm, err) != cudaSuccess)
+        return BI_ERR_CUDA;
+    return bi::launch_status();
+}
+
+// Clusters of 2S CTAs of the cluster-split kernel that fit on the device at once (cached per
+// device and S).  The grid never exceeds it, so every cluster is resident and walks its tiles.
+int split_clusters(int S) {
+    static std::mutex mu;
+    static int cached[64][cs::MAX_S + 1];
+    int dev = 0;
+    if (S < 2 || S > cs::MAX_S || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev][S] == 0) {
+        cached[dev][S] = -1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * S));
+        cfg.blockDim = dim3(THREADS);
+        cfg.dynamicSmemBytes = cs::SMEM_BYTES;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)(2 * S);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, bi_gemm_bf16_cluster_kernel, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return -1;
+        }
+        cached[dev][S] = n > 0 ? n : -1;
+    }
+    return cached[dev][S];
+}
+
+bool cluster_smem_attr() {
+    static std::once_flag once[64];
+    static bool ok[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::call_once(once[dev], [&] {
+        ok[dev] = cudaFuncSetAttribute(bi_gemm_bf16_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)cs::SMEM_BYTES) == cudaSuccess &&
+                  cudaFuncSetAttribute(bi_gemm_bf16_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                       1) == cudaSuccess;
+    });
+    return ok[dev];
+}
+
+// The cluster-split kernel: 256 x 256 tiles, K in S slices on S CTA pairs of one cluster.
+int launch_gemm_cluster(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N,
+                        int64_t K, bool c_bf16, int S, cudaStream_t stream) {
+    uint32_t* err = bi::device_error_word();
+    if (!err || !cluster_smem_attr()) return BI_ERR_CUDA;
+    if (S < 2 || S > cs::MAX_S || S > (K + BK - 1) / BK) return BI_ERR_INVALID_ARG;
+    const int fit = split_clusters(S);
+    if (fit <= 0) return BI_ERR_CUDA;
+    CUtensorMap tmA, tmW;
+    if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, BK,
+                          pair::ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    if (!bi::make_tmap_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, (uint64_t)N, (uint64_t)K, (uint64_t)ldw * 2, 64,
+                          BK, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    const int64_t tiles = ((M + pair::TILE_M - 1) / pair::TILE_M) * ((N + pair::TILE_N - 1) / pair::TILE_N);
+    const int64_t clusters = tiles < fit ? tiles : fit;
+    const int gm = 16;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * S * clusters));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = cs::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    unsigned na = 0;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)(2 * S);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+    if (bi::pdl_enabled()) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, bi_gemm_bf16_cluster_kernel, tmA, tmW, C, (int)M, (int)N, (int)K, c_bf16 ? 1 : 0, gm,
+                           S, err) != cudaSuccess)
+        return BI_ERR_CUDA;
     return bi::launch_status();
 }
 
@@ -785,15 +1006,13 @@ int splits_for(int64_t N, int64_t K) {
 }
 
 int launch_gemm(const void* A, int64_t lda, const void* W, int64_t ldw, void* C, int64_t M, int64_t N, int64_t K,
-                bool c_bf16, int splits, void* ws, size_t ws_bytes, cudaStream_t stream) {
-    if (use_pairs(N, K)) return launch_gemm_pair(A, lda, W, ldw, C, M, N, K, c_bf16, splits, ws, ws_bytes, stream);
+                bool c_bf16, int splits, cudaStream_t stream) {
+    if (use_pairs(N, K)) {
+        if (splits == 1) return launch_gemm_pair(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
+        return launch_gemm_cluster(A, lda, W, ldw, C, M, N, K, c_bf16, splits, stream);
+    }
     if (splits != 1) return BI_ERR_INVALID_ARG;
     return launch_gemm_bn<256>(A, lda, W, ldw, C, M, N, K, c_bf16, stream);
-}
-
-size_t gemm_ws_bytes(int64_t M, int64_t N, int S) {
-    if (M <= 0 || N <= 0 || S <= 1) return 0;
-    return split_counter_bytes(M, N) + split_partial_bytes(M, N, S);
 }
 
 int gemm_shape_checks(const void* A, const void* W, const void* C, int64_t M, int64_t N, int64_t K, int c_dtype) {
@@ -852,39 +1071,38 @@ BI_API int bi_gemm_splits(int64_t N, int64_t K) {
 }
 
 BI_API size_t bi_gemm_counter_bytes(int64_t M, int64_t N, int64_t K) {
-    if (M <= 0 || N <= 0 || K <= 0 || splits_for(N, K) <= 1) return 0;
-    return split_counter_bytes(M, N);
+    (void)M; (void)N; (void)K;
+    return 0;  // a K split meets on chip: no counters
 }
 
 BI_API size_t bi_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
-    if (N <= 0 || K <= 0) return 0;
-    return gemm_ws_bytes(M, N, splits_for(N, K));
+    (void)M; (void)N; (void)K;
+    return 0;  // a K split meets on chip: no workspace
 }
 
 BI_API int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype, void* ws,
                    size_t ws_bytes, void* stream) {
+    (void)ws; (void)ws_bytes;
     const int c = gemm_shape_checks(A, W, C, M, N, K, c_dtype);
     if (c < 0) return BI_OK;
     if (c != BI_OK) return c;
-    const int S = splits_for(N, K);
-    if (S > 1 && (!ws || !bi::aligned16(ws) || ws_bytes < gemm_ws_bytes(M, N, S))) return BI_ERR_WORKSPACE;
-    return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, S, ws, ws_bytes, bi::as_stream(stream));
+    return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, splits_for(N, K), bi::as_stream(stream));
 }
 
 BI_API size_t bi_ctrl_gemm_split_workspace_size(int64_t M, int64_t N, int64_t K, int32_t splits) {
-    (void)K;
-    return gemm_ws_bytes(M, N, splits);
+    (void)M; (void)N; (void)K; (void)splits;
+    return 0;
 }
 
 BI_API int bi_ctrl_gemm_split(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype,
                               int32_t splits, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws; (void)ws_bytes;
     const int c = gemm_shape_checks(A, W, C, M, N, K, c_dtype);
     if (c < 0) return BI_OK;
     if (c != BI_OK) return c;
     if (!use_pairs(N, K) && splits != 1) return BI_ERR_UNSUPPORTED_SHAPE;
-    if (splits < 1 || splits > pair::MAX_SPLIT || splits > (K + BK - 1) / BK) return BI_ERR_INVALID_ARG;
-    if (splits > 1 && (!ws || !bi::aligned16(ws) || ws_bytes < gemm_ws_bytes(M, N, splits))) return BI_ERR_WORKSPACE;
-    return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, splits, ws, ws_bytes, bi::as_stream(stream));
+    if (splits < 1 || splits > cs::MAX_S || splits > (K + BK - 1) / BK) return BI_ERR_INVALID_ARG;
+    return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, splits, bi::as_stream(stream));
 }
 
 BI_API size_t bi_ctrl_gemm_splitk_workspace_size(int64_t M, int64_t N, int64_t K) {
@@ -900,7 +1118,7 @@ BI_API int bi_ctrl_gemm_splitk(const void* A, const void* W, void* C, int64_t M,
     if (c != BI_OK) return c;
     cudaStream_t s = bi::as_stream(stream);
     const int S = splitk_for(M, N, K);
-    if (S == 1) return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, 1, nullptr, 0, s);
+    if (S == 1) return launch_gemm(A, K, W, N, C, M, N, K, c_dtype == BI_BF16, 1, s);
     const size_t need = (size_t)S * M * N * sizeof(float);
     if (!ws || ws_bytes < need || !bi::aligned16(ws)) return BI_ERR_WORKSPACE;
     const int64_t KS = K / S;
@@ -908,7 +1126,7 @@ BI_API int bi_ctrl_gemm_splitk(const void* A, const void* W, void* C, int64_t M,
     for (int i = 0; i < S; ++i) {
         const int st = launch_gemm(static_cast<const __nv_bfloat16*>(A) + i * KS, K,
                                    static_cast<const __nv_bfloat16*>(W) + i * KS * N, N, part + (int64_t)i * M * N, M,
-                                   N, KS, false, 1, nullptr, 0, s);
+                                   N, KS, false, 1, s);
         if (st != BI_OK) return st;
     }
     const int64_t MN = M * N;  // N % 8 == 0, so MN is a multiple of 4

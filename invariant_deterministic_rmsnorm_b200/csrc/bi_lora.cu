@@ -674,7 +674,7 @@ int launch_expand(const float* t, const void* B, void* y, int64_t M, int64_t N, 
     dim3 grid((unsigned)((N + EX_TN - 1) / EX_TN), (unsigned)((M + EX_TM - 1) / EX_TM));
     auto k = ybf16 ? lora_expand_kernel<R, true> : lora_expand_kernel<R, false>;
     if (!set_smem_once(k, L::BYTES)) return BI_ERR_CUDA;
-    if (bi::launch_pdl(k, grid, dim3(EX_THREADS), L::BYTES, s, 1u, t, static_cast<const __nv_bfloat16*>(B), y,
+    if (bi::launch_pdl(k, grid, dim3(EX_THREADS), L::BYTES, s, 0u, t, static_cast<const __nv_bfloat16*>(B), y,
                        (int)M, (int)N, ldy, scale) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();

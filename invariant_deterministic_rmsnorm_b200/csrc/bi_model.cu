@@ -197,7 +197,7 @@ BI_API int bi_embed(const int32_t* tokens, const void* table, void* out, int64_t
     if (H % 8 != 0 || !bi::aligned16(table) || !bi::aligned16(out)) return BI_ERR_MISALIGNED;
     uint32_t* err = bi::device_error_word();
     if (!err) return BI_ERR_CUDA;
-    if (bi::launch_pdl(embed_kernel, dim3((unsigned)T), dim3(256), 0, bi::as_stream(stream), 1u,
+    if (bi::launch_pdl(embed_kernel, dim3((unsigned)T), dim3(256), 0, bi::as_stream(stream), 0u,
                        tokens, static_cast<const __nv_bfloat16*>(table), static_cast<__nv_bfloat16*>(out), H, vocab,
                        err) != cudaSuccess)
         return BI_ERR_CUDA;
@@ -212,7 +212,7 @@ BI_API int bi_rope_table(void* table, int64_t positions, int32_t head_dim, doubl
     const int half = head_dim / 2;
     if (positions > ((int64_t)1 << 38) / half) return BI_ERR_UNSUPPORTED_SHAPE;
     const int64_t n = positions * half;
-    if (bi::launch_pdl(rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, bi::as_stream(stream), 1u,
+    if (bi::launch_pdl(rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, bi::as_stream(stream), 0u,
                        static_cast<float2*>(table), positions, half, log(theta), head_dim) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();
@@ -231,7 +231,7 @@ BI_API int bi_rope(void* x, int64_t T, int64_t ld_row, int32_t heads, int32_t he
     const int work = heads * (head_dim / 4);
     if ((work + 127) / 128 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
     dim3 grid((unsigned)T, (unsigned)((work + 127) / 128));
-    if (bi::launch_pdl(rope_kernel, dim3(grid), dim3(128), 0, bi::as_stream(stream), 1u,
+    if (bi::launch_pdl(rope_kernel, dim3(grid), dim3(128), 0, bi::as_stream(stream), 0u,
                        static_cast<__nv_bfloat16*>(x), ld_row, heads, head_dim, pos,
                        static_cast<const float4*>(table), table_rows, err) != cudaSuccess)
         return BI_ERR_CUDA;
@@ -246,7 +246,7 @@ BI_API int bi_kv_append(const void* src, int64_t ld_src, const int32_t* dst_row,
     if (row_elems % 8 != 0 || ld_src % 8 != 0 || !bi::aligned16(src) || !bi::aligned16(dst)) return BI_ERR_MISALIGNED;
     uint32_t* err = bi::device_error_word();
     if (!err) return BI_ERR_CUDA;
-    if (bi::launch_pdl(kv_append_kernel, dim3((unsigned)T), dim3(256), 0, bi::as_stream(stream), 1u,
+    if (bi::launch_pdl(kv_append_kernel, dim3((unsigned)T), dim3(256), 0, bi::as_stream(stream), 0u,
                        static_cast<const __nv_bfloat16*>(src), ld_src, dst_row, static_cast<__nv_bfloat16*>(dst),
                        row_elems, dst_rows, err) != cudaSuccess)
         return BI_ERR_CUDA;
@@ -260,7 +260,7 @@ BI_API int bi_add(void* h, int64_t ldh, const void* d, int64_t ldd, int64_t T, i
     if (N % 8 != 0 || ldh % 8 != 0 || ldd % 8 != 0 || !bi::aligned16(h) || !bi::aligned16(d)) return BI_ERR_MISALIGNED;
     if ((N / 8 + 255) / 256 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
     if (bi::launch_pdl(add_kernel, dim3((unsigned)T, (unsigned)((N / 8 + 255) / 256)), dim3(256), 0,
-                       bi::as_stream(stream), 1u,
+                       bi::as_stream(stream), 0u,
                        static_cast<__nv_bfloat16*>(h), ldh, static_cast<const __nv_bfloat16*>(d), ldd,
                        N) != cudaSuccess)
         return BI_ERR_CUDA;
@@ -275,7 +275,7 @@ BI_API int bi_swiglu(const void* gu, int64_t ld_gu, void* out, int64_t ld_out, i
         return BI_ERR_MISALIGNED;
     if ((N / 8 + 255) / 256 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
     if (bi::launch_pdl(swiglu_kernel, dim3((unsigned)T, (unsigned)((N / 8 + 255) / 256)), dim3(256), 0,
-                       bi::as_stream(stream), 1u,
+                       bi::as_stream(stream), 0u,
                        static_cast<const __nv_bfloat16*>(gu), ld_gu, static_cast<__nv_bfloat16*>(out), ld_out,
                        N) != cudaSuccess)
         return BI_ERR_CUDA;
@@ -286,7 +286,7 @@ BI_API int bi_argmax(const float* x, int64_t ld, int64_t T, int64_t N, int32_t* 
     if (T < 0 || N <= 0 || ld < N || !rows_ok(T) || N > 0x7fffffffLL) return BI_ERR_INVALID_ARG;
     if (T == 0) return BI_OK;
     if (!x || !out) return BI_ERR_INVALID_ARG;
-    if (bi::launch_pdl(argmax_kernel, dim3((unsigned)T), dim3(ARGMAX_THREADS), 0, bi::as_stream(stream), 1u,
+    if (bi::launch_pdl(argmax_kernel, dim3((unsigned)T), dim3(ARGMAX_THREADS), 0, bi::as_stream(stream), 0u,
                        x, ld, N, out) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();
@@ -296,7 +296,7 @@ BI_API int bi_advance(int32_t* v, int64_t n, int32_t step, void* stream) {
     if (n < 0 || n > ((int64_t)1 << 40)) return BI_ERR_INVALID_ARG;
     if (n == 0) return BI_OK;
     if (!v) return BI_ERR_INVALID_ARG;
-    if (bi::launch_pdl(advance_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, bi::as_stream(stream), 1u,
+    if (bi::launch_pdl(advance_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, bi::as_stream(stream), 0u,
                        v, n, step) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();

@@ -488,7 +488,7 @@ BI_API int bi_prefill_attn(const void* q, int64_t ldq, int64_t q_rows, const voi
                           64, KB, CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
     dim3 grid((unsigned)n_tiles, (unsigned)Hq);
-    if (bi::launch_pdl(prefill_attn_tc_kernel, grid, dim3(THREADS), SMEM_BYTES, bi::as_stream(stream), 1u, tmQ, tmK,
+    if (bi::launch_pdl(prefill_attn_tc_kernel, grid, dim3(THREADS), SMEM_BYTES, bi::as_stream(stream), 0u, tmQ, tmK,
                        tmV, q_indptr, q_tile_indptr, kv_indptr, q_pos0, B, Hq, Hkv, (int)q_rows, (int)cache_tokens,
                        n_tiles, (float)((double)scale * 1.4426950408889634), static_cast<__nv_bfloat16*>(out), ldo,
                        err) != cudaSuccess)

@@ -213,7 +213,7 @@ int launch_rows(const TIO* x, const TW* w, TIO* y, int64_t M, int nvec, int thre
         per_sm = (n > 0 ? n : 1) * sms;
     }
     const int64_t grid = M < per_sm ? M : per_sm;
-    if (bi::launch_pdl(rmsnorm_rows_kernel<TIO, TW, VPT>, dim3((unsigned)grid), dim3(threads), 0, s, 1u, x, w, y, M,
+    if (bi::launch_pdl(rmsnorm_rows_kernel<TIO, TW, VPT>, dim3((unsigned)grid), dim3(threads), 0, s, 0u, x, w, y, M,
                        nvec, ldx, ldy, hf, eps) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();

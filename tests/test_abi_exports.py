@@ -110,27 +110,23 @@ def test_model_ops_host_checks(lib):
 
 
 def test_gemm_split_plan_host(lib):
-    """The GEMM plan keeps one K slice for every shape (the split was measured to lose at large
-    M, and the plan may not depend on M), so bi_gemm needs no workspace.  The split kernel's
-    workspace arithmetic and argument checks are those of bi_ctrl_gemm_split."""
+    """A K split meets on chip, so no GEMM call needs a workspace.  The plan's split counts are
+    those bi_gemm_splits reports (a function of N and K only); the argument checks of
+    bi_ctrl_gemm_split run before any launch."""
     for N, K in ((6144, 4096), (4096, 4096), (4096, 14336), (14336, 4096), (512, 256), (28672, 4096),
                  (32000, 4096)):
-        assert lib.bi_gemm_splits(N, K) == 1, (N, K)
+        assert 1 <= lib.bi_gemm_splits(N, K) <= 4, (N, K)
         assert lib.bi_gemm_workspace_size(4096, N, K) == 0
         assert lib.bi_gemm_counter_bytes(4096, N, K) == 0
+    for N, K in ((28672, 4096), (32000, 4096), (512, 256)):
+        assert lib.bi_gemm_splits(N, K) == 1, (N, K)  # single-CTA plan, or too small to split
     for M in (1, 8, 255, 256, 257, 4096):
-        tiles = -(-M // 256) * 16
-        counters = -(-tiles * 8 * 4 // 256) * 256  # one counter per (tile, CTA, epilogue warp)
-        for S in (2, 3, 4):
-            assert lib.bi_ctrl_gemm_split_workspace_size(M, 4096, 14336, S) == counters + (S - 1) * M * 4096 * 4
-        assert lib.bi_ctrl_gemm_split_workspace_size(M, 4096, 14336, 1) == 0
+        for S in (1, 2, 3, 4):
+            assert lib.bi_ctrl_gemm_split_workspace_size(M, 4096, 14336, S) == 0
     a = 1 << 20
     P = ctypes.c_void_p
-    # a split without a workspace, with one too small or misaligned: refused before any launch
-    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 2, None, 0, None) == 4
-    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 2, P(a), 64, None) == 4
-    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 2, P(a + 8), 1 << 30, None) == 4
     assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 5, None, 0, None) == 1
+    assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 4096, 1, 0, None, 0, None) == 1
     assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 64, 1, 2, None, 0, None) == 1  # 1 K block
     assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 28672, 4096, 1, 2, None, 0, None) == 2
     assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 0, 4096, 4096, 1, 2, None, 0, None) == 0  # empty batch

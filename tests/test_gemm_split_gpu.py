@@ -1,9 +1,10 @@
 """The K split of bi_gemm's CTA-pair plan on the GPU.
 
 "Defeating Nondeterminism in LLM Inference", section "Multiplicación de matrices": a split
-of K is batch-invariant when it does not depend on the batch.  bi_gemm's plan keeps one
-slice (S = 1) for every shape; bi_ctrl_gemm_split runs the same CTA-pair kernel with a
-split count given by the caller, which the tests below use to reach every S.
+of K is batch-invariant when it does not depend on the batch.  bi_ctrl_gemm_split runs
+bi_gemm's tiles with a split count given by the caller (S = 1: the CTA-pair kernel; S > 1:
+the cluster-split kernel, S CTA pairs whose partials meet in distributed shared memory),
+which the tests below use to reach every S.
 
   * small-integer operands: every partial sum is exact in fp32, so the output equals the
     oracle bit for bit at every S.
@@ -11,7 +12,7 @@ split count given by the caller, which the tests below use to reach every S.
     ((P0 + P1) + P2) + P3 (any order that adds the two 1s first gives 2^24 + 2).
   * random operands: relative Frobenius error <= 1e-5 against the fp64 oracle.
   * bits of a row do not depend on the batch at a fixed S.
-  * the counters of the workspace are zero again after a call.
+  * no workspace is needed, and two calls in a row give the same bits.
 """
 import numpy as np
 import pytest
@@ -28,8 +29,8 @@ pytestmark = pytest.mark.gpu
 RAGGED = (333, 776, 2056)
 
 
-def _split(A_np, W_np, S, out=torch.float32, ws=None):
-    C = binding.bi_ctrl_gemm_split(dev(A_np), dev(W_np), S, out_dtype=out, workspace=ws)
+def _split(A_np, W_np, S, out=torch.float32):
+    C = binding.bi_ctrl_gemm_split(dev(A_np), dev(W_np), S, out_dtype=out)
     torch.cuda.synchronize()
     return host(C)
 
@@ -94,30 +95,34 @@ def test_split_rows_are_batch_invariant(S):
         assert np.array_equal(solo[0].view(np.uint32), full[r].view(np.uint32)), r
 
 
-def test_counters_return_to_zero():
+def test_no_workspace_and_repeatable():
     M, N, K = RAGGED
-    S = 3
     lib = binding.library()
-    need = lib.bi_ctrl_gemm_split_workspace_size(M, N, K, S)
-    counters = need - (S - 1) * M * N * 4
-    assert counters > 0
-    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for S in (1, 2, 3, 4):
+        assert lib.bi_ctrl_gemm_split_workspace_size(M, N, K, S) == 0
+    assert lib.bi_gemm_workspace_size(M, N, K) == 0
     A, W = inputs.gemm_case(M, N, K, seed_a=67, seed_w=68)
     binding.bi_clear_device_error()
-    first = _split(A, W, S, ws=ws)
-    assert int(ws[:counters].count_nonzero()) == 0
-    again = _split(A, W, S, ws=ws)  # the same workspace serves the next call
+    first = _split(A, W, 3)
+    again = _split(A, W, 3)
     assert np.array_equal(first.view(np.uint32), again.view(np.uint32))
     assert binding.bi_get_device_error() == 0
 
 
-def test_split_workspace_and_argument_errors():
+@pytest.mark.parametrize("S", [2, 3, 4])
+def test_split_bf16_output_is_the_rounded_fp32(S):
+    M, N, K = RAGGED
+    A, W = inputs.gemm_case(M, N, K, seed_a=75, seed_w=76)
+    assert np.array_equal(_split(A, W, S, torch.bfloat16), inputs.f32_to_bf16_bits(_split(A, W, S)))
+
+
+def test_split_argument_errors():
     A, W = inputs.gemm_case(8, 4096, 4096, seed_a=69, seed_w=70)
     a, w = dev(A), dev(W)
     with pytest.raises(binding.BIError):
-        binding.bi_ctrl_gemm_split(a, w, 2, workspace=torch.zeros(16, dtype=torch.uint8, device="cuda"))
-    with pytest.raises(binding.BIError):
         binding.bi_ctrl_gemm_split(a, w, 5)
+    with pytest.raises(binding.BIError):
+        binding.bi_ctrl_gemm_split(a, w, 0)
     wide = dev(inputs.gemm_case(8, 28672, 64, seed_a=71, seed_w=72)[1])
     with pytest.raises(binding.BIError):
         binding.bi_ctrl_gemm_split(dev(A[:, :64]), wide, 2)
