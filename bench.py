@@ -459,6 +459,19 @@ def run_ours(args, rank, world, local_rank):
     gates = gate_table(device, stream, load_peaks()[0]) if not args.no_gates else None
 
     peaks, peak_src = load_peaks()
+    # Back-to-back time of each op's kernel at the step's own configuration (from the gate table:
+    # launches in a graph with no event between them, inputs rotating past the L2).  Inside the
+    # step every op is bracketed by events, so its time there also holds its launch.
+    b2b = {}
+    if gates:
+        pick = {"rmsnorm": ("rmsnorm_H4096", "M", M_TOKENS), "gemm_qkv": ("gemm_K4096_N6144", "M", M_TOKENS),
+                "gemm_up": ("gemm_K4096_N14336", "M", M_TOKENS), "gemm_down": ("gemm_K14336_N4096", "M", M_TOKENS),
+                "lora_shrink": (f"lora_shrink_r{LORA_RANK}", "M", M_TOKENS),
+                "lora_expand": ("lora_expand_r16", "M", M_TOKENS), "decode_attn": ("decode_attn", "B", args.attn_batch)}
+        for name, (table, key, n) in pick.items():
+            for row in gates.get(table, {}).get("rows", []):
+                if row.get(key) == n:
+                    b2b[name] = row
     # A kernel timed inside a long step (a timed region of half a second or more, long enough for
     # the 1 kW power cap to engage) is compared with the sustained bf16 figure; a short region
     # gets the burst figure.
@@ -478,6 +491,9 @@ def run_ours(args, rank, world, local_rank):
             unit = "TFLOP/s"
         per_op[op["name"]] = {"us": round(avg_s * 1e6, 2), "achieved": round(ach, 1), "unit": unit,
                               "frac": round(ach / peak, 4), "desc": op["desc"]}
+        if op["name"] in b2b:
+            r_ = b2b[op["name"]]
+            per_op[op["name"]]["back_to_back"] = {"us": r_["us"], "achieved": r_["achieved"], "frac": r_["frac"]}
 
     gemm_ops = [i for i, op in enumerate(ops) if op["kind"] == "tensor"]
     if gemm_ops:
@@ -693,8 +709,24 @@ def gate_table(device, stream, peaks):
 
     def point(key, n, work, ms, peak, gate, unit):
         ach = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
-        return {key: n, "us": round(ms * 1e3, 2), "achieved": round(ach, 1), "frac": round(ach / peak, 4),
-                "gate": gate, "met": bool(ach / peak >= gate)}
+        pt = {key: n, "us": round(ms * 1e3, 2), "achieved": round(ach, 1), "frac": round(ach / peak, 4),
+              "gate": gate, "met": bool(ach / peak >= gate)}
+        if unit == "GB/s":
+            # context: a device-to-device copy with the same traffic (half read, half written), timed the
+            # same way -- what launch, ramp-up and drain leave of the peak at this size
+            cms = copy_ms(work)
+            pt["copy_us"] = round(cms * 1e3, 2)
+            pt["frac_of_copy"] = round(cms / ms, 4)
+        return pt
+
+    def copy_ms(nbytes):
+        half = max(16, (int(nbytes) // 2) // 16 * 16)
+        R = _copies(nbytes)
+        src = [torch.empty(half, dtype=torch.uint8, device=device).fill_(1) for _ in range(R)]
+        dst = [torch.empty(half, dtype=torch.uint8, device=device) for _ in range(R)]
+        ms = _time_graph([lambda j=j: dst[j].copy_(src[j], non_blocking=True) for j in range(R)], stream)
+        del src, dst
+        return ms
 
     out = {"peaks": {"bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"]}}
     with torch.cuda.stream(stream):
@@ -734,6 +766,18 @@ def gate_table(device, stream, peaks):
                                   "GB/s"))
                 del xs
             out[f"lora_shrink_r{r}"] = {"unit": "GB/s", "rows": rows}
+        # the expand (no target of its own; the shrink's companion), r = 16 into bf16 y
+        B_l = rows_dev(81, 16, HIDDEN).mul_(0.02)
+        rows = []
+        for M in (1024, 4096):
+            R = _copies(2 * 2 * HIDDEN * M)
+            ys = [rows_dev(100 + j, M, HIDDEN) for j in range(R)]
+            t = rows_dev(101, M, 16).float()
+            ms = _time_graph([lambda j=j: B.bi_lora_expand(t, B_l, ys[j], stream=stream) for j in range(R)], stream)
+            rows.append(point("M", M, 4 * M * 16 + 2 * 16 * HIDDEN + 2 * 2 * HIDDEN * M, ms, peaks["hbm_gbs"], 0.75,
+                              "GB/s"))
+            del ys
+        out["lora_expand_r16"] = {"unit": "GB/s", "rows": rows}
         kv_len = inputs.kv_lengths(256)
         indptr, T = inputs.kv_layout(kv_len, 256)
         g = torch.Generator(device=device).manual_seed(5)

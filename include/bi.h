@@ -66,8 +66,8 @@ int bi_abi_version(void);
  * (0 = no error).  Return value: BI_OK, BI_ERR_TIMEOUT if *code != 0, or
  * BI_ERR_CUDA.  bi_clear_device_error() zeroes the word, ordered on `stream`.
  * Bits: 0x1 a producer's wait for a free stage, 0x2 a wait for a loaded stage,
- * 0x4 a wait for the accumulator, 0x8 a cluster handshake, 0x10 a GEMM's last K slice
- * waiting for the other slices of its tile; 0x100 decode-attention
+ * 0x4 a wait for the accumulator, 0x8 a cluster handshake (partials or a receive buffer of
+ * another CTA of the cluster); 0x100 decode-attention
  * layout, 0x200 embedding token id, 0x400 KV-append destination row, 0x800
  * prefill-attention layout, 0x1000 RoPE position (the last five are input checks made on
  * the device).
@@ -113,30 +113,19 @@ int bi_rmsnorm(const void* x, const void* w, void* y, int64_t M, int64_t H, int6
  *   C    device, [M, N] row-major, dtype c_dtype (BI_F32: the fp32 accumulator as is;
  *        BI_BF16: the accumulator rounded to nearest even)
  *   M    >= 0 rows.  N, K > 0, multiples of 8 (16-byte rows for the TMA unit).
- *   ws, ws_bytes  workspace of at least bi_gemm_workspace_size(M, N, K) bytes, 16-byte
- *        aligned; NULL is accepted when that size is 0, as it is for every shape in this
- *        version (the plan does not split K).  A plan that splits K uses it like this:
- *          - its first bi_gemm_counter_bytes(M, N, K) bytes are counters.  They must be
- *            zero when the call starts, and a call that completes leaves them zero.
- *            Zero-fill a new workspace once.  After a call that set a device error bit,
- *            zero it again before reuse.
- *          - fp32 partial sums are written to the last bytes of the buffer.
- *          - several calls may share one workspace when no call's partials can reach
- *            another call's counters: ws_bytes >= the largest counter bytes plus the
- *            largest partial bytes among them.  Calls that run concurrently need
- *            separate workspaces.
- *        BI_ERR_WORKSPACE if the workspace is missing or too small.
+ *   ws, ws_bytes  unused: no plan needs a workspace (bi_gemm_workspace_size and
+ *        bi_gemm_counter_bytes return 0), so NULL and 0 are fine.  Kept in the signature so that
+ *        callers written against a plan with a workspace stay valid.
  *
  * Arithmetic: bf16 x bf16 -> fp32 in tensor memory, K walked in ascending 64-wide
  * blocks.  The plan (tile, MMA shape, K order, split count) is a function of (N, K) and
  * the device only:
  *   - N <= 256 x (SM pairs): 256 x 256 tiles on 2-CTA clusters,
- *     tcgen05.mma.cta_group::2 256x256x16.  The kernel can split K into S contiguous
- *     slices; slice s accumulates its K blocks in fp32, and the output is
- *     ((P0 + P1) + ...) + P(S-1), summed in that order in fp32.  The plan's
- *     S = bi_gemm_splits(N, K) is 1 for every shape: a split pays only while M fills one or
- *     two rows of tiles and costs more than it saves at larger M.  bi_ctrl_gemm_split runs
- *     other S.
+ *     tcgen05.mma.cta_group::2 256x256x16.  K may be cut into S = bi_gemm_splits(N, K)
+ *     contiguous slices (S <= 4): slice s accumulates its K blocks in fp32, and the output is
+ *     ((P0 + P1) + ...) + P(S-1), summed in that order in fp32 and rounded once.  The S slices
+ *     of a tile run on S CTA pairs of one thread-block cluster, and their partials meet in
+ *     distributed shared memory, never in HBM.  bi_ctrl_gemm_split runs other S.
  *   - wider N: 128 x 256 tiles on one CTA, tcgen05.mma.cta_group::1 128x256x16, no split.
  * Rows past M and columns past N or K are zero-filled on load and never stored.  C may
  * not alias A or W.
@@ -163,11 +152,13 @@ int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t
  *   ws, ws_bytes  workspace of bi_lora_shrink_workspace_size() bytes.  That size is
  *         always 0, because the partials never leave the chip.  ws may be NULL.
  *
- * Arithmetic: one cluster of split_k CTAs per 64-row tile.  CTA s accumulates its
- * contiguous K slice with mma.sync (bf16 in, fp32 accumulate, K ascending).  CTA 0
- * then adds the partials over distributed shared memory, s = 0, 1, ..., split_k-1 in
- * order, each add rounded to nearest.  No atomics.  The plan depends on (K, r,
- * split_k) only.
+ * Arithmetic: slice s of K (the contiguous range [s K / split_k, (s + 1) K / split_k)) gives
+ * the partial P_s, accumulated with mma.sync (bf16 in, fp32 accumulate) in 16-deep K steps
+ * in ascending order.  t = ((P_0 + P_1) + ...) + P_{split_k - 1}, each add rounded to nearest.
+ * No atomics.  A thread-block cluster of split_k CTAs (CTA s = slice s) computes 128-row tiles
+ * with eight compute warps of 16 rows; the partials meet in distributed shared memory, and every
+ * CTA of the cluster adds the slices of 128 / split_k of the tile's rows.  The plan depends on
+ * (K, r, split_k) only.
  */
 size_t bi_lora_shrink_workspace_size(int64_t M, int64_t K, int32_t r, int32_t split_k);
 int bi_lora_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r, int32_t split_k,

@@ -61,8 +61,8 @@ int bi_ctrl_gemm_splitk(const void* A, const void* W, void* C, int64_t M, int64_
  * batch-invariant like bi_gemm; it is here to time the plan's candidates against each
  * other at every batch size.  splits in 1 .. 4 and at most ceil(K / 64); a weight too wide
  * for the CTA-pair tiles takes splits = 1 only (BI_ERR_UNSUPPORTED_SHAPE otherwise).
- * The workspace follows bi_gemm's rules, with bi_ctrl_gemm_split_workspace_size bytes
- * (counters first, bi_gemm_counter_bytes' layout).
+ * splits = 1 runs the CTA-pair kernel; splits > 1 runs the cluster-split kernel (bi.h, bi_gemm).
+ * No workspace is needed: bi_ctrl_gemm_split_workspace_size returns 0, and ws may be NULL.
  */
 size_t bi_ctrl_gemm_split_workspace_size(int64_t M, int64_t N, int64_t K, int32_t splits);
 int bi_ctrl_gemm_split(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K, int c_dtype,

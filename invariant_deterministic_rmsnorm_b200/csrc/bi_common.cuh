@@ -69,7 +69,6 @@ enum : uint32_t {
     DEVERR_WAIT_FULL = 1u << 1,     // MMA issuer waited too long for a loaded stage
     DEVERR_WAIT_ACCUM = 1u << 2,    // epilogue waited too long for the accumulator
     DEVERR_WAIT_CLUSTER = 1u << 3,  // cluster barrier / DSMEM handshake ran out
-    DEVERR_WAIT_SPLIT = 1u << 4,    // GEMM: the last K slice of a tile waited too long for the others
     DEVERR_BAD_LAYOUT = 1u << 8,    // decode attention: kv_indptr / kv_len violate the documented layout
     DEVERR_BAD_TOKEN = 1u << 9,     // embedding: token id outside [0, vocab)
     DEVERR_BAD_DST_ROW = 1u << 10,  // KV append: destination row outside the cache

@@ -11,16 +11,16 @@
 //   - N up to 256 x (SM pairs) (18944 on a B200): 256 x 256 tiles over a 2-CTA cluster,
 //     tcgen05.mma.cta_group::2 256 x 256 x 16;
 //   - wider N: 128 x 256 tiles on one CTA, tcgen05.mma.cta_group::1 128 x 256 x 16.
-// In both, the K-block order is ascending (64 at a time).  The pair kernel can also split K into
-// S contiguous slices: slice s of a tile accumulates its K blocks in TMEM like an unsplit
-// tile, slices 0 .. S-2 store fp32 partials, and slice S-1 adds them in slice order,
-// ((P0 + P1) + ...) + P(S-1), before the output rounding.  The slices meet through integer
-// counters; no floating-point atomic is used.  The plan's S is 1 (splits_for); other S run
-// through bi_ctrl_gemm_split.  A row's tile position and the batch size M change which CTA
-// computes the row.  They never change the instructions that produce its bits.  Rows past M
-// are zero-filled by the TMA unit and are never stored.
+// In both, the K-block order is ascending (64 at a time).  The 256 x 256 tiles can also split K
+// into S contiguous slices (the cluster-split kernel): slice s of a tile accumulates its K
+// blocks in TMEM like an unsplit tile, on its own CTA pair of a 2S-CTA cluster, and the pairs
+// add their partials in slice order, ((P0 + P1) + ...) + P(S-1), through distributed shared
+// memory before the output rounding; no floating-point atomic is used.  The plan's S comes from
+// splits_for(N, K); other S run through bi_ctrl_gemm_split.  A row's tile position and the batch
+// size M change which CTA computes the row.  They never change the instructions that produce
+// its bits.  Rows past M are zero-filled by the TMA unit and are never stored.
 //
-// CTA structure (192 threads; in the pair kernel two CTAs per cluster):
+// CTA structure (192 threads; in the pair kernel two CTAs per cluster, 2S in the split kernel):
 //   warp 0      TMA producer.  Pair kernel: 128 rows of A [128 x 64] and 128 columns of W
 //               [64 x 128] per stage, 6-stage ring, completion bytes of both CTAs counted by
 //               the leader.  Single-CTA kernel: A [128 x 64] and W [64 x 256], 4-stage ring.
@@ -536,7 +536,7 @@ struct Bars {
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
-    uint64_t rfull[EPI_WARPS][RING];         // owner: every other slice's piece of this slot has landed
+    uint64_t rfull[EPI_WARPS][RING];         // owner: every lane of every other slice stored its piece
     uint64_t rfree[EPI_WARPS][RING][MAX_S];  // sender: slot r of warp w in slice o's CTA may be refilled
     uint32_t tmem_addr;
     int abort;
@@ -592,7 +592,7 @@ bi_gemm_bf16_cluster_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
         mbar_init(smem_u32(&bars->drain), 1);
         for (int w = 0; w < EPI_WARPS; ++w)
             for (int r = 0; r < cs::RING; ++r) {
-                mbar_init(smem_u32(&bars->rfull[w][r]), 1);
+                mbar_init(smem_u32(&bars->rfull[w][r]), (uint32_t)(32 * (S - 1)));  // every lane of each sender
                 for (int o = 0; o < cs::MAX_S; ++o) mbar_init(smem_u32(&bars->rfree[w][r][o]), 1);
             }
         bars->abort = 0;
@@ -736,11 +736,11 @@ bi_gemm_bf16_cluster_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
                     const uint32_t bar = mapa(rfull0 + (uint32_t)slot * 8u, owner);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        st_async_v4(dst + 16u * i, r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3], bar);
+                        st_cluster_v4(dst + 16u * i, r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+                    mbar_arrive_cluster(bar);  // release: this lane's stores are visible before its arrival
                     continue;
                 }
                 // this slice owns chunk c: wait for the other slices' pieces, add in slice order
-                if (lane == 0) mbar_arrive_expect_tx(rfull0 + (uint32_t)slot * 8u, (uint32_t)((S - 1) * cs::PIECE));
                 const bool full_ok = __all_sync(0xffffffffu, mbar_wait_cluster(rfull0 + (uint32_t)slot * 8u, par, abort));
                 if (!full_ok) {
                     if (lane == 0) fail(err, abort, bi::DEVERR_WAIT_CLUSTER);

@@ -177,11 +177,13 @@ lora_shrink_atomic_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
 //     c, c + clusters, ...; its producer warp keeps one TMA ring streaming across tiles, so a
 //     cluster's second tile loads while its first is being combined.
 //   - Distributed, pushed combine.  Compute warp w owns rows [16w, 16w + 16) of the tile.  When
-//     its chain ends, it stores its fragment of the partial (st.async) straight into the shared
-//     memory of the CTA that combines those rows: CTA d = w * split / 8 combines rows
-//     [128 d / split, 128 (d + 1) / split).  The stores complete bytes on d's receive barrier.
-//     A combiner warp in every CTA then adds its rows' split partials from its own shared memory,
-//     in slice order, and writes t.  Every CTA combines; no CTA reads a peer's shared memory.
+//     its chain ends, it stores its fragment of the partial straight into the shared memory of
+//     the CTA that combines those rows (CTA d = w * split / 8 combines rows
+//     [128 d / split, 128 (d + 1) / split)), and every lane then arrives, with release semantics
+//     at cluster scope, on d's receive barrier: each lane publishes its own stores.  A combiner
+//     warp in every CTA waits for the 8 x 32 arrivals (acquire), adds its rows' split partials
+//     from its own shared memory in slice order, and writes t.  Every CTA combines; no CTA reads
+//     a peer's shared memory.
 //   - Receive buffers rotate (two for r <= 16, one above), and a combiner hands a buffer back to
 //     the senders with a remote arrive once it has read it.
 // Every wait is bounded.  A cluster barrier at the end keeps each CTA's shared memory alive until
@@ -230,7 +232,6 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
     const int kbase = (int)slice * KS;
     const int nchunks = KS / SH_KC;
     const int rows_per = SH_TM / split;  // rows of a tile that each CTA combines
-    constexpr uint32_t RECV_TX = (uint32_t)L::RECV;  // bytes a combiner receives per tile
 
     if (tid == 0) {
         for (int i = 0; i < L::STAGES; ++i) {
@@ -238,7 +239,7 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
             mbar_init(smem_u32(&empty[i]), SO_CWARPS);
         }
         for (int b = 0; b < L::NB; ++b) {
-            mbar_init(smem_u32(&rfull[b]), 1);
+            mbar_init(smem_u32(&rfull[b]), SO_CWARPS * 32);  // every lane of the 8 sending warps
             for (int d = 0; d < SH_MAX_SPLIT; ++d) mbar_init(smem_u32(&rfree[b * SH_MAX_SPLIT + d]), 1);
         }
         *abort = 0;
@@ -283,7 +284,6 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
             const int b = j % L::NB;
             const uint32_t par = (uint32_t)(j / L::NB) & 1u;
-            if (lane == 0) mbar_arrive_expect_tx(smem_u32(&rfull[b]), RECV_TX);
             const bool ok = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&rfull[b]), par, abort));
             if (!ok) {
                 if (lane == 0) atomicOr(err, bi::DEVERR_WAIT_CLUSTER);
@@ -367,14 +367,242 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
 #pragma unroll
             for (int nt = 0; nt < R / 8; ++nt) {
                 const uint32_t col = (uint32_t)(nt * 8 + q * 2) * 4u;
-                st_async_v2(dst + col, acc[nt][0], acc[nt][1], bar);
-                st_async_v2(dst + (uint32_t)(8 * R * 4) + col, acc[nt][2], acc[nt][3], bar);
+                st_cluster_v2(dst + col, acc[nt][0], acc[nt][1]);
+                st_cluster_v2(dst + (uint32_t)(8 * R * 4) + col, acc[nt][2], acc[nt][3]);
             }
+            mbar_arrive_cluster(bar);  // release: this lane's stores above are visible before the arrival
         }
     }
     // no CTA leaves while a peer may still store into its shared memory or signal its barriers
     __syncwarp();
     cluster_sync();
+}
+
+// ------------------------------------------------------------------ shrink on tcgen05 (r = 64)
+// At r = 64 the mma.sync kernel above spends its time feeding the warp-level MMAs from shared
+// memory (every warp reloads the A chunk's fragments for its 16 rows).  This variant keeps the
+// same slices, clusters, TMA ring and on-chip combine, but one thread issues tcgen05.mma
+// (M = 128 rows of x, N = 64, K = 16) straight from the TMA-written tiles into a TMEM
+// accumulator, four warps read it back, and each row's partial is pushed to the CTA that
+// combines it.  Slice s's partial is one fp32 chain over its K slice in 16-deep ascending steps;
+// the combine is the same ((P0 + P1) + ...) + P(split-1).  The tensor core's accumulation is not
+// the warp-level MMA's, so r = 64 results differ from the mma.sync kernel's in the last bits; both
+// are batch-invariant, and parity holds against the oracle.
+constexpr int ST_THREADS = 7 * 32;  // producer, MMA issuer, four TMEM readers, combiner
+
+template <int R>
+struct TcLayout {
+    static_assert(R == 64, "the tcgen05 shrink takes r = 64 (a 128-byte-swizzled N-major B operand)");
+    static constexpr int X_STAGE = SH_TM * SH_KC * 2;  // 16 KB
+    static constexpr int A_STAGE = SH_KC * R * 2;      // 8 KB: one [64 K x 64 r] box
+    static constexpr int STAGE = X_STAGE + A_STAGE;
+    static constexpr int RECV = SH_TM * R * 4;         // one buffer of partials for this CTA's rows
+    static constexpr int BUDGET = 112 * 1024 - 1024 - 256;  // two CTAs per SM
+    static constexpr int STAGES = (BUDGET - RECV) / STAGE;
+    static_assert(STAGES >= 3, "the ring needs at least three stages");
+    static constexpr int RECV_OFF = STAGES * STAGE;
+    static constexpr int BAR_OFF = RECV_OFF + RECV;
+    // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, rfull, rfree[SH_MAX_SPLIT], then
+    // the TMEM address and the abort flag
+    static constexpr int NBARS = 2 * STAGES + 5 + 1 + SH_MAX_SPLIT;
+    static constexpr size_t BYTES = 1024 + (size_t)BAR_OFF + NBARS * 8 + 16;
+    static constexpr uint32_t TMEM_COLS = 2 * R;  // two accumulators
+};
+
+template <int R>
+__global__ void __launch_bounds__(ST_THREADS, 2)
+lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
+                      float* __restrict__ t, int M, int KS, int split, int n_tiles, uint32_t* err) {
+    using L = TcLayout<R>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* recv = reinterpret_cast<float*>(base + L::RECV_OFF);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L::BAR_OFF);
+    uint64_t* empty = full + L::STAGES;
+    uint64_t* tfull = empty + L::STAGES;  // [2]
+    uint64_t* tempty = tfull + 2;         // [2]
+    uint64_t* drain = tempty + 2;
+    uint64_t* rfull = drain + 1;          // every row of every slice for this CTA's rows is stored
+    uint64_t* rfree = rfull + 1;          // [8]: CTA d's receive buffer may be written again
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rfree + SH_MAX_SPLIT);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const uint32_t slice = cluster_ctarank();
+    const int kbase = (int)slice * KS;
+    const int nchunks = KS / SH_KC;
+    const int rows_per = SH_TM / split;
+
+    if (tid == 0) {
+        for (int i = 0; i < L::STAGES; ++i) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&tfull[b]), 1);
+            mbar_init(smem_u32(&tempty[b]), 4);
+        }
+        mbar_init(smem_u32(drain), 1);
+        mbar_init(smem_u32(rfull), SH_TM);  // one arrival per row of the tile, from whichever slice
+        for (int d = 0; d < SH_MAX_SPLIT; ++d) mbar_init(smem_u32(&rfree[d]), 1);
+        *abort = 0;
+        fence_barrier_init();
+        fence_proxy_async_shared();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // every CTA's barriers exist before any signal crosses the cluster
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // x and A may come from the kernel before this one; it may still read t
+    pdl_trigger();
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer: one ring across all tiles
+        if (lane == 0) {
+            prefetch_tmap(&tmX);
+            prefetch_tmap(&tmA);
+            uint32_t it = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
+                for (int c = 0; c < nchunks; ++c, ++it) {
+                    const int st = (int)(it % L::STAGES);
+                    const uint32_t round = it / L::STAGES;
+                    if (!mbar_wait(smem_u32(&empty[st]), (round & 1u) ^ 1u, abort)) {
+                        atomicOr(err, bi::DEVERR_WAIT_TMA);
+                        *abort = 1;
+                        break;
+                    }
+                    uint8_t* sx = base + st * L::STAGE;
+                    const uint32_t fb = smem_u32(&full[st]);
+                    mbar_arrive_expect_tx(fb, L::STAGE);
+                    tma_load_2d(smem_u32(sx), &tmX, kbase + c * SH_KC, tile * SH_TM, fb);
+                    tma_load_2d(smem_u32(sx + L::X_STAGE), &tmA, 0, kbase + c * SH_KC, fb);
+                }
+            }
+            if (*abort) {
+                for (uint32_t i = it > (uint32_t)L::STAGES ? it - L::STAGES : 0u; i < it; ++i)
+                    (void)mbar_wait(smem_u32(&full[i % L::STAGES]), (i / L::STAGES) & 1u, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc_bf16_f32(SH_TM, R, 0, 1);
+            uint32_t it = 0, local = 0;
+            for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x, ++local) {
+                const uint32_t acc = local & 1u, use = local >> 1;
+                if (!mbar_wait(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort)) {
+                    atomicOr(err, bi::DEVERR_WAIT_ACCUM);
+                    *abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * R;
+                for (int c = 0; c < nchunks; ++c, ++it) {
+                    const int st = (int)(it % L::STAGES);
+                    if (!mbar_wait(smem_u32(&full[st]), (it / L::STAGES) & 1u, abort)) {
+                        atomicOr(err, bi::DEVERR_WAIT_FULL);
+                        *abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t xs = smem_u32(base + st * L::STAGE);
+                    const uint32_t as = xs + L::X_STAGE;
+#pragma unroll
+                    for (int k = 0; k < SH_KC / 16; ++k) {
+                        // x: K-major, 128-byte swizzle, 32 bytes per 16-deep step along the row
+                        const uint64_t adesc = make_smem_desc(xs + k * 32, 16, 1024, 2);
+                        // A chunk: N-major (r contiguous), 128-byte swizzle, 16 K-rows of 128 bytes per step
+                        const uint64_t bdesc = make_smem_desc(as + k * 16 * 128, 8192, 1024, 2);
+                        mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (c | k) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(smem_u32(&empty[st]));  // the stage is free once these MMAs have read it
+                }
+                mma_commit(smem_u32(&tfull[acc]));  // this slice's partial of the tile is complete
+            }
+            mma_commit(smem_u32(drain));  // TMEM is released only after every MMA completed
+            (void)mbar_wait(smem_u32(drain), 0u, nullptr);
+        }
+    } else if (warp <= 5) {
+        // ------------------------------------------------ TMEM readers: one row of the partial per lane
+        const int quarter = warp & 3;            // this warp may read TMEM lanes 32*quarter .. +31
+        const int row = quarter * 32 + lane;     // row of the tile
+        const int d = row / rows_per;            // the CTA that combines it
+        const int lrow = row - d * rows_per;
+        const uint32_t dst = mapa(smem_u32(recv) + (uint32_t)((((int)slice * rows_per + lrow) * R) * 4), (uint32_t)d);
+        const uint32_t bar = mapa(smem_u32(rfull), (uint32_t)d);
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+        uint32_t local = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++local) {
+            const uint32_t acc = local & 1u, use = local >> 1;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&tfull[acc]), use & 1u, abort));
+            if (!ok || *abort) {
+                if (lane == 0 && !ok) atomicOr(err, bi::DEVERR_WAIT_ACCUM);
+                *abort = 1;
+                break;
+            }
+            tc_fence_after();
+            uint32_t v[2][32];
+            tmem_ld_32x32b_x32(lane_addr + acc * R, v[0]);
+            tmem_ld_32x32b_x32(lane_addr + acc * R + 32, v[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));  // the accumulator may be reused
+            // d has read what this lane pushed for the previous tile (one receive buffer)
+            if (!mbar_wait_cluster(smem_u32(&rfree[d]), (local & 1u) ^ 1u, abort)) {
+                atomicOr(err, bi::DEVERR_WAIT_CLUSTER);
+                *abort = 1;
+                break;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    st_cluster_v4(dst + (uint32_t)((h * 32 + i) * 4), v[h][i], v[h][i + 1], v[h][i + 2], v[h][i + 3]);
+            mbar_arrive_cluster(bar);  // release: this row is visible before the arrival
+        }
+    } else {
+        // ------------------------------------------------ combiner: this CTA's rows of every tile
+        uint32_t j = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(rfull), j & 1u, abort));
+            if (!ok) {
+                if (lane == 0) atomicOr(err, bi::DEVERR_WAIT_CLUSTER);
+                *abort = 1;
+                break;
+            }
+            const int row0 = tile * SH_TM + (int)slice * rows_per;
+            for (int i = lane; i < rows_per * R / 4; i += 32) {
+                const int row = (4 * i) / R, col = (4 * i) % R;
+                float4 v = *reinterpret_cast<const float4*>(recv + row * R + col);
+                for (int sl = 1; sl < split; ++sl) {  // ((P0 + P1) + P2) + ...: slice order
+                    const float4 p = *reinterpret_cast<const float4*>(recv + (sl * rows_per + row) * R + col);
+                    v.x = __fadd_rn(v.x, p.x);
+                    v.y = __fadd_rn(v.y, p.y);
+                    v.z = __fadd_rn(v.z, p.z);
+                    v.w = __fadd_rn(v.w, p.w);
+                }
+                if (row0 + row < M) *reinterpret_cast<float4*>(t + (size_t)(row0 + row) * R + col) = v;
+            }
+            __syncwarp();
+            if (lane < split) mbar_arrive_cluster(mapa(smem_u32(&rfree[slice]), (uint32_t)lane));
+        }
+    }
+    // no CTA leaves, or frees TMEM, while a peer may still store into it or signal it
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, L::TMEM_COLS);
+    }
 }
 
 // ------------------------------------------------------------------ expand
@@ -633,6 +861,54 @@ int launch_shrink_ordered(const void* x, const void* A, float* t, int64_t M, int
     return bi::launch_status();
 }
 
+template <int R>
+int launch_shrink_tc(const void* x, const void* A, float* t, int64_t M, int64_t K, int split, cudaStream_t s) {
+    using L = TcLayout<R>;
+    uint32_t* err = bi::device_error_word();
+    auto kern = lora_shrink_tc_kernel<R>;
+    if (!err || !set_smem_once(kern, L::BYTES)) return BI_ERR_CUDA;
+    static std::mutex mu;
+    static int fit_cache[64][4];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BI_ERR_CUDA;
+    const int si = split == 1 ? 0 : (split == 2 ? 1 : (split == 4 ? 2 : 3));
+    int fit;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (fit_cache[dev][si] == 0) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(1, (unsigned)split, 1);
+            cfg.blockDim = dim3(ST_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = L::BYTES;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1;
+            attr[0].val.clusterDim.y = (unsigned)split;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return BI_ERR_CUDA;
+            fit_cache[dev][si] = n > 0 ? n : 1;
+        }
+        fit = fit_cache[dev][si];
+    }
+    CUtensorMap tmX, tmA;
+    if (!bi::make_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2,
+                          SH_KC, SH_TM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)R, (uint64_t)K, (uint64_t)R * 2, R,
+                          SH_KC, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BI_ERR_CUDA;
+    const int n_tiles = (int)((M + SH_TM - 1) / SH_TM);
+    const int clusters = n_tiles < fit ? n_tiles : fit;
+    if (bi::launch_pdl(kern, dim3((unsigned)clusters, (unsigned)split), dim3(ST_THREADS), L::BYTES, s,
+                       (unsigned)split, tmX, tmA, t, (int)M, (int)(K / split), (int)split, n_tiles,
+                       err) != cudaSuccess)
+        return BI_ERR_CUDA;
+    return bi::launch_status();
+}
+
 template <bool ATOMIC>
 int shrink_dispatch(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r, int32_t split,
                     cudaStream_t s) {
@@ -641,7 +917,7 @@ int shrink_dispatch(const void* x, const void* A, float* t, int64_t M, int64_t K
             case 8: return launch_shrink_ordered<8>(x, A, t, M, K, split, s);
             case 16: return launch_shrink_ordered<16>(x, A, t, M, K, split, s);
             case 32: return launch_shrink_ordered<32>(x, A, t, M, K, split, s);
-            case 64: return launch_shrink_ordered<64>(x, A, t, M, K, split, s);
+            case 64: return launch_shrink_tc<64>(x, A, t, M, K, split, s);
             default: return BI_ERR_UNSUPPORTED_SHAPE;
         }
     } else {

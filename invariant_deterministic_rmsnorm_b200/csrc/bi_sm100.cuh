@@ -311,12 +311,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
         }
     }
 }
-// 8-byte store into the shared memory of a CTA of this cluster (`addr` from mapa); its bytes count
-// as completed transactions on that CTA's mbarrier `bar` (also a mapa address) once they land.
-__device__ __forceinline__ void st_async_v2(uint32_t addr, float a, float b, uint32_t bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
-                 :: "r"(addr), "f"(a), "f"(b), "r"(bar) : "memory");
-}
 
 }  // namespace sm100
 }  // namespace bi
@@ -333,12 +327,29 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
-// 16-byte store into the shared memory of a CTA of this cluster; its bytes complete transactions on
-// that CTA's mbarrier `bar` (both mapa addresses).
-__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
-                 :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar) : "memory");
+
+}  // namespace sm100
+}  // namespace bi
+
+namespace bi {
+namespace sm100 {
+
+// Plain 8-byte store into the shared memory of a CTA of this cluster (`addr` from mapa).  Pair it
+// with a release arrive by the same thread (mbar_arrive_cluster) to publish it.
+__device__ __forceinline__ void st_cluster_v2(uint32_t addr, float a, float b) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" :: "r"(addr), "f"(a), "f"(b) : "memory");
+}
+
+}  // namespace sm100
+}  // namespace bi
+
+namespace bi {
+namespace sm100 {
+
+// Plain 16-byte store into the shared memory of a CTA of this cluster (`addr` from mapa).
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
 }
 
 }  // namespace sm100
