@@ -712,19 +712,20 @@ def gate_table(device, stream, peaks):
         pt = {key: n, "us": round(ms * 1e3, 2), "achieved": round(ach, 1), "frac": round(ach / peak, 4),
               "gate": gate, "met": bool(ach / peak >= gate)}
         if unit == "GB/s":
-            # context: a device-to-device copy with the same traffic (half read, half written), timed the
-            # same way -- what launch, ramp-up and drain leave of the peak at this size
+            # context: an elementwise copy kernel with the same traffic (half read, half written), timed
+            # the same way -- what launch, ramp-up and drain leave of the peak at this size
             cms = copy_ms(work)
             pt["copy_us"] = round(cms * 1e3, 2)
             pt["frac_of_copy"] = round(cms / ms, 4)
         return pt
 
     def copy_ms(nbytes):
-        half = max(16, (int(nbytes) // 2) // 16 * 16)
+        # an elementwise kernel on the SMs (a graph-captured copy_ would become a copy-engine node)
+        half = max(8, (int(nbytes) // 4) // 8 * 8)  # bf16 elements: half the bytes read, half written
         R = _copies(nbytes)
-        src = [torch.empty(half, dtype=torch.uint8, device=device).fill_(1) for _ in range(R)]
-        dst = [torch.empty(half, dtype=torch.uint8, device=device) for _ in range(R)]
-        ms = _time_graph([lambda j=j: dst[j].copy_(src[j], non_blocking=True) for j in range(R)], stream)
+        src = [torch.ones(half, dtype=torch.bfloat16, device=device) for _ in range(R)]
+        dst = [torch.empty(half, dtype=torch.bfloat16, device=device) for _ in range(R)]
+        ms = _time_graph([lambda j=j: torch.mul(src[j], 1.0, out=dst[j]) for j in range(R)], stream)
         del src, dst
         return ms
 
@@ -1008,7 +1009,13 @@ def run_sweep(args):
             t_uns = _time_graph([lambda j=j: B.bi_lora_shrink(xs[j], A_l, t=t, split_k=1, stream=stream)
                                  for j in range(R)], stream)
             t_exp = _time_graph([lambda j=j: B.bi_lora_expand(t, B_l, ys[j], stream=stream) for j in range(R)], stream)
-            table.append({"M": M, "shrink_gbs": round(by_s / (t_det / 1e3), 1),
+            extra = {}
+            if r == 64:  # the tcgen05 study kernel beside the plan's mma.sync kernel
+                t_tc = _time_graph([lambda j=j: B.bi_ctrl_lora_shrink_tc(xs[j], A_l, t=t, split_k=8, stream=stream)
+                                    for j in range(R)], stream)
+                extra = {"shrink_tc_us": round(t_tc * 1e3, 2),
+                         "shrink_tc_frac": round(by_s / (t_tc / 1e3) / peaks["hbm_gbs"], 3)}
+            table.append({**extra, "M": M, "shrink_gbs": round(by_s / (t_det / 1e3), 1),
                           "shrink_frac": round(by_s / (t_det / 1e3) / peaks["hbm_gbs"], 3),
                           "shrink_us": round(t_det * 1e3, 2), "atomic_us": round(t_atom * 1e3, 2),
                           "unsplit_us": round(t_uns * 1e3, 2), "expand_gbs": round(by_e / (t_exp / 1e3), 1),
@@ -1295,6 +1302,22 @@ def run_contrast(args):
     print(json.dumps(contrast_composition(dec["bi"], dec["fast"], prompts, filler, BF, probe_steps)), flush=True)
 
 
+def run_one_op(args):
+    """A few launches of one op of the step, at the step's configuration, on rotating inputs: the
+    target of a one-kernel profiler capture (the other ops' inputs are built but not launched)."""
+    import torch
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        ops, _ = build_ops(device, stream, args.attn_batch)
+        op = next(o for o in ops if o["name"] == args.op)
+        for k in range(args.launches):
+            op["launch"](k)
+    torch.cuda.synchronize()
+    print(json.dumps({"op": args.op, "launches": args.launches, "desc": op["desc"]}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1320,6 +1343,11 @@ def main():
                     help="position-invariant scheduling (fixed-shape decode over batch-dependent fast kernels) "
                          "against the batch-invariant decoder (one GPU)")
     ap.add_argument("--contrast-batches", type=int, nargs="+", default=[1, 8, 32, 128])
+    ap.add_argument("--op", default=None,
+                    choices=["rmsnorm", "gemm_qkv", "lora_shrink", "lora_expand", "gemm_up", "gemm_down",
+                             "decode_attn"],
+                    help="launch only this op of the step, --launches times, and exit (for profiler captures)")
+    ap.add_argument("--launches", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -1335,6 +1363,9 @@ def main():
         return
     if args.contrast:
         run_contrast(args)
+        return
+    if args.op:
+        run_one_op(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -60,6 +60,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_lora_shrink": ([P, P, P, I64, I64, I32, I32, P, Z, P], C),
         "bi_lora_expand": ([P, P, P, I64, I32, I64, I64, F, C, P], C),
         "bi_ctrl_lora_shrink_atomic": ([P, P, P, I64, I64, I32, I32, P], C),
+        "bi_ctrl_lora_shrink_tc": ([P, P, P, I64, I64, I32, I32, P], C),
         "bi_decode_attn_workspace_size": ([I64, I32, I32, I32], Z),
         "bi_decode_attn": ([P, P, P, P, P, I32, I64, I32, I32, I32, F, I32, P, C, P, Z, P], C),
         "bi_ctrl_rmsnorm_split": ([P, P, P, I64, I64, I64, I64, F, C, C, P], C),
@@ -215,6 +216,20 @@ def bi_ctrl_lora_shrink_atomic(x: torch.Tensor, A: torch.Tensor, t: torch.Tensor
         t = torch.empty((M, r), dtype=torch.float32, device=x.device)
     st = library().bi_ctrl_lora_shrink_atomic(_ptr(x), _ptr(A), _ptr(t), M, K, r, split_k, _stream(stream))
     _check("bi_ctrl_lora_shrink_atomic", st)
+    return t
+
+
+def bi_ctrl_lora_shrink_tc(x: torch.Tensor, A: torch.Tensor, t: torch.Tensor | None = None, split_k: int = 8,
+                           stream=None) -> torch.Tensor:
+    """The r = 64 shrink on tcgen05 (the study behind keeping mma.sync in the plan)."""
+    _bf16_2d(x, "x")
+    _bf16_2d(A, "A")
+    M, K = x.shape
+    r = A.shape[1]
+    if t is None:
+        t = torch.empty((M, r), dtype=torch.float32, device=x.device)
+    st = library().bi_ctrl_lora_shrink_tc(_ptr(x), _ptr(A), _ptr(t), M, K, r, split_k, _stream(stream))
+    _check("bi_ctrl_lora_shrink_tc", st)
     return t
 
 

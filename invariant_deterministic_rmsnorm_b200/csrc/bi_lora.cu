@@ -379,8 +379,10 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
 }
 
 // ------------------------------------------------------------------ shrink on tcgen05 (r = 64)
-// At r = 64 the mma.sync kernel above spends its time feeding the warp-level MMAs from shared
-// memory (every warp reloads the A chunk's fragments for its 16 rows).  This variant keeps the
+// The study of the tcgen05 alternative for r = 64 (bi_ctrl_lora_shrink_tc; the plan keeps the
+// mma.sync kernel above, which measured faster at the large batches).  At r = 64 the mma.sync
+// kernel feeds its warp-level MMAs from shared memory (every warp reloads the A chunk's
+// fragments for its 16 rows).  This variant keeps the
 // same slices, clusters, TMA ring and on-chip combine, but one thread issues tcgen05.mma
 // (M = 128 rows of x, N = 64, K = 16) straight from the TMA-written tiles into a TMEM
 // accumulator, four warps read it back, and each row's partial is pushed to the CTA that
@@ -917,7 +919,7 @@ int shrink_dispatch(const void* x, const void* A, float* t, int64_t M, int64_t K
             case 8: return launch_shrink_ordered<8>(x, A, t, M, K, split, s);
             case 16: return launch_shrink_ordered<16>(x, A, t, M, K, split, s);
             case 32: return launch_shrink_ordered<32>(x, A, t, M, K, split, s);
-            case 64: return launch_shrink_tc<64>(x, A, t, M, K, split, s);
+            case 64: return launch_shrink_ordered<64>(x, A, t, M, K, split, s);
             default: return BI_ERR_UNSUPPORTED_SHAPE;
         }
     } else {
@@ -970,6 +972,15 @@ BI_API int bi_lora_shrink(const void* x, const void* A, float* t, int64_t M, int
     if (c < 0) return BI_OK;
     if (c != BI_OK) return c;
     return shrink_dispatch<false>(x, A, t, M, K, r, split_k, bi::as_stream(stream));
+}
+
+BI_API int bi_ctrl_lora_shrink_tc(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r,
+                                  int32_t split_k, void* stream) {
+    const int c = shrink_checks(x, A, t, M, K, r, split_k);
+    if (c < 0) return BI_OK;
+    if (c != BI_OK) return c;
+    if (r != 64) return BI_ERR_UNSUPPORTED_SHAPE;
+    return launch_shrink_tc<64>(x, A, t, M, K, split_k, bi::as_stream(stream));
 }
 
 BI_API int bi_ctrl_lora_shrink_atomic(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r,

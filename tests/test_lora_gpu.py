@@ -204,3 +204,26 @@ def test_expand_batch_invariance(r):
             for i, w in enumerate(pos):
                 bad += int(not torch.equal(yb[int(w)].view(torch.int16), solo[i][0]))
     assert bad == 0
+
+
+# ------------------------------------------------------------------ the r = 64 tcgen05 study kernel
+@pytest.mark.parametrize("M", [1, 130, 4096])
+def test_shrink_tc_r64(M):
+    """bi_ctrl_lora_shrink_tc: small-integer operands exact (every partial sum is an integer below
+    2^24), random operands within the shrink's tolerance of the oracle's split-8 sum, rows
+    independent of the batch, and replays identical."""
+    xi = inputs.small_int_bf16(66, (M, K))
+    Ai = inputs.small_int_bf16(67, (K, 64))
+    t = host(binding.bi_ctrl_lora_shrink_tc(dev(xi), dev(Ai)))
+    assert np.array_equal(t.astype(np.float64), oracle.lora_shrink(xi, Ai))
+    x, A, _, _ = inputs.lora_case(M, 64)
+    xd, Ad = dev(x), dev(A)
+    t = binding.bi_ctrl_lora_shrink_tc(xd, Ad)
+    ref = oracle_rows(oracle.lora_shrink_split, x, A, 8)
+    err = rel_frobenius(host(t), ref)
+    assert err <= 2e-3 and err <= 1e-4, err
+    for r_ in sorted({0, M // 2, M - 1}):
+        solo = binding.bi_ctrl_lora_shrink_tc(xd[r_:r_ + 1].contiguous(), Ad)
+        assert torch.equal(solo[0].view(torch.int32), t[r_].view(torch.int32))
+    for _ in range(5):
+        assert torch.equal(binding.bi_ctrl_lora_shrink_tc(xd, Ad).view(torch.int32), t.view(torch.int32))
