@@ -262,8 +262,7 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                         mma_m16n8k16_bf16(acc, a, qf[kk]);
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+                release_stage(smem_u32(&empty[st]), lane);
                 ++it;
             }
             const int gg = lane >> 2, hq = (lane & 3) * 2;
@@ -361,8 +360,7 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     mma_m16n8k16_bf16(oacc_lo, a, bl);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+            release_stage(smem_u32(&empty[st]), lane);
             ++it;
         }
 

@@ -143,8 +143,7 @@ lora_shrink_atomic_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
                     mma_m16n8k16_bf16(acc[nt], a, b);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+            release_stage(smem_u32(&empty[st]), lane);
         }
         // every warp is done reading the stages before any partial overwrites them
         asm volatile("bar.sync 1, %0;" :: "n"(SH_CWARPS * 32) : "memory");
@@ -348,8 +347,7 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
                         mma_m16n8k16_bf16(acc[nt], a, bf);
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+                release_stage(smem_u32(&empty[st]), lane);
             }
             if (!ok) break;
             const int b = j % L::NB;

@@ -44,6 +44,17 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
 }
 
+// A warp hands a TMA-filled ring stage back to its producer after reading it with ordinary
+// shared-memory loads (ld.shared, ldmatrix).  Those reads are generic-proxy accesses and the
+// refill is an async-proxy write, so a proxy fence has to order them: without it the arrival
+// may become visible while the warp's last loads are still in flight, and the refill then
+// overwrites the first rows of the stage under them.  Every lane fences; lane 0 arrives.
+__device__ __forceinline__ void release_stage(uint32_t bar, int lane) {
+    fence_proxy_async_shared();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ bool mbar_test_parity(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
