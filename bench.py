@@ -458,6 +458,7 @@ def run_ours(args, rank, world, local_rank):
         return None
     # rank 0 alone, after the last collective: the gate points at every batch size they apply to
     gates = gate_table(device, stream, load_peaks()[0]) if not args.no_gates else None
+    follow_on = next_rows(device, load_peaks()[0]) if not args.no_next else None
 
     peaks, peak_src = load_peaks()
     # Back-to-back time of each op's kernel at the step's own configuration (from the gate table:
@@ -550,6 +551,7 @@ def run_ours(args, rank, world, local_rank):
         "bi_violations": viol,
         "invariance_tax": tax,
         "gates": gates,
+        "next_rows": follow_on,
         "clocks": clocks, "clocks_step_without_op_events": clocks_step, "cpu_baseline": cpu,
         # what the result was produced with (GPU, driver, CUDA, torch, commit)
         "pin": harness_pin(),
@@ -1069,14 +1071,7 @@ def run_replay_study(args):
             x = _to_dev(inputs.rows(inputs.SEED_X, M, HIDDEN, "bf16"), device)
             res = {"M": M}
             for name, fn in (("atomic", B.bi_ctrl_lora_shrink_atomic), ("ordered", B.bi_lora_shrink)):
-                first = fn(x, A_l, split_k=8).clone()
-                diff_runs, diff_elems = 0, 0
-                for _ in range(n - 1):
-                    t = fn(x, A_l, split_k=8)
-                    ne = int((t.view(torch.int32) != first.view(torch.int32)).sum())
-                    diff_runs += int(ne > 0)
-                    diff_elems += ne
-                torch.cuda.synchronize()
+                diff_runs, diff_elems = _replay_differing(fn, x, A_l, n)
                 res[f"{name}_replays_differing_pct"] = round(100.0 * diff_runs / (n - 1), 2)
                 res[f"{name}_elements_differing_pct"] = round(100.0 * diff_elems / ((n - 1) * M * r), 3)
             rows.append(res)
@@ -1099,6 +1094,56 @@ def _decoder_flops(shape, lens_new, lens_total):
     return proj, attn
 
 
+def decoder_point(dec, shape, prompts, B, steps, warmup, peaks):
+    """Prefill of the first B prompts (the second of two passes is timed; the first also does the
+    per-device set-up), then `steps` greedy decode steps replayed from one CUDA graph after
+    `warmup` untimed replays.  Returns the prefill and decode records."""
+    import torch
+    weight_bytes = 2 * sum(r * c for name, r, c, _, _ in shape.matrices() if name != "embed")
+    kv_row_bytes = 2 * 2 * shape.kv_heads * shape.head_dim * shape.layers  # K and V, all layers
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    slots = list(range(B))
+    lens = np.array([len(p) for p in prompts[:B]])
+    prefill_ms = []
+    for _ in range(2):
+        dec.reset()
+        torch.cuda.synchronize()
+        e0, e1 = ev(), ev()
+        e0.record()
+        dec.forward(slots, prompts[:B], "prefill")
+        e1.record()
+        torch.cuda.synchronize()
+        prefill_ms.append(e0.elapsed_time(e1))
+    T = int(lens.sum())
+    proj, attn = _decoder_flops(shape, lens, lens)
+    ms = prefill_ms[-1]
+    pre = {"phase": "prefill", "requests": B, "tokens": T, "ms": round(ms, 2),
+           "tokens_per_s": round(T / ms * 1e3), "model_tflops": round((proj + attn) / ms / 1e9, 1),
+           "frac_of_bf16_peak": round((proj + attn) / ms / 1e9 / peaks["bf16_tflops"], 3),
+           "attn_share_of_flops": round(attn / (proj + attn), 3)}
+    g = dec.decode_graph(slots)
+    for _ in range(warmup):
+        g.replay()
+    ctx = dec.length[slots].copy()
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    kv_read = kv_row_bytes * float(np.sum(ctx + 0.5 * (steps + 1)))  # mean context over the timed steps
+    step_bytes = weight_bytes + B * 2 * shape.hidden + kv_read
+    dec_rec = {"phase": "decode", "requests": B, "steps": steps, "ms_per_step": round(ms, 4),
+               "tokens_per_s": round(B / ms * 1e3), "mean_context": round(float(np.mean(ctx)) + steps / 2, 1),
+               "hbm_gbs": round(step_bytes / ms / 1e6, 1),
+               "frac_of_hbm": round(step_bytes / ms / 1e6 / peaks["hbm_gbs"], 3),
+               "bytes_per_step": int(step_bytes)}
+    return pre, dec_rec
+
+
 def run_decoder(args):
     """The 4-layer Llama-3-8B-shaped decoder built from the batch-invariant kernels: prefill
     throughput, and greedy decode steps replayed from a CUDA graph, at several batch sizes.
@@ -1115,50 +1160,68 @@ def run_decoder(args):
     dec = Decoder(shape, w, max_seqs=n_max, max_len=2048 + 2 * steps + 8 + args.warmup)
     all_lens = inputs.prompt_lengths(n_max)
     prompts = [inputs.prompt(i, int(n), shape.vocab) for i, n in enumerate(all_lens)]
-    weight_bytes = 2 * sum(r * c for name, r, c, _, _ in shape.matrices() if name != "embed")
-    kv_row_bytes = 2 * 2 * shape.kv_heads * shape.head_dim * shape.layers  # K and V, all layers
-    ev = lambda: torch.cuda.Event(enable_timing=True)
     for B in args.decoder_batches:
-        slots, lens = list(range(B)), all_lens[:B]
-        # prefill (the first pass also does the per-device set-up; time the second)
-        prefill_ms = []
-        for _ in range(2):
-            dec.reset()
-            torch.cuda.synchronize()
-            e0, e1 = ev(), ev()
-            e0.record()
-            dec.forward(slots, prompts[:B], "prefill")
-            e1.record()
-            torch.cuda.synchronize()
-            prefill_ms.append(e0.elapsed_time(e1))
-        T = int(lens.sum())
-        proj, attn = _decoder_flops(shape, lens, lens)
-        ms = prefill_ms[-1]
-        print(json.dumps({"phase": "prefill", "requests": B, "tokens": T, "ms": round(ms, 2),
-                          "tokens_per_s": round(T / ms * 1e3), "model_tflops": round((proj + attn) / ms / 1e9, 1),
-                          "frac_of_bf16_peak": round((proj + attn) / ms / 1e9 / peaks["bf16_tflops"], 3),
-                          "attn_share_of_flops": round(attn / (proj + attn), 3)}), flush=True)
-        # decode: greedy steps replayed from one graph; the timed replays follow `warmup` untimed ones
-        g = dec.decode_graph(slots)
-        for _ in range(args.warmup):
-            g.replay()
-        ctx = dec.length[slots].copy()
-        torch.cuda.synchronize()
-        e0, e1 = ev(), ev()
-        e0.record()
-        for _ in range(steps):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / steps
-        kv_read = kv_row_bytes * float(np.sum(ctx + 0.5 * (steps + 1)))  # mean context over the timed steps
-        step_bytes = weight_bytes + B * 2 * shape.hidden + kv_read
-        print(json.dumps({"phase": "decode", "requests": B, "steps": steps, "ms_per_step": round(ms, 4),
-                          "tokens_per_s": round(B / ms * 1e3), "mean_context": round(float(np.mean(ctx)) + steps / 2, 1),
-                          "hbm_gbs": round(step_bytes / ms / 1e6, 1),
-                          "frac_of_hbm": round(step_bytes / ms / 1e6 / peaks["hbm_gbs"], 3),
-                          "bytes_per_step": int(step_bytes)}), flush=True)
-        del g
+        for rec in decoder_point(dec, shape, prompts, B, steps, args.warmup, peaks):
+            print(json.dumps(rec), flush=True)
+
+
+def _replay_differing(fn, x, A, n):
+    """Launches n shrinks of identical inputs; returns (replays whose output differs in any bit
+    from the first, output elements differing summed over the replays)."""
+    import torch
+    first = fn(x, A, split_k=8).clone()
+    runs, elems = 0, 0
+    for _ in range(n - 1):
+        t = fn(x, A, split_k=8)
+        ne = int((t.view(torch.int32) != first.view(torch.int32)).sum())
+        runs += int(ne > 0)
+        elems += ne
+    torch.cuda.synchronize()
+    return runs, elems
+
+
+def next_rows(device, peaks, replays=20, probe_steps=4):
+    """Compact measurements of the follow-on rows, for the bench line (rank 0, outside the timed
+    region): the replay study at M = 4096, and the 4-layer decoder at 8 requests (prefill and
+    graph-replayed decode throughput, and whether a probe's logits are bitwise equal alone and
+    inside the batch at the prefill and each of `probe_steps` greedy steps)."""
+    import torch
+    from invariant_deterministic_rmsnorm_b200 import binding as B
+    from invariant_deterministic_rmsnorm_b200.decoder import Decoder
+    out = {"replay_study": {}}
+    M = 4096
+    x = _to_dev(inputs.rows(inputs.SEED_X, M, HIDDEN, "bf16"), device)
+    for r in (16, 64):
+        A_l = _to_dev(inputs.normal_bf16(inputs.SEED_WEIGHTS + 20, (HIDDEN, r), 0.0, 0.02), device)
+        row = {"replays": replays}
+        for name, fn in (("atomic", B.bi_ctrl_lora_shrink_atomic), ("ordered", B.bi_lora_shrink)):
+            runs, elems = _replay_differing(fn, x, A_l, replays)
+            row[f"{name}_replays_differing_pct"] = round(100.0 * runs / (replays - 1), 2)
+            row[f"{name}_elements_differing_pct"] = round(100.0 * elems / ((replays - 1) * M * r), 3)
+        out["replay_study"][f"r={r},M={M},split_k=8"] = row
+    del x
+    shape = inputs.LLAMA3_8B_4L
+    w = inputs.decoder_weights_device(shape, device=device)
+    nb = 8
+    lens = inputs.prompt_lengths(nb)
+    prompts = [inputs.prompt(i, int(n), shape.vocab) for i, n in enumerate(lens)]
+    dec = Decoder(shape, w, max_seqs=nb, max_len=2048 + 2 * probe_steps + 16)
+    pre, dec_rec = decoder_point(dec, shape, prompts, nb, 8, 3, peaks)
+    # the probe (prompt 0) alone, then at a seeded random position among the other seven
+    dec.reset()
+    solo, _ = dec.generate([0], [prompts[0]], probe_steps)
+    at = int(np.random.default_rng(inputs.SEED_POSITIONS).integers(1, nb))
+    order = list(range(1, nb))
+    order.insert(at, 0)
+    dec.reset()
+    batch, _ = dec.generate(list(range(nb)), [prompts[i] for i in order], probe_steps, keep=[at])
+    equal = all(np.array_equal(a.view(np.uint32), b.view(np.uint32)) for a, b in zip(solo[0], batch[0]))
+    out["decoder_4layer"] = {"prefill": pre, "decode": dec_rec,
+                             "probe_bitwise_alone_vs_batch": {"batch": nb, "position": at,
+                                                              "steps_compared": probe_steps + 1, "equal": equal}}
+    del dec, w
+    torch.cuda.empty_cache()
+    return out
 
 
 class FastOps:
@@ -1328,6 +1391,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-tax", action="store_true", help="skip the invariance-tax comparison")
     ap.add_argument("--no-gates", action="store_true", help="skip the per-batch-size gate table")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the replay-study and decoder measurements that follow the step")
     ap.add_argument("--replay-study", action="store_true",
                     help="identical-input replay study of the atomic vs ordered split-K shrink (one GPU)")
     ap.add_argument("--replays", type=int, default=200)

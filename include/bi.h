@@ -213,9 +213,15 @@ int bi_lora_expand(const float* t, const void* B, void* y, int64_t M, int32_t r,
  * with s_j = scale * q . k_j (bf16 products, fp32 sums over fixed trees).  The chunks are
  * merged in order c = 0, 1, ... with an fp32 log-sum-exp rescale, and out = o / l.
  *
- * Layout violations that only the device can see (kv_indptr not chunk-aligned, kv_len
- * out of range, kv_indptr[b + 1] > total_tokens) set bit 0x100 of the device error word.
- * The affected rows of out are then left unwritten; the other rows are computed as usual.
+ * Layout violations that only the device can see (kv_indptr negative or not chunk-aligned,
+ * kv_len out of range, kv_indptr[b + 1] > total_tokens) set bit 0x100 of the device error
+ * word.  The affected rows of out are then left unwritten; the other rows are computed as
+ * usual.  A decreasing kv_indptr (sequences that overlap) also sets bit 0x100 and voids the
+ * whole call: no chunk is computed and out holds no result.
+ *
+ * Work split: the live chunks of the batch (ceil(kv_len[b] / 256) per sequence), not the
+ * cache's capacity, are divided among the persistent CTAs, so a few requests in a large
+ * cache still use every SM.  Which CTA computes a chunk never changes its arithmetic.
  */
 size_t bi_decode_attn_workspace_size(int64_t total_tokens, int32_t Hq, int32_t head_dim, int32_t chunk);
 int bi_decode_attn(const void* q, const void* k, const void* v, const int32_t* kv_indptr, const int32_t* kv_len,

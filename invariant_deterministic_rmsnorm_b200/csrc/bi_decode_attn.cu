@@ -9,16 +9,18 @@
 // a multiple of the chunk size, so every request's chunks start at its own token 0 and
 // never depend on its neighbours.  Query head h reads kv head h / (Hq / Hkv).
 //
-// Phase 1 (one CTA per (chunk slot, kv head)).  Slot s covers packed tokens
-// [s*256, s*256 + 256).  The CTA finds the sequence that owns the slot.  Its tokens
-// [c*256, min(c*256 + 256, L)) are chunk c of that sequence.  The CTA computes, for the
-// group's query heads:
+// Phase 1 (persistent CTAs over the live work items (sequence, chunk, kv head)).  Chunk c of
+// sequence b is its tokens [c*256, min(c*256 + 256, L)).  The items are counted on the device
+// from kv_indptr and kv_len and cut into one contiguous range per CTA, so a small batch in a
+// large cache still spreads over every SM.  For each item the CTA computes, for the group's
+// query heads:
 //     s_j = scale * q . k_j          (mma.sync m16n8k16: bf16 products, fp32 accumulate)
 //     m_c = max_j s_j                (exact; order-free)
 //     p_j = exp(s_j - m_c),  l_c = sum_j p_j     (fixed shuffle / shared-memory trees)
 //     o_c = sum_j p_j v_j            (fp32 FMAs, fixed token order per thread, fixed tree)
-// and stores (o_c, m_c, l_c) to the workspace.  K and V reach shared memory through TMA,
-// 128B-swizzled.  V reuses K's buffer once the scores are done.
+// and stores (o_c, m_c, l_c) to the workspace row of cache slot kv_indptr[b] / 256 + c.  K and
+// V reach shared memory through TMA, 128B-swizzled.  V reuses K's buffer once the scores are
+// done.
 //
 // Phase 2 (one warp per (sequence, query head)) merges chunks c = 0, 1, ... in order:
 //     m' = max(m, m_c);  l = l e^(m - m') + l_c e^(m_c - m');  o = o e^(m - m') + o_c e^(m_c - m')
@@ -69,70 +71,104 @@ __device__ __forceinline__ uint32_t kv_addr(uint32_t stage, int j, int d) {
 
 __device__ __forceinline__ void compute_barrier() { asm volatile("bar.sync 1, %0;" :: "n"(CTHREADS) : "memory"); }
 
-struct Item {
-    int b;       // sequence
-    int c;       // chunk of that sequence
-    int n_tok;   // live tokens in the chunk (0: nothing to do)
-    int64_t tok0;
-};
-
-// Remembers the sequence found for the previous slot; slots of one CTA increase, so the
-// next slot usually belongs to the same sequence and needs no memory access at all.
-struct SeqCache {
-    int b = -1;
-    int64_t lo_tok = 0, hi_tok = 0;  // the sequence's tokens [lo_tok, hi_tok) of the packed buffer
-    int len = 0;
-};
-
-// The (sequence, chunk) that owns CH-token slot `slot` of the packed cache.
+// Live chunks of sequence b: ceil(len / CH) when its layout is valid, else 0 and *bad.  A
+// sequence whose capacity reaches past the cache's T tokens is refused whole, so that the merge
+// never reads a slot this phase did not write.
 template <int CH>
-__device__ __forceinline__ Item item_of(int slot, const int32_t* __restrict__ kv_indptr,
-                                        const int32_t* __restrict__ kv_len, int B, int64_t T, bool& bad,
-                                        SeqCache& sc) {
-    Item it{0, 0, 0, (int64_t)slot * CH};
-    bad = false;
-    int lo;
-    if (sc.b >= 0 && it.tok0 >= sc.lo_tok && it.tok0 < sc.hi_tok) {
-        lo = sc.b;
-    } else {
-        if (it.tok0 < kv_indptr[0] || it.tok0 >= kv_indptr[B]) return it;
-        lo = 0;
-        int hi = B;  // the last b with kv_indptr[b] <= tok0
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (kv_indptr[mid] <= it.tok0) lo = mid; else hi = mid;
-        }
-        sc.b = lo;
-        sc.lo_tok = kv_indptr[lo];
-        sc.hi_tok = kv_indptr[lo + 1];
-        sc.len = kv_len[lo];
-    }
-    const int64_t sbase = sc.lo_tok;
-    const int len = sc.len;
-    const int64_t cap = sc.hi_tok - sbase;
-    // a sequence whose capacity reaches past the cache's T tokens is refused whole, so that the
-    // merge never reads a slot this phase did not write
-    if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap || sc.hi_tok > T) {
-        bad = (it.tok0 - sbase) < CH;  // report once per sequence
-        return it;
-    }
-    it.b = lo;
-    it.c = (int)((it.tok0 - sbase) / CH);
-    it.n_tok = max(0, min(CH, len - it.c * CH));
-    return it;
+__device__ __forceinline__ int live_chunks(const int32_t* __restrict__ kv_indptr, const int32_t* __restrict__ kv_len,
+                                           int b, int64_t T, bool* bad) {
+    const int64_t lo = kv_indptr[b], hi = kv_indptr[b + 1];
+    const int len = kv_len[b];
+    *bad = lo < 0 || (lo % CHUNK) != 0 || len <= 0 || (int64_t)len > hi - lo || hi > T;
+    return *bad ? 0 : (len + CH - 1) / CH;
 }
 
-// Phase 1, persistent: CTA i handles a contiguous range of work items; item w = (slot w / Hkv,
-// kv head w % Hkv), so consecutive items share a slot and usually a sequence.
+// Block-wide sums and scans of 64-bit counts (every thread of the block calls them).
+__device__ __forceinline__ int64_t block_sum(int64_t v, int64_t* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    __syncthreads();  // the scratch may still be read by a previous call
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    int64_t t = 0;
+    for (int w = 0; w < nw; ++w) t += scratch[w];
+    return t;
+}
+// inclusive prefix of v over the threads in order; *total is the block's sum
+__device__ __forceinline__ int64_t block_scan(int64_t v, int64_t* scratch, int64_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int64_t x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    __syncthreads();
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    int64_t before = 0, t = 0;
+    for (int w = 0; w < nw; ++w) {
+        if (w < warp) before += scratch[w];
+        t += scratch[w];
+    }
+    *total = t;
+    return before + x;
+}
+
+// Walks a CTA's contiguous range of work items in order.  Item order: sequences in order, the
+// live chunks of each in order, the kv heads of each chunk in order.  Empty and invalid
+// sequences hold no items.  Which CTA computes an item never changes how it is computed.
+template <int CH>
+struct WorkCursor {
+    const int32_t* kv_indptr;
+    const int32_t* kv_len;
+    int B;
+    int64_t T;
+    int Hkv;
+    int b, c, g, nc, len;
+    int64_t lo;
+
+    __device__ __forceinline__ void load() {
+        bool bad;
+        nc = live_chunks<CH>(kv_indptr, kv_len, b, T, &bad);
+        lo = kv_indptr[b];
+        len = kv_len[b];
+    }
+    __device__ __forceinline__ void start(int b0, int c0, int g0) {
+        b = b0;
+        c = c0;
+        g = g0;
+        load();
+    }
+    __device__ __forceinline__ int64_t tok0() const { return lo + (int64_t)c * CH; }
+    __device__ __forceinline__ int n_tok() const { return min(CH, len - c * CH); }
+    __device__ __forceinline__ void next() {
+        if (++g < Hkv) return;
+        g = 0;
+        if (++c < nc) return;
+        c = 0;
+        do {
+            if (++b >= B) return;
+            load();
+        } while (nc == 0);
+    }
+};
+
+// Phase 1, persistent: the batch's live work items, (sequence, chunk, kv head) in that order,
+// are cut into one contiguous range per CTA.  Every CTA counts them itself from kv_indptr and
+// kv_len, so the cut follows the tokens the batch holds, not the capacity of the cache.
 // A producer warp streams each item's K sub-blocks, then its V sub-blocks, through an NSTAGES ring;
 // eight compute warps consume them in the same order.
 template <int G, int CH>
 __global__ void __launch_bounds__(THREADS, 2)
 decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ kv_indptr,
-                         const int32_t* __restrict__ kv_len, int B, int64_t T, int Hq, int Hkv, int n_items,
+                         const int32_t* __restrict__ kv_len, int B, int64_t T, int Hq, int Hkv,
                          float scale, float* __restrict__ o_part, float* __restrict__ ml_part, uint32_t* err) {
     using L = AttnLayout<G>;
+    __shared__ int64_t s_scan[THREADS / 32];
+    __shared__ int s_first[2];  // sequence and chunk of this CTA's first item
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* sS = reinterpret_cast<float*>(base + L::S_OFF);
@@ -146,10 +182,6 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t stage0 = smem_u32(base);
-    const int per_cta = (n_items + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int w_begin = (int)blockIdx.x * per_cta;
-    const int w_end = min(n_items, w_begin + per_cta);
-
     if (tid == 0) {
         for (int i = 0; i < NSTAGES; ++i) {
             mbar_init(smem_u32(&full[i]), 1);
@@ -163,20 +195,59 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     pdl_wait();  // q, the cache and the index arrays may come from the kernels just before this one
     pdl_trigger();
 
+    // ---- this CTA's range of the live work items
+    // live chunks of every sequence; a decreasing kv_indptr (overlapping sequences) is refused
+    int64_t mine = 0;
+    int nc_mine = 0;  // sequence tid's live chunks (used when the batch fits one pass)
+    bool order_ok = true;
+    for (int b = tid; b < B; b += THREADS) {
+        bool bad;
+        const int nc = live_chunks<CH>(kv_indptr, kv_len, b, T, &bad);
+        if (bad && blockIdx.x == 0) atomicOr(err, DEVERR_BAD_LAYOUT);
+        order_ok = order_ok && kv_indptr[b + 1] >= kv_indptr[b];
+        mine += nc;
+        if (b == tid) nc_mine = nc;
+    }
+    const bool ordered = __syncthreads_and(order_ok) != 0;
+    if (!ordered && blockIdx.x == 0 && tid == 0) atomicOr(err, DEVERR_BAD_LAYOUT);
+    const int64_t n_items = ordered ? block_sum(mine, s_scan) * Hkv : 0;
+    const int64_t per_cta = (n_items + gridDim.x - 1) / gridDim.x;
+    const int64_t w_begin = min(n_items, (int64_t)blockIdx.x * per_cta);
+    const int64_t w_end = min(n_items, w_begin + per_cta);
+    if (w_begin < w_end) {  // uniform across the CTA
+        const int64_t j0 = w_begin / Hkv;  // the first item's place among the live chunks
+        int64_t before = 0;                // live chunks of the sequences before this pass
+        for (int t0 = 0; t0 < B; t0 += THREADS) {
+            const int b = t0 + tid;
+            int nc = nc_mine;
+            if (t0 != 0) {
+                bool bad;
+                nc = b < B ? live_chunks<CH>(kv_indptr, kv_len, b, T, &bad) : 0;
+            }
+            int64_t pass_total;
+            const int64_t excl = before + block_scan(nc, s_scan, &pass_total) - nc;
+            if (nc > 0 && excl <= j0 && j0 < excl + nc) {
+                s_first[0] = b;
+                s_first[1] = (int)(j0 - excl);
+            }
+            before += pass_total;
+            if (before > j0) break;
+        }
+        __syncthreads();
+    }
+    WorkCursor<CH> cur{kv_indptr, kv_len, B, T, Hkv, 0, 0, 0, 0, 0, 0};
+    if (w_begin < w_end) cur.start(s_first[0], s_first[1], (int)(w_begin % Hkv));
+
     if (warp == CWARPS) {
         // ------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             uint32_t it = 0;
-            SeqCache sc;
-            for (int w = w_begin; w < w_end && !*abort; ++w) {
-                const int slot = w / Hkv, g = w % Hkv;
-                bool bad;
-                const Item itm = item_of<CH>(slot, kv_indptr, kv_len, B, T, bad, sc);
-                if (bad && g == 0) atomicOr(err, DEVERR_BAD_LAYOUT);
-                if (itm.n_tok == 0) continue;
-                const int nsub = (itm.n_tok + SUB - 1) / SUB;
+            for (int64_t w = w_begin; w < w_end && !*abort; ++w, cur.next()) {
+                const int g = cur.g, n_tok = cur.n_tok();
+                const int64_t tok0 = cur.tok0();
+                const int nsub = (n_tok + SUB - 1) / SUB;
                 for (int pass = 0; pass < 2 && !*abort; ++pass) {
                     const CUtensorMap* tm = pass == 0 ? &tmK : &tmV;
                     for (int sb = 0; sb < nsub; ++sb, ++it) {
@@ -186,19 +257,19 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                             *abort = 1;
                             break;
                         }
-                        const int live = min(SUB, itm.n_tok - sb * SUB);
+                        const int live = min(SUB, n_tok - sb * SUB);
                         const int ngrp = (live + BOX_TOK - 1) / BOX_TOK;
                         const uint32_t fb = smem_u32(&full[st]);
                         const bool with_q = pass == 0 && sb == 0;  // the item's queries ride on its first stage
                         mbar_arrive_expect_tx(fb, (uint32_t)(ngrp * 2 * BOX_BYTES + (with_q ? L::Q_BYTES : 0)));
                         if (with_q)
                             bulk_load(smem_u32(base + L::Q_OFF + st * L::Q_BYTES),
-                                      q + ((int64_t)itm.b * Hq + (int64_t)g * G) * D, L::Q_BYTES, fb);
+                                      q + ((int64_t)cur.b * Hq + (int64_t)g * G) * D, L::Q_BYTES, fb);
                         const uint32_t dst = stage0 + st * STAGE_BYTES;
                         for (int tg = 0; tg < ngrp; ++tg)
                             for (int hf = 0; hf < 2; ++hf)
                                 tma_load_2d(dst + (tg * 2 + hf) * BOX_BYTES, tm, g * D + hf * 64,
-                                            (int)(itm.tok0 + sb * SUB + tg * BOX_TOK), fb);
+                                            (int)(tok0 + sb * SUB + tg * BOX_TOK), fb);
                     }
                 }
             }
@@ -212,13 +283,9 @@ decode_attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 
     // ---------------------------------------------------- compute warps
     uint32_t it = 0;
-    SeqCache sc;
-    for (int w = w_begin; w < w_end; ++w) {
-        const int slot = w / Hkv, g = w % Hkv;
-        bool bad;
-        const Item itm = item_of<CH>(slot, kv_indptr, kv_len, B, T, bad, sc);
-        if (itm.n_tok == 0) continue;
-        const int n_tok = itm.n_tok;
+    for (int64_t w = w_begin; w < w_end; ++w, cur.next()) {
+        const int g = cur.g, n_tok = cur.n_tok();
+        const int64_t slot = cur.tok0() / CH;  // the item's row of the partials
         const int nsub = (n_tok + SUB - 1) / SUB;
 
         // ---- scores: in stage sb, warp w owns the 16 tokens [16 w, 16 w + 16)
@@ -405,7 +472,7 @@ decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restri
     const int len = kv_len[b];
     const int64_t cap = (int64_t)kv_indptr[b + 1] - sbase;
     // the same checks as phase 1: a sequence past the cache's T tokens has no partials to merge
-    if ((sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap || (int64_t)kv_indptr[b + 1] > T) {
+    if (sbase < 0 || (sbase % CHUNK) != 0 || len <= 0 || (int64_t)len > cap || (int64_t)kv_indptr[b + 1] > T) {
         if (lane == 0) atomicOr(err, DEVERR_BAD_LAYOUT);  // out row left unwritten
         return;
     }
@@ -509,14 +576,14 @@ int launch_chunks(const void* q, const void* k, const void* v, const int32_t* kv
         !bi::make_tmap_2d(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, row, (uint64_t)T, row * 2, 64, BOX_TOK,
                           CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
+    // the live items (counted on the device) are at most one per (CH-token slot of the cache, kv head)
     const int64_t items = ((T + CH - 1) / CH) * Hkv;
-    if (items > 0x7fffffffLL) return BI_ERR_UNSUPPORTED_SHAPE;
     const int sms = num_sms();
     if (sms <= 0) return BI_ERR_CUDA;
     const int64_t ctas = 2LL * sms;  // two persistent CTAs per SM: one computes while the other waits
     dim3 grid((unsigned)(items < ctas ? items : ctas));
     if (bi::launch_pdl(kern, grid, dim3(THREADS), L::BYTES, s, 0u, tmK, tmV, static_cast<const __nv_bfloat16*>(q),
-                       kv_indptr, kv_len, B, T, Hq, Hkv, (int)items, scale, o_part, ml_part, err) != cudaSuccess)
+                       kv_indptr, kv_len, B, T, Hq, Hkv, scale, o_part, ml_part, err) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();
 }

@@ -166,3 +166,43 @@ def test_batch_invariance():
         assert torch.equal(binding.bi_decode_attn(q, k, v, ip, ln, out_dtype=torch.float32).view(torch.int32),
                            first.view(torch.int32))
     assert binding.bi_get_device_error() == 0
+
+
+def test_small_batch_in_a_large_cache():
+    """Six requests in scattered 2048-token slots of a 128-slot cache (a serving engine's
+    layout: each sequence's capacity runs to the next listed sequence).  The live chunks are
+    spread over the CTAs, not the cache's capacity; the outputs are bitwise those of the same
+    requests packed tightly, and match the oracle."""
+    cap, n_slots = 2048, 128
+    slots = [3, 17, 18, 60, 100, 127]
+    lens = [1, 2048, 700, 257, 1999, 256]
+    reqs = _device_seqs(inputs.SEED_PROBES + 5, lens)
+    T = n_slots * cap
+    k = torch.zeros((T, 8, D), dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros_like(k)
+    for s, (qq, kk, vv) in zip(slots, reqs):
+        k[s * cap:s * cap + kk.shape[0]] = kk
+        v[s * cap:s * cap + vv.shape[0]] = vv
+    q = torch.stack([r[0] for r in reqs]).contiguous()
+    ip = torch.tensor(slots + [slots[-1] + 1], dtype=torch.int32, device="cuda") * cap
+    ln = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    binding.bi_clear_device_error()
+    got = binding.bi_decode_attn(q, k, v, ip, ln, out_dtype=torch.float32)
+    packed = binding.bi_decode_attn(*_pack(reqs), out_dtype=torch.float32)
+    assert torch.equal(got.view(torch.int32), packed.view(torch.int32))
+    assert binding.bi_get_device_error() == 0
+    for b, (qq, kk, vv) in enumerate(reqs):
+        ref = oracle.decode_attn(host(qq)[None], host(kk), host(vv), np.array([0, kk.shape[0]], np.int64),
+                                 np.array([kk.shape[0]], np.int32), 8, 1.0 / np.sqrt(D))
+        assert rel_frobenius(host(got[b]), ref[0]) <= 1e-4, b
+
+
+def test_decreasing_kv_indptr_is_reported():
+    """Overlapping sequences (a decreasing kv_indptr) are refused on the device: bit 0x100 and no fault."""
+    kv_len = np.array([100, 100], np.int32)
+    q, k, v, indptr, T = inputs.attn_case(kv_len, 32, 8, D, CHUNK, 17)
+    k3 = np.zeros((1024, 8, D), np.uint16)
+    binding.bi_clear_device_error()
+    binding.bi_decode_attn(dev(q), dev(k3), dev(k3), dev(np.array([512, 0, 1024], np.int32)), dev(kv_len))
+    assert binding.bi_get_device_error() & 0x100
+    binding.bi_clear_device_error()
