@@ -32,11 +32,14 @@ int bi_ctrl_lora_shrink_atomic(const void* x, const void* A, float* t, int64_t M
 
 /*
  * bi_ctrl_lora_shrink_tc -- bi_lora_shrink at r = 64 on tcgen05 instead of mma.sync: the same K
- * slices, cluster and slice-ordered on-chip combine, with each slice's partial accumulated by
- * tcgen05.mma (M = 128 rows, N = 64, K = 16) in TMEM.  The study behind keeping mma.sync in the
- * plan: faster here at small batches, slower at M = 4096.  Batch-invariant and deterministic;
- * its bits differ from bi_lora_shrink's in the last places (a different accumulation inside the
- * 16-deep steps).  Arguments as bi_lora_shrink; r must be 64.
+ * slices and slice-ordered on-chip combine, with each slice's partial accumulated by
+ * tcgen05.mma (M = 128 rows, N = 64, K = 16) in its own TMEM accumulator.  A cluster holds
+ * split_k CTAs of one slice each while the row tiles fit the GPU's clusters of that size in
+ * one round, else split_k / 2 CTAs of two slices each; both give the same bits.  The study
+ * behind keeping mma.sync in the plan: within 5 % of it at every batch size measured
+ * (faster at most).  Batch-invariant and deterministic; its bits differ from bi_lora_shrink's
+ * in the last places (a different accumulation inside the 16-deep steps).  Arguments as
+ * bi_lora_shrink; r must be 64.
  */
 int bi_ctrl_lora_shrink_tc(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r, int32_t split_k,
                            void* stream);

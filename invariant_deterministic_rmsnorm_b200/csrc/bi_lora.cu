@@ -377,18 +377,26 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
 }
 
 // ------------------------------------------------------------------ shrink on tcgen05 (r = 64)
-// The study of the tcgen05 alternative for r = 64 (bi_ctrl_lora_shrink_tc; the plan keeps the
-// mma.sync kernel above, which measured faster at the large batches).  At r = 64 the mma.sync
-// kernel feeds its warp-level MMAs from shared memory (every warp reloads the A chunk's
-// fragments for its 16 rows).  This variant keeps the
-// same slices, clusters, TMA ring and on-chip combine, but one thread issues tcgen05.mma
-// (M = 128 rows of x, N = 64, K = 16) straight from the TMA-written tiles into a TMEM
-// accumulator, four warps read it back, and each row's partial is pushed to the CTA that
-// combines it.  Slice s's partial is one fp32 chain over its K slice in 16-deep ascending steps;
-// the combine is the same ((P0 + P1) + ...) + P(split-1).  The tensor core's accumulation is not
-// the warp-level MMA's, so r = 64 results differ from the mma.sync kernel's in the last bits; both
-// are batch-invariant, and parity holds against the oracle.
+// The tcgen05 alternative for r = 64 (bi_ctrl_lora_shrink_tc).  At r = 64 the mma.sync kernel
+// feeds its warp-level MMAs from shared memory: every warp reloads the whole A chunk for its 16
+// rows.  Here one thread issues tcgen05.mma (M = 128 rows of x, N = 64, K = 16) straight from the
+// TMA-written tiles into TMEM, four warps read the partials back, and each row's partials are
+// pushed to the CTA that combines it.
+//
+// A kernel that allocates TMEM gets one CTA per SM from the cluster scheduler, and clusters of 8
+// then fit only 15 at a time (120 SMs).  So a cluster holds C CTAs, C = split or split / 2, and
+// each CTA computes SPC = split / C slices of K: slice s = SPC * rank + l.  Every slice keeps its
+// own TMEM accumulator and its own chain over its 512 (K / split) columns in 16-deep ascending
+// steps from zero, exactly as if one CTA computed it, and the combine is the same ((P0 + P1) +
+// ...) + P(split-1), so both shapes give the same bits.  The host takes C = split while the
+// tiles fit the GPU's clusters of that size at once, and C = split / 2 beyond, where the bigger
+// clusters would need a second round.  With one CTA per SM the ring gets about 140 KB.
+// The tensor core's accumulation is not the warp-level MMA's, so r = 64 results differ from the
+// mma.sync kernel's in the last bits; both are batch-invariant, and parity holds against the
+// oracle.
 constexpr int ST_THREADS = 7 * 32;  // producer, MMA issuer, four TMEM readers, combiner
+constexpr int ST_MAX_CLUSTER = SH_MAX_SPLIT;
+constexpr int ST_MAX_SPC = 2;  // slices per CTA
 
 template <int R>
 struct TcLayout {
@@ -396,23 +404,27 @@ struct TcLayout {
     static constexpr int X_STAGE = SH_TM * SH_KC * 2;  // 16 KB
     static constexpr int A_STAGE = SH_KC * R * 2;      // 8 KB: one [64 K x 64 r] box
     static constexpr int STAGE = X_STAGE + A_STAGE;
-    static constexpr int RECV = SH_TM * R * 4;         // one buffer of partials for this CTA's rows
-    static constexpr int BUDGET = 112 * 1024 - 1024 - 256;  // two CTAs per SM
-    static constexpr int STAGES = (BUDGET - RECV) / STAGE;
-    static_assert(STAGES >= 3, "the ring needs at least three stages");
+    // one receive buffer: [split slices][128 / C rows this CTA combines][R] fp32, at most 64 KB
+    // (split / C <= ST_MAX_SPC)
+    static constexpr int RECV = ST_MAX_SPC * SH_TM * R * 4;
+    static constexpr int BUDGET = 224 * 1024;  // one CTA per SM
+    static constexpr int STAGES_FIT = (BUDGET - 1024 - 512 - RECV) / STAGE;
+    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+    static_assert(STAGES >= 4, "the ring needs at least four stages");
     static constexpr int RECV_OFF = STAGES * STAGE;
     static constexpr int BAR_OFF = RECV_OFF + RECV;
-    // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, rfull, rfree[SH_MAX_SPLIT], then
+    // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, rfull, rfree[ST_MAX_CLUSTER], then
     // the TMEM address and the abort flag
-    static constexpr int NBARS = 2 * STAGES + 5 + 1 + SH_MAX_SPLIT;
+    static constexpr int NBARS = 2 * STAGES + 5 + 1 + ST_MAX_CLUSTER;
     static constexpr size_t BYTES = 1024 + (size_t)BAR_OFF + NBARS * 8 + 16;
-    static constexpr uint32_t TMEM_COLS = 2 * R;  // two accumulators
+    // two accumulator sets (double-buffered across tiles) of ST_MAX_SPC slices
+    static constexpr uint32_t TMEM_COLS = 2 * ST_MAX_SPC * R;
 };
 
 template <int R>
-__global__ void __launch_bounds__(ST_THREADS, 2)
+__global__ void __launch_bounds__(ST_THREADS, 1)
 lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
-                      float* __restrict__ t, int M, int KS, int split, int n_tiles, uint32_t* err) {
+                      float* __restrict__ t, int M, int KS, int split, int C, int n_tiles, uint32_t* err) {
     using L = TcLayout<R>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -422,18 +434,18 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
     uint64_t* tfull = empty + L::STAGES;  // [2]
     uint64_t* tempty = tfull + 2;         // [2]
     uint64_t* drain = tempty + 2;
-    uint64_t* rfull = drain + 1;          // every row of every slice for this CTA's rows is stored
-    uint64_t* rfree = rfull + 1;          // [8]: CTA d's receive buffer may be written again
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rfree + SH_MAX_SPLIT);
+    uint64_t* rfull = drain + 1;          // every slice of every row this CTA combines is stored
+    uint64_t* rfree = rfull + 1;          // [ST_MAX_CLUSTER]: CTA d's receive buffer may be written again
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rfree + ST_MAX_CLUSTER);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const uint32_t slice = cluster_ctarank();
-    const int kbase = (int)slice * KS;
+    const int rank = (int)cluster_ctarank();
+    const int spc = split / C;  // slices per CTA (C: CTAs of the cluster)
     const int nchunks = KS / SH_KC;
-    const int rows_per = SH_TM / split;
+    const int rows_per = SH_TM / C;  // rows of a tile that each CTA combines
 
     if (tid == 0) {
         for (int i = 0; i < L::STAGES; ++i) {
@@ -445,8 +457,8 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
             mbar_init(smem_u32(&tempty[b]), 4);
         }
         mbar_init(smem_u32(drain), 1);
-        mbar_init(smem_u32(rfull), SH_TM);  // one arrival per row of the tile, from whichever slice
-        for (int d = 0; d < SH_MAX_SPLIT; ++d) mbar_init(smem_u32(&rfree[d]), 1);
+        mbar_init(smem_u32(rfull), SH_TM);  // one arrival per row of the tile, from its reader lane
+        for (int d = 0; d < ST_MAX_CLUSTER; ++d) mbar_init(smem_u32(&rfree[d]), 1);
         *abort = 0;
         fence_barrier_init();
         fence_proxy_async_shared();
@@ -464,28 +476,33 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
     pdl_trigger();
 
     if (warp == 0) {
-        // ------------------------------------------------ producer: one ring across all tiles
+        // ------------------------------------------------ producer: one ring across all tiles and slices
         if (lane == 0) {
             prefetch_tmap(&tmX);
             prefetch_tmap(&tmA);
             uint32_t it = 0;
-            for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
-                for (int c = 0; c < nchunks; ++c, ++it) {
-                    const int st = (int)(it % L::STAGES);
-                    const uint32_t round = it / L::STAGES;
-                    if (!mbar_wait(smem_u32(&empty[st]), (round & 1u) ^ 1u, abort)) {
-                        atomicOr(err, bi::DEVERR_WAIT_TMA);
-                        *abort = 1;
-                        break;
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < n_tiles && !stop; tile += gridDim.x) {
+                for (int l = 0; l < spc && !stop; ++l) {
+                    const int kbase = (spc * rank + l) * KS;
+                    for (int c = 0; c < nchunks; ++c, ++it) {
+                        const int st = (int)(it % L::STAGES);
+                        const uint32_t round = it / L::STAGES;
+                        if (*abort || !mbar_wait(smem_u32(&empty[st]), (round & 1u) ^ 1u, abort)) {
+                            if (!*abort) atomicOr(err, bi::DEVERR_WAIT_TMA);
+                            *abort = 1;
+                            stop = true;
+                            break;
+                        }
+                        uint8_t* sx = base + st * L::STAGE;
+                        const uint32_t fb = smem_u32(&full[st]);
+                        mbar_arrive_expect_tx(fb, L::STAGE);
+                        tma_load_2d(smem_u32(sx), &tmX, kbase + c * SH_KC, tile * SH_TM, fb);
+                        tma_load_2d(smem_u32(sx + L::X_STAGE), &tmA, 0, kbase + c * SH_KC, fb);
                     }
-                    uint8_t* sx = base + st * L::STAGE;
-                    const uint32_t fb = smem_u32(&full[st]);
-                    mbar_arrive_expect_tx(fb, L::STAGE);
-                    tma_load_2d(smem_u32(sx), &tmX, kbase + c * SH_KC, tile * SH_TM, fb);
-                    tma_load_2d(smem_u32(sx + L::X_STAGE), &tmA, 0, kbase + c * SH_KC, fb);
                 }
             }
-            if (*abort) {
+            if (*abort) {  // let loads already in flight land before the shared memory is released
                 for (uint32_t i = it > (uint32_t)L::STAGES ? it - L::STAGES : 0u; i < it; ++i)
                     (void)mbar_wait(smem_u32(&full[i % L::STAGES]), (i / L::STAGES) & 1u, nullptr);
             }
@@ -495,7 +512,8 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc_bf16_f32(SH_TM, R, 0, 1);
             uint32_t it = 0, local = 0;
-            for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x, ++local) {
+            bool stop = false;
+            for (int tile = blockIdx.x; tile < n_tiles && !stop && !*abort; tile += gridDim.x, ++local) {
                 const uint32_t acc = local & 1u, use = local >> 1;
                 if (!mbar_wait(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort)) {
                     atomicOr(err, bi::DEVERR_WAIT_ACCUM);
@@ -503,39 +521,43 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * R;
-                for (int c = 0; c < nchunks; ++c, ++it) {
-                    const int st = (int)(it % L::STAGES);
-                    if (!mbar_wait(smem_u32(&full[st]), (it / L::STAGES) & 1u, abort)) {
-                        atomicOr(err, bi::DEVERR_WAIT_FULL);
-                        *abort = 1;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t xs = smem_u32(base + st * L::STAGE);
-                    const uint32_t as = xs + L::X_STAGE;
+                for (int l = 0; l < spc && !stop; ++l) {
+                    // slice spc * rank + l: its own accumulator, its own chain from zero
+                    const uint32_t d_tmem = tmem_base + (acc * ST_MAX_SPC + (uint32_t)l) * R;
+                    for (int c = 0; c < nchunks; ++c, ++it) {
+                        const int st = (int)(it % L::STAGES);
+                        if (!mbar_wait(smem_u32(&full[st]), (it / L::STAGES) & 1u, abort)) {
+                            atomicOr(err, bi::DEVERR_WAIT_FULL);
+                            *abort = 1;
+                            stop = true;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t xs = smem_u32(base + st * L::STAGE);
+                        const uint32_t as = xs + L::X_STAGE;
 #pragma unroll
-                    for (int k = 0; k < SH_KC / 16; ++k) {
-                        // x: K-major, 128-byte swizzle, 32 bytes per 16-deep step along the row
-                        const uint64_t adesc = make_smem_desc(xs + k * 32, 16, 1024, 2);
-                        // A chunk: N-major (r contiguous), 128-byte swizzle, 16 K-rows of 128 bytes per step
-                        const uint64_t bdesc = make_smem_desc(as + k * 16 * 128, 8192, 1024, 2);
-                        mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (c | k) != 0 ? 1u : 0u);
+                        for (int k = 0; k < SH_KC / 16; ++k) {
+                            // x: K-major, 128-byte swizzle, 32 bytes per 16-deep step along the row
+                            const uint64_t adesc = make_smem_desc(xs + k * 32, 16, 1024, 2);
+                            // A chunk: N-major (r contiguous), 128-byte swizzle, 16 K-rows of 128 bytes per step
+                            const uint64_t bdesc = make_smem_desc(as + k * 16 * 128, 8192, 1024, 2);
+                            mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (c | k) != 0 ? 1u : 0u);
+                        }
+                        mma_commit(smem_u32(&empty[st]));  // the stage is free once these MMAs have read it
                     }
-                    mma_commit(smem_u32(&empty[st]));  // the stage is free once these MMAs have read it
                 }
-                mma_commit(smem_u32(&tfull[acc]));  // this slice's partial of the tile is complete
+                if (!stop) mma_commit(smem_u32(&tfull[acc]));  // this CTA's slices of the tile are complete
             }
             mma_commit(smem_u32(drain));  // TMEM is released only after every MMA completed
             (void)mbar_wait(smem_u32(drain), 0u, nullptr);
         }
     } else if (warp <= 5) {
-        // ------------------------------------------------ TMEM readers: one row of the partial per lane
+        // ------------------------------------------------ TMEM readers: one row of the partials per lane
         const int quarter = warp & 3;            // this warp may read TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;     // row of the tile
         const int d = row / rows_per;            // the CTA that combines it
         const int lrow = row - d * rows_per;
-        const uint32_t dst = mapa(smem_u32(recv) + (uint32_t)((((int)slice * rows_per + lrow) * R) * 4), (uint32_t)d);
+        const uint32_t peer_recv = mapa(smem_u32(recv), (uint32_t)d);
         const uint32_t bar = mapa(smem_u32(rfull), (uint32_t)d);
         const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
         uint32_t local = 0;
@@ -547,26 +569,34 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
                 *abort = 1;
                 break;
             }
-            tc_fence_after();
-            uint32_t v[2][32];
-            tmem_ld_32x32b_x32(lane_addr + acc * R, v[0]);
-            tmem_ld_32x32b_x32(lane_addr + acc * R + 32, v[1]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));  // the accumulator may be reused
             // d has read what this lane pushed for the previous tile (one receive buffer)
-            if (!mbar_wait_cluster(smem_u32(&rfree[d]), (local & 1u) ^ 1u, abort)) {
-                atomicOr(err, bi::DEVERR_WAIT_CLUSTER);
+            const bool freed = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&rfree[d]), (local & 1u) ^ 1u, abort));
+            if (!freed) {
+                if (lane == 0) atomicOr(err, bi::DEVERR_WAIT_CLUSTER);
                 *abort = 1;
                 break;
             }
+            tc_fence_after();
+            for (int l = 0; l < spc; ++l) {
+                uint32_t v[2][32];
+                tmem_ld_32x32b_x32(lane_addr + (acc * ST_MAX_SPC + (uint32_t)l) * R, v[0]);
+                tmem_ld_32x32b_x32(lane_addr + (acc * ST_MAX_SPC + (uint32_t)l) * R + 32, v[1]);
+                tmem_wait_ld();
+                // row lrow of slice s in d's buffer [split][rows_per][R]; the 16-byte pieces of a row
+                // are rotated by the row, so that the 32 lanes' stores spread over the banks
+                const int s = spc * rank + l;
+                const uint32_t dst = peer_recv + (uint32_t)(((s * rows_per + lrow) * R) * 4);
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    st_cluster_v4(dst + (uint32_t)((h * 32 + i) * 4), v[h][i], v[h][i + 1], v[h][i + 2], v[h][i + 3]);
-            mbar_arrive_cluster(bar);  // release: this row is visible before the arrival
+                    for (int i = 0; i < 32; i += 4)
+                        st_cluster_v4(dst + (uint32_t)((((h * 8 + i / 4) + lrow) & (R / 4 - 1)) * 16), v[h][i],
+                                      v[h][i + 1], v[h][i + 2], v[h][i + 3]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));  // the accumulators may be reused
+            mbar_arrive_cluster(bar);  // release: this row's slices are visible before the arrival
         }
     } else {
         // ------------------------------------------------ combiner: this CTA's rows of every tile
@@ -578,12 +608,13 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
                 *abort = 1;
                 break;
             }
-            const int row0 = tile * SH_TM + (int)slice * rows_per;
+            const int row0 = tile * SH_TM + rank * rows_per;
             for (int i = lane; i < rows_per * R / 4; i += 32) {
                 const int row = (4 * i) / R, col = (4 * i) % R;
-                float4 v = *reinterpret_cast<const float4*>(recv + row * R + col);
+                const int piece = (((col >> 2) + row) & (R / 4 - 1)) * 4;  // where the readers put it
+                float4 v = *reinterpret_cast<const float4*>(recv + row * R + piece);
                 for (int sl = 1; sl < split; ++sl) {  // ((P0 + P1) + P2) + ...: slice order
-                    const float4 p = *reinterpret_cast<const float4*>(recv + (sl * rows_per + row) * R + col);
+                    const float4 p = *reinterpret_cast<const float4*>(recv + (sl * rows_per + row) * R + piece);
                     v.x = __fadd_rn(v.x, p.x);
                     v.y = __fadd_rn(v.y, p.y);
                     v.z = __fadd_rn(v.z, p.z);
@@ -592,7 +623,8 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
                 if (row0 + row < M) *reinterpret_cast<float4*>(t + (size_t)(row0 + row) * R + col) = v;
             }
             __syncwarp();
-            if (lane < split) mbar_arrive_cluster(mapa(smem_u32(&rfree[slice]), (uint32_t)lane));
+            // this CTA's buffer has been read: every sender in the cluster may refill it
+            if (lane < C) mbar_arrive_cluster(mapa(smem_u32(&rfree[rank]), (uint32_t)lane));
         }
     }
     // no CTA leaves, or frees TMEM, while a peer may still store into it or signal it
@@ -867,31 +899,44 @@ int launch_shrink_tc(const void* x, const void* A, float* t, int64_t M, int64_t 
     uint32_t* err = bi::device_error_word();
     auto kern = lora_shrink_tc_kernel<R>;
     if (!err || !set_smem_once(kern, L::BYTES)) return BI_ERR_CUDA;
-    static std::mutex mu;
-    static int fit_cache[64][4];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BI_ERR_CUDA;
-    const int si = split == 1 ? 0 : (split == 2 ? 1 : (split == 4 ? 2 : 3));
-    int fit;
-    {
+    // clusters of c CTAs that fit at once (cached per device and cluster size 1, 2, 4, 8)
+    static std::mutex mu;
+    static int fit_cache[64][4];
+    auto fit = [&](int c) -> int {
+        const int ci = c == 1 ? 0 : (c == 2 ? 1 : (c == 4 ? 2 : 3));
         std::lock_guard<std::mutex> lock(mu);
-        if (fit_cache[dev][si] == 0) {
+        if (fit_cache[dev][ci] == 0) {
             cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(1, (unsigned)split, 1);
+            cfg.gridDim = dim3(1, (unsigned)c, 1);
             cfg.blockDim = dim3(ST_THREADS, 1, 1);
             cfg.dynamicSmemBytes = L::BYTES;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
             attr[0].val.clusterDim.x = 1;
-            attr[0].val.clusterDim.y = (unsigned)split;
+            attr[0].val.clusterDim.y = (unsigned)c;
             attr[0].val.clusterDim.z = 1;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return BI_ERR_CUDA;
-            fit_cache[dev][si] = n > 0 ? n : 1;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return -1;
+            }
+            fit_cache[dev][ci] = n > 0 ? n : 1;
         }
-        fit = fit_cache[dev][si];
+        return fit_cache[dev][ci];
+    };
+    const int n_tiles = (int)((M + SH_TM - 1) / SH_TM);
+    // one slice per CTA while the tiles fit in one round of such clusters, else two
+    int C = split;
+    int fc = fit(C);
+    if (fc < 0) return BI_ERR_CUDA;
+    if (split >= 2 && n_tiles > fc) {
+        C = split / 2;
+        fc = fit(C);
+        if (fc < 0) return BI_ERR_CUDA;
     }
     CUtensorMap tmX, tmA;
     if (!bi::make_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2,
@@ -900,11 +945,9 @@ int launch_shrink_tc(const void* x, const void* A, float* t, int64_t M, int64_t 
     if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)R, (uint64_t)K, (uint64_t)R * 2, R,
                           SH_KC, CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
-    const int n_tiles = (int)((M + SH_TM - 1) / SH_TM);
-    const int clusters = n_tiles < fit ? n_tiles : fit;
-    if (bi::launch_pdl(kern, dim3((unsigned)clusters, (unsigned)split), dim3(ST_THREADS), L::BYTES, s,
-                       (unsigned)split, tmX, tmA, t, (int)M, (int)(K / split), (int)split, n_tiles,
-                       err) != cudaSuccess)
+    const int clusters = n_tiles < fc ? n_tiles : fc;
+    if (bi::launch_pdl(kern, dim3((unsigned)clusters, (unsigned)C), dim3(ST_THREADS), L::BYTES, s, (unsigned)C, tmX,
+                       tmA, t, (int)M, (int)(K / split), (int)split, C, n_tiles, err) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();
 }
