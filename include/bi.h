@@ -153,12 +153,14 @@ int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t
  *         always 0, because the partials never leave the chip.  ws may be NULL.
  *
  * Arithmetic: slice s of K (the contiguous range [s K / split_k, (s + 1) K / split_k)) gives
- * the partial P_s, accumulated with mma.sync (bf16 in, fp32 accumulate) in 16-deep K steps
- * in ascending order.  t = ((P_0 + P_1) + ...) + P_{split_k - 1}, each add rounded to nearest.
- * No atomics.  A thread-block cluster of split_k CTAs (CTA s = slice s) computes 128-row tiles
- * with eight compute warps of 16 rows; the partials meet in distributed shared memory, and every
- * CTA of the cluster adds the slices of 128 / split_k of the tile's rows.  The plan depends on
- * (K, r, split_k) only.
+ * the partial P_s, accumulated in fp32 from bf16 products in 16-deep K steps in ascending
+ * order, starting from zero: with mma.sync at r = 8, 16 and 32, with tcgen05.mma (one TMEM
+ * accumulator per slice) at r = 64.  t = ((P_0 + P_1) + ...) + P_{split_k - 1}, each add
+ * rounded to nearest.  No atomics.  The partials meet on chip (distributed shared memory of
+ * a thread-block cluster), and every CTA of the cluster adds all slices of its share of a
+ * 128-row tile's rows.  The arithmetic depends on (K, r, split_k) only; the cluster shape of
+ * the r = 64 kernel (split_k CTAs of one slice, or split_k / 2 of two) follows the number of
+ * tiles and gives the same bits either way.
  */
 size_t bi_lora_shrink_workspace_size(int64_t M, int64_t K, int32_t r, int32_t split_k);
 int bi_lora_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r, int32_t split_k,

@@ -31,15 +31,17 @@ int bi_ctrl_lora_shrink_atomic(const void* x, const void* A, float* t, int64_t M
                                int32_t split_k, void* stream);
 
 /*
- * bi_ctrl_lora_shrink_tc -- bi_lora_shrink at r = 64 on tcgen05 instead of mma.sync: the same K
- * slices and slice-ordered on-chip combine, with each slice's partial accumulated by
- * tcgen05.mma (M = 128 rows, N = 64, K = 16) in its own TMEM accumulator.  A cluster holds
- * split_k CTAs of one slice each while the row tiles fit the GPU's clusters of that size in
- * one round, else split_k / 2 CTAs of two slices each; both give the same bits.  The study
- * behind keeping mma.sync in the plan: within 5 % of it at every batch size measured
- * (faster at most).  Batch-invariant and deterministic; its bits differ from bi_lora_shrink's
- * in the last places (a different accumulation inside the 16-deep steps).  Arguments as
- * bi_lora_shrink; r must be 64.
+ * bi_ctrl_lora_shrink_tc -- the shrink on tcgen05 at r = 16, 32 or 64: the same K slices and
+ * slice-ordered on-chip combine as bi_lora_shrink, with each slice's partial accumulated by
+ * tcgen05.mma (M = 128 rows, N = r, K = 16) in its own TMEM accumulator.  A cluster holds
+ * split_k CTAs of one slice each while the row tiles fit the GPU's clusters of that size in one
+ * round, else split_k / 2 CTAs of two slices each (same bits either way); the partials cross
+ * the cluster as bulk shared-memory copies and four warps per CTA combine them.  At r = 64 it
+ * is bi_lora_shrink's kernel (bitwise the same call).  At r = 16 and 32 it is the study behind
+ * keeping mma.sync there: slower at r = 16, within a few percent at r = 32.  Batch-invariant and
+ * deterministic; at r = 16 and 32 its bits differ from bi_lora_shrink's in the last places (a
+ * different accumulation inside the 16-deep steps).  Arguments as bi_lora_shrink; r must be 16,
+ * 32 or 64.
  */
 int bi_ctrl_lora_shrink_tc(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r, int32_t split_k,
                            void* stream);

@@ -221,7 +221,8 @@ def bi_ctrl_lora_shrink_atomic(x: torch.Tensor, A: torch.Tensor, t: torch.Tensor
 
 def bi_ctrl_lora_shrink_tc(x: torch.Tensor, A: torch.Tensor, t: torch.Tensor | None = None, split_k: int = 8,
                            stream=None) -> torch.Tensor:
-    """The r = 64 shrink on tcgen05 (the study behind keeping mma.sync in the plan)."""
+    """The shrink on tcgen05 at r = 16, 32 or 64 (bi_lora_shrink's kernel at r = 64; the study
+    behind keeping mma.sync at r = 16 and 32)."""
     _bf16_2d(x, "x")
     _bf16_2d(A, "A")
     M, K = x.shape

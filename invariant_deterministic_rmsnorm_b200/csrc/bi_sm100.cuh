@@ -103,6 +103,17 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                  :: "r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
 }
 
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this CTA's shared
+// memory to shared memory of a CTA of the cluster (`dst` and `bar` are shared::cluster addresses,
+// from mapa); the bytes complete on that CTA's mbarrier.  No multicast.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "r"(src), "r"(bytes), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until the source of every bulk copy this thread committed has been read
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 // ---------------------------------------------------------------- tcgen05
 // TMEM allocation: executed by one full warp; writes the TMEM base address to smem `dst`.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t ncols) {

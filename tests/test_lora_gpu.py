@@ -227,17 +227,18 @@ def test_expand_batch_invariance(r):
     assert bad == 0
 
 
-# ------------------------------------------------------------------ the r = 64 tcgen05 study kernel
+# ------------------------------------------------------------------ the tcgen05 shrink
+@pytest.mark.parametrize("r", [16, 32, 64])
 @pytest.mark.parametrize("M", [1, 130, 4096])
-def test_shrink_tc_r64(M):
+def test_shrink_tc(M, r):
     """bi_ctrl_lora_shrink_tc: small-integer operands exact (every partial sum is an integer below
     2^24), random operands within the shrink's tolerance of the oracle's split-8 sum, rows
     independent of the batch, and replays identical."""
     xi = inputs.small_int_bf16(66, (M, K))
-    Ai = inputs.small_int_bf16(67, (K, 64))
+    Ai = inputs.small_int_bf16(67, (K, r))
     t = host(binding.bi_ctrl_lora_shrink_tc(dev(xi), dev(Ai)))
     assert np.array_equal(t.astype(np.float64), oracle.lora_shrink(xi, Ai))
-    x, A, _, _ = inputs.lora_case(M, 64)
+    x, A, _, _ = inputs.lora_case(M, r)
     xd, Ad = dev(x), dev(A)
     t = binding.bi_ctrl_lora_shrink_tc(xd, Ad)
     ref = oracle_rows(oracle.lora_shrink_split, x, A, 8)
