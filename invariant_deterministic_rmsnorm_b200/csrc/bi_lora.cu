@@ -195,15 +195,18 @@ struct OrderedLayout {
     static constexpr int X_STAGE = SH_TM * SH_KC * 2;  // 16 KB, 128B-swizzled rows of 64 K
     static constexpr int A_STAGE = SH_KC * R * 2;
     static constexpr int STAGE = X_STAGE + A_STAGE;
-    static constexpr int NB = R >= 32 ? 1 : 2;         // receive buffers
+    static constexpr int NB = 1;                       // receive buffers
     static constexpr int RECV = SH_TM * R * 4;         // one buffer: [slice][rows this CTA combines][R] fp32
+    // every compute warp stages its 16 rows of partials here before one bulk copy sends them
+    static constexpr int STAGING = SH_TM * R * 4;
     // two CTAs per SM: at most 112 KB each, including the 1 KB alignment pad and the barriers
     static constexpr int BUDGET = 112 * 1024 - 1024 - 256;
-    static constexpr int STAGES_FIT = (BUDGET - NB * RECV) / STAGE;
+    static constexpr int STAGES_FIT = (BUDGET - NB * RECV - STAGING) / STAGE;
     static constexpr int STAGES = STAGES_FIT > SH_MAX_STAGES ? SH_MAX_STAGES : STAGES_FIT;
     static_assert(STAGES >= 3, "the ring needs at least three stages");
     static constexpr int RECV_OFF = STAGES * STAGE;
-    static constexpr int BAR_OFF = RECV_OFF + NB * RECV;
+    static constexpr int STAGING_OFF = RECV_OFF + NB * RECV;
+    static constexpr int BAR_OFF = STAGING_OFF + STAGING;
     // full[STAGES], empty[STAGES], rfull[NB], rfree[NB][SH_MAX_SPLIT], then the abort flag
     static constexpr int NBARS = 2 * STAGES + NB + NB * SH_MAX_SPLIT;
     static constexpr size_t BYTES = 1024 + (size_t)BAR_OFF + NBARS * 8 + 16;
@@ -218,6 +221,7 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* recv = reinterpret_cast<float*>(base + L::RECV_OFF);
+    float* staging = reinterpret_cast<float*>(base + L::STAGING_OFF);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L::BAR_OFF);
     uint64_t* empty = full + L::STAGES;
     uint64_t* rfull = empty + L::STAGES;        // [NB]: every slice's partial of this CTA's rows has landed
@@ -238,7 +242,7 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
             mbar_init(smem_u32(&empty[i]), SO_CWARPS);
         }
         for (int b = 0; b < L::NB; ++b) {
-            mbar_init(smem_u32(&rfull[b]), SO_CWARPS * 32);  // every lane of the 8 sending warps
+            mbar_init(smem_u32(&rfull[b]), 1);  // per tile: this CTA's expected bytes, then the copies
             for (int d = 0; d < SH_MAX_SPLIT; ++d) mbar_init(smem_u32(&rfree[b * SH_MAX_SPLIT + d]), 1);
         }
         *abort = 0;
@@ -279,6 +283,8 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
         }
     } else if (warp == SO_CWARPS + 1) {
         // ------------------------------------------------ combiner: this CTA's rows of every tile
+        const uint32_t tile_bytes = (uint32_t)(SH_TM * R * 4);  // every slice of this CTA's rows
+        if (lane == 0 && (int)blockIdx.x < n_tiles) mbar_arrive_expect_tx(smem_u32(&rfull[0]), tile_bytes);
         int j = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
             const int b = j % L::NB;
@@ -304,6 +310,9 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
                 if (row0 + row < M) *reinterpret_cast<float4*>(t + (size_t)(row0 + row) * R + col) = v;
             }
             __syncwarp();
+            // the next tile's bytes, posted before any sender may send them
+            if (lane == 0 && tile + (int)gridDim.x < n_tiles) mbar_arrive_expect_tx(smem_u32(&rfull[0]), tile_bytes);
+            __syncwarp();
             // buffer b of this CTA has been read: every sender in the cluster may refill it
             if (lane < split) mbar_arrive_cluster(mapa(smem_u32(&rfree[b * SH_MAX_SPLIT + slice]), (uint32_t)lane));
         }
@@ -313,6 +322,8 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
         const int lrow0 = warp * 16 - d * rows_per;        // first of them inside d's share
         const uint32_t peer_recv = mapa(smem_u32(recv), (uint32_t)d);
         const uint32_t peer_rfull = mapa(smem_u32(rfull), (uint32_t)d);
+        const uint32_t stg = smem_u32(staging + warp * 16 * R);  // this warp's 16 rows, as d holds them
+        bool pending = false;  // lane 0 issued a copy whose source may still be read
         const int g = lane >> 2, q = lane & 3;
         uint32_t it = 0;
         int j = 0;
@@ -359,19 +370,31 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
                 *abort = 1;
                 break;
             }
-            // rows lrow0 + g and lrow0 + g + 8 of this slice's block in d's buffer b
-            const uint32_t dst = peer_recv + (uint32_t)((b * SH_TM * R + ((int)slice * rows_per + lrow0 + g) * R) * 4);
-            const uint32_t bar = peer_rfull + (uint32_t)b * 8u;
+            // stage rows g and g + 8 of this warp's 16, then one bulk copy puts the block at rows
+            // lrow0 .. lrow0 + 15 of this slice in d's buffer b, completing on d's receive barrier
+            if (lane == 0 && pending) bulk_wait_read();  // the previous tile's copy has read the staging
+            __syncwarp();
 #pragma unroll
             for (int nt = 0; nt < R / 8; ++nt) {
                 const uint32_t col = (uint32_t)(nt * 8 + q * 2) * 4u;
-                st_cluster_v2(dst + col, acc[nt][0], acc[nt][1]);
-                st_cluster_v2(dst + (uint32_t)(8 * R * 4) + col, acc[nt][2], acc[nt][3]);
+                asm volatile("st.shared.v2.f32 [%0], {%1, %2};" :: "r"(stg + (uint32_t)(g * R * 4) + col),
+                             "f"(acc[nt][0]), "f"(acc[nt][1]) : "memory");
+                asm volatile("st.shared.v2.f32 [%0], {%1, %2};" :: "r"(stg + (uint32_t)((g + 8) * R * 4) + col),
+                             "f"(acc[nt][2]), "f"(acc[nt][3]) : "memory");
             }
-            mbar_arrive_cluster(bar);  // release: this lane's stores above are visible before the arrival
+            fence_proxy_async_shared();  // the copy engine reads what these generic stores wrote
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t dst = peer_recv + (uint32_t)((b * SH_TM * R + ((int)slice * rows_per + lrow0) * R) * 4);
+                bulk_copy_to_peer(dst, stg, (uint32_t)(16 * R * 4), peer_rfull + (uint32_t)b * 8u);
+                bulk_commit();
+                pending = true;
+            }
         }
     }
-    // no CTA leaves while a peer may still store into its shared memory or signal its barriers
+    // no CTA leaves while a peer may still store into its shared memory or signal its barriers,
+    // or while its own bulk copies may still read its staging rows
+    if (warp < SO_CWARPS && lane == 0) bulk_wait_read();
     __syncwarp();
     cluster_sync();
 }
