@@ -225,7 +225,7 @@ def _to_dev(a, device):
     return torch.from_numpy(a).to(device)
 
 
-def build_ops(device, stream, attn_batch=None):
+def build_ops(device, stream, attn_batch=None, lora_rank=LORA_RANK):
     """Allocate the synthetic workload on the device and return the list of ops of one step.
 
     Each op: dict(name, kind 'hbm'|'tensor', work (bytes or flops per launch), launch(k), src, desc).
@@ -261,7 +261,7 @@ def build_ops(device, stream, attn_batch=None):
     qkv = gemm_op("gemm_qkv", lambda k: xns[k % R], H, 6144, inputs.SEED_WEIGHTS + 10)
 
     # LoRA on the q projection: t = x A (split-K = 8, ordered combine), q += bf16(t) B
-    r = LORA_RANK
+    r = lora_rank
     A_l = _to_dev(inputs.normal_bf16(inputs.SEED_WEIGHTS + 20, (H, r), 0.0, 0.02), device)
     B_l = _to_dev(inputs.normal_bf16(inputs.SEED_WEIGHTS + 21, (r, H), 0.0, 0.02), device)
     t = torch.empty((M, r), dtype=torch.float32, device=device)
@@ -1378,7 +1378,7 @@ def run_one_op(args):
     device = torch.device("cuda", 0)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
-        ops, _ = build_ops(device, stream, args.attn_batch)
+        ops, _ = build_ops(device, stream, args.attn_batch, args.lora_rank)
         op = next(o for o in ops if o["name"] == args.op)
         for k in range(args.launches):
             op["launch"](k)
@@ -1418,6 +1418,8 @@ def main():
                              "decode_attn"],
                     help="launch only this op of the step, --launches times, and exit (for profiler captures)")
     ap.add_argument("--launches", type=int, default=4)
+    ap.add_argument("--lora-rank", type=int, default=LORA_RANK, choices=[8, 16, 32, 64],
+                    help="LoRA rank of the --op lora_shrink / lora_expand launches (the step uses 16)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
