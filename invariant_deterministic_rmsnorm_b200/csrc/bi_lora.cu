@@ -779,27 +779,49 @@ lora_expand_kernel(const float* __restrict__ t, const __nv_bfloat16* __restrict_
         }
     }
 
-    // 1. bf16(t) rows into shared memory (rows past M and columns past R are zero).
-    for (int i = tid; i < EX_TM * L::RP / 4; i += EX_THREADS) {
+    // 1-2. Every global load of t and of the B tile is issued before the first shared-memory store,
+    //      so that their L2 latencies overlap instead of adding up.
+    constexpr int T_ITERS = EX_TM * L::RP / 4 / EX_THREADS;   // float4 pieces of t per thread
+    constexpr int B_ITERS = L::RP * (EX_TN / 8) / EX_THREADS;  // 8-column pieces of B per thread
+    static_assert(T_ITERS * EX_THREADS * 4 == EX_TM * L::RP && B_ITERS * EX_THREADS * 8 == L::RP * EX_TN,
+                  "the staging loops cover their tiles exactly");
+    float4 tv[T_ITERS];
+    uint4 bv[B_ITERS];
+#pragma unroll
+    for (int j = 0; j < T_ITERS; ++j) {
+        const int i = tid + j * EX_THREADS;
         const int row = (4 * i) / L::RP, k = (4 * i) % L::RP;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (m0 + row < M && k < R) v = *reinterpret_cast<const float4*>(t + (size_t)(m0 + row) * R + k);
-        uint2 p = make_uint2(bi::pack_bf16x2(v.x, v.y), bi::pack_bf16x2(v.z, v.w));
+        tv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (m0 + row < M && k < R) tv[j] = *reinterpret_cast<const float4*>(t + (size_t)(m0 + row) * R + k);
+    }
+#pragma unroll
+    for (int j = 0; j < B_ITERS; ++j) {
+        const int i = tid + j * EX_THREADS;
+        const int k = i / (EX_TN / 8), c = i % (EX_TN / 8);
+        const int col = n0 + c * 8;
+        bv[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (k < R && col < N) bv[j] = bi::ld_cached_v4(B + (size_t)k * N + col);
+    }
+    // 1. bf16(t) rows into shared memory (rows past M and columns past R are zero).
+#pragma unroll
+    for (int j = 0; j < T_ITERS; ++j) {
+        const int i = tid + j * EX_THREADS;
+        const int row = (4 * i) / L::RP, k = (4 * i) % L::RP;
+        const uint2 p = make_uint2(bi::pack_bf16x2(tv[j].x, tv[j].y), bi::pack_bf16x2(tv[j].z, tv[j].w));
         *reinterpret_cast<uint2*>(sT + row * L::T_PITCH + k * 2) = p;
     }
     // 2. The B tile [R, 128], permuted: the 8 weights of output columns [8c, 8c + 8) (c = 4 gg + qq)
     //    go, two at a time, to shared-memory columns 32 gg + 8 p + 2 qq, p = 0..3.  Columns past N
     //    and rows past R are zero.
-    for (int i = tid; i < L::RP * (EX_TN / 8); i += EX_THREADS) {
+#pragma unroll
+    for (int j = 0; j < B_ITERS; ++j) {
+        const int i = tid + j * EX_THREADS;
         const int k = i / (EX_TN / 8), c = i % (EX_TN / 8);
-        const int col = n0 + c * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (k < R && col < N) v = bi::ld_cached_v4(B + (size_t)k * N + col);
         uint32_t* dst = reinterpret_cast<uint32_t*>(sB + k * L::B_PITCH) + 16 * (c >> 2) + (c & 3);
-        dst[0] = v.x;
-        dst[4] = v.y;
-        dst[8] = v.z;
-        dst[12] = v.w;
+        dst[0] = bv[j].x;
+        dst[4] = bv[j].y;
+        dst[8] = bv[j].z;
+        dst[12] = bv[j].w;
     }
     __syncthreads();
     pdl_trigger();
