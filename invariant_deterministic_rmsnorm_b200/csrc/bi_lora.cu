@@ -392,9 +392,10 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
             }
         }
     }
-    // no CTA leaves while a peer may still store into its shared memory or signal its barriers,
-    // or while its own bulk copies may still read its staging rows
-    if (warp < SO_CWARPS && lane == 0) bulk_wait_read();
+    // no CTA leaves while a peer may still store into its shared memory or signal its barriers:
+    // every bulk copy of this CTA has landed before it joins the final cluster barrier (on an
+    // error path a receiver may have stopped waiting for them)
+    if (warp < SO_CWARPS && lane == 0) bulk_wait_all();
     __syncwarp();
     cluster_sync();
 }
@@ -697,7 +698,9 @@ lora_shrink_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_cons
                 if (lane < C) mbar_arrive_cluster(mapa(smem_u32(&rfree[rank]), (uint32_t)lane));
             }
         }
-        if (pending) bulk_wait_read();  // the staging rows stay valid until the copies have read them
+        // the copies have landed (destination writes included) before this CTA joins the final
+        // cluster barrier, after which a receiver may leave
+        if (pending) bulk_wait_all();
     }
     // no CTA leaves, or frees TMEM, while a peer may still store into it or signal it
     tc_fence_before();
