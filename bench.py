@@ -48,6 +48,8 @@ HIDDEN = 4096
 EPS = 1e-6
 ROTATE = 4  # activation buffer sets cycled through by consecutive steps
 LORA_RANK = 16
+NOMINAL_HBM_GBS = 8000.0       # B200 datasheet HBM3e bandwidth (context only)
+NOMINAL_BF16_TFLOPS = 2250.0   # B200 datasheet dense bf16 tensor peak (context only)
 ATTN_BATCH = 64
 
 # DRAM traffic per launch from an ncu capture, valid only while the kernel source is unchanged.
@@ -531,7 +533,9 @@ def run_ours(args, rank, world, local_rank):
                 "peak_source": (f"{peak_src} (MEASURED_PEAKS.json" + (f", {tensor_peak_name})" if bound == "tensor"
                                                                        else ", hbm_gbs)"))
                 if peak_src == "measured" else "fallback",
-                "algorithmic_work_per_launch": dop["work"]}
+                "algorithmic_work_per_launch": dop["work"],
+                # the datasheet figures, context only: 8 TB/s HBM3e, 2.25 PFLOP/s dense bf16
+                "frac_of_nominal": round(ach / (NOMINAL_HBM_GBS if bound == "hbm" else NOMINAL_BF16_TFLOPS), 4)}
 
     cpu = cpu_baseline(args.cpu_seconds)
     line = {
