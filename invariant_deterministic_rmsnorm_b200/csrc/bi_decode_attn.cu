@@ -480,33 +480,43 @@ decode_attn_merge_kernel(const float* __restrict__ o_part, const float* __restri
     const int64_t slot0 = sbase / CH;
     float m = -INFINITY, l = 0.0f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    // The merge is sequential in c; the loads are not.  Fetch PF chunks ahead, merge them in order.
-    constexpr int PF = 16;
-    for (int c0 = 0; c0 < nch; c0 += PF) {
-        float2 mlc[PF];
-        float4 oc[PF];
+    // The merge is sequential in c; the loads are not.  Two register buffers of PF chunks: the
+    // loads of the next PF chunks are in flight while the current PF are merged, in order.
+    constexpr int PF = 8;
+    float2 mlA[PF], mlB[PF];
+    float4 oA[PF], oB[PF];
+    auto fetch = [&](int c0, float2 (&ml)[PF], float4 (&ov)[PF]) {
 #pragma unroll
         for (int i = 0; i < PF; ++i) {
             if (c0 + i < nch) {
                 const int64_t idx = (slot0 + c0 + i) * Hq + h;
-                mlc[i] = *reinterpret_cast<const float2*>(ml_part + idx * 2);
-                oc[i] = *reinterpret_cast<const float4*>(o_part + idx * D + lane * 4);
+                ml[i] = *reinterpret_cast<const float2*>(ml_part + idx * 2);
+                ov[i] = *reinterpret_cast<const float4*>(o_part + idx * D + lane * 4);
             }
         }
+    };
+    auto merge = [&](int c0, const float2 (&ml)[PF], const float4 (&ov)[PF]) {
 #pragma unroll
         for (int i = 0; i < PF; ++i) {
             if (c0 + i < nch) {
-                const float mn = fmaxf(m, mlc[i].x);
+                const float mn = fmaxf(m, ml[i].x);
                 const float a = expf(__fsub_rn(m, mn));   // 0 on the first chunk (m = -inf)
-                const float bsc = expf(__fsub_rn(mlc[i].x, mn));
-                l = __fmaf_rn(l, a, __fmul_rn(mlc[i].y, bsc));
-                o.x = __fmaf_rn(o.x, a, __fmul_rn(oc[i].x, bsc));
-                o.y = __fmaf_rn(o.y, a, __fmul_rn(oc[i].y, bsc));
-                o.z = __fmaf_rn(o.z, a, __fmul_rn(oc[i].z, bsc));
-                o.w = __fmaf_rn(o.w, a, __fmul_rn(oc[i].w, bsc));
+                const float bsc = expf(__fsub_rn(ml[i].x, mn));
+                l = __fmaf_rn(l, a, __fmul_rn(ml[i].y, bsc));
+                o.x = __fmaf_rn(o.x, a, __fmul_rn(ov[i].x, bsc));
+                o.y = __fmaf_rn(o.y, a, __fmul_rn(ov[i].y, bsc));
+                o.z = __fmaf_rn(o.z, a, __fmul_rn(ov[i].z, bsc));
+                o.w = __fmaf_rn(o.w, a, __fmul_rn(ov[i].w, bsc));
                 m = mn;
             }
         }
+    };
+    fetch(0, mlA, oA);
+    for (int c0 = 0; c0 < nch; c0 += 2 * PF) {
+        fetch(c0 + PF, mlB, oB);
+        merge(c0, mlA, oA);
+        fetch(c0 + 2 * PF, mlA, oA);
+        merge(c0 + PF, mlB, oB);
     }
     const float r0 = __fdiv_rn(o.x, l), r1 = __fdiv_rn(o.y, l), r2 = __fdiv_rn(o.z, l), r3 = __fdiv_rn(o.w, l);
     const int64_t off = ((int64_t)b * Hq + h) * D + lane * 4;
