@@ -55,7 +55,7 @@ ATTN_BATCH = 64
 # DRAM traffic per launch from an ncu capture, valid only while the kernel source is unchanged.
 # {op: (sha256 of the kernel source at capture time, bytes per launch, how it was taken)}
 TRAFFIC = {
-    "decode_attn": ("d07898d88ccd5973", (4050818048 + 66076672 + 64504320 + 0 + 4050444800 + 62865664 + 64504064 + 0) // 2,
+    "decode_attn": ("0f19d0d513c0942f", (4050612224 + 65890816 + 64502272 + 768 + 4050790144 + 62856192 + 64501504 + 6912) // 2,
                     "decode_attn_chunk_kernel + decode_attn_merge_kernel, B=64 (the step's decode batch), mean of "
                     "two launches"),
 }
