@@ -227,7 +227,7 @@ def _to_dev(a, device):
     return torch.from_numpy(a).to(device)
 
 
-def build_ops(device, stream, attn_batch=None, lora_rank=LORA_RANK):
+def build_ops(device, stream, attn_batch=None, lora_rank=LORA_RANK, tokens=M_TOKENS):
     """Allocate the synthetic workload on the device and return the list of ops of one step.
 
     Each op: dict(name, kind 'hbm'|'tensor', work (bytes or flops per launch), launch(k), src, desc).
@@ -239,7 +239,7 @@ def build_ops(device, stream, attn_batch=None, lora_rank=LORA_RANK):
 
     attn_batch = attn_batch or ATTN_BATCH
     ops = []
-    M, H = M_TOKENS, HIDDEN
+    M, H = tokens, HIDDEN
     x_np, w_np = inputs.rmsnorm_case(M, H, "bf16")
     w = _to_dev(w_np, device)
     # R rotating activation sets so that consecutive steps never find their inputs in L2
@@ -1375,14 +1375,15 @@ def run_contrast(args):
 
 
 def run_one_op(args):
-    """A few launches of one op of the step, at the step's configuration, on rotating inputs: the
-    target of a one-kernel profiler capture (the other ops' inputs are built but not launched)."""
+    """A few launches of one op of the step, at the step's configuration (or M = --tokens), on
+    rotating inputs: the target of a one-kernel profiler capture (the other ops' inputs are built
+    but not launched)."""
     import torch
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
-        ops, _ = build_ops(device, stream, args.attn_batch, args.lora_rank)
+        ops, _ = build_ops(device, stream, args.attn_batch, args.lora_rank, args.tokens)
         op = next(o for o in ops if o["name"] == args.op)
         for k in range(args.launches):
             op["launch"](k)
@@ -1422,6 +1423,8 @@ def main():
                              "decode_attn"],
                     help="launch only this op of the step, --launches times, and exit (for profiler captures)")
     ap.add_argument("--launches", type=int, default=4)
+    ap.add_argument("--tokens", type=int, default=M_TOKENS,
+                    help="batch size M of the --op launches (the step uses 4096)")
     ap.add_argument("--lora-rank", type=int, default=LORA_RANK, choices=[8, 16, 32, 64],
                     help="LoRA rank of the --op lora_shrink / lora_expand launches (the step uses 16)")
     args = ap.parse_args()
