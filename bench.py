@@ -777,6 +777,26 @@ def gate_table(device, stream, peaks):
                                   "GB/s"))
                 del xs
             out[f"lora_shrink_r{r}"] = {"unit": "GB/s", "rows": rows}
+        # the RMSNorm fused with the r = 16 shrink of its output (one pass over x), beside the two
+        # calls it replaces launched back to back the same way
+        A16 = rows_dev(82, HIDDEN, 16).mul_(0.02)
+        rows = []
+        for M in (1024, 4096, 8192):
+            R = _copies(2 * 2 * HIDDEN * M)
+            xs = [rows_dev(70 + j, M, HIDDEN) for j in range(R)]
+            ys = [torch.empty_like(xs[0]) for _ in range(R)]
+            t = torch.empty((M, 16), dtype=torch.float32, device=device)
+            ms = _time_graph([lambda j=j: B.bi_rmsnorm_lora_shrink(xs[j], w, A16, y=ys[j], t=t, eps=EPS,
+                                                                   stream=stream) for j in range(R)], stream)
+            two = _time_graph([lambda j=j: (B.bi_rmsnorm(xs[j], w, y=ys[j], eps=EPS, stream=stream),
+                                            B.bi_lora_shrink(ys[j], A16, t=t, split_k=8, stream=stream))
+                               for j in range(R)], stream)
+            pt = point("M", M, 2 * 2 * HIDDEN * M + 2 * HIDDEN + 2 * HIDDEN * 16 + 4 * M * 16, ms, peaks["hbm_gbs"],
+                       0.75, "GB/s")
+            pt["two_calls_us"] = round(two * 1e3, 2)
+            rows.append(pt)
+            del xs, ys
+        out["rmsnorm_lora_shrink_r16"] = {"unit": "GB/s", "rows": rows}
         # the expand (no target of its own; the shrink's companion), r = 16 into bf16 y
         B_l = rows_dev(81, 16, HIDDEN).mul_(0.02)
         rows = []

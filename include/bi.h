@@ -167,6 +167,34 @@ int bi_lora_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K,
                    void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * bi_rmsnorm_lora_shrink -- y = RMSNorm(x) . w and t = y . A in one pass
+ *
+ * Sources: the RMSNorm section of "Defeating Nondeterminism in LLM Inference" (Spanish
+ * summary, "Diseño de kernels invariantes al batch") and "Reproducible LoRA Inference Through
+ * Deterministic Split-K Reduction" (abstract).  The fused form of bi_rmsnorm followed by
+ * bi_lora_shrink on its output, for the case where the normalised rows feed a LoRA-adapted
+ * projection: the CTA that normalises a row multiplies it by A from its shared memory, so the
+ * shrink does not read y back from HBM.
+ *
+ *   x, y  device, bf16 [M, H] with row strides ldx, ldy (elements); y may equal x (then ldy = ldx)
+ *   w     device, bf16 [H], the RMSNorm weight
+ *   A     device, bf16 [H, r] row-major, the LoRA down-projection
+ *   t     device, fp32 [M, r] row-major, overwritten
+ *   H     4096; r 8 or 16; split_k 8.  Other shapes give BI_ERR_UNSUPPORTED_SHAPE: call bi_rmsnorm
+ *         and bi_lora_shrink instead, which give the same bits.
+ *   x, y, w, A, t 16-byte aligned, ldx and ldy multiples of 8.
+ *
+ * Arithmetic: y is bitwise bi_rmsnorm(x, w, eps) (bf16 in and out, bf16 weight) and t is
+ * bitwise bi_lora_shrink(y, A, r, split_k): every element goes through the same operations in
+ * the same order (bi_rmsnorm's per-row reduction tree for H = 4096; per K slice an mma.sync
+ * chain of 16-deep steps from zero, then ((P_0 + P_1) + ...) + P_7).  Batch-invariant like
+ * both.  Persistent CTAs walk 8-row tiles; which CTA takes a tile never changes a row's
+ * arithmetic.  A stage that does not arrive in time sets bit 0x2 of the device error word.
+ */
+int bi_rmsnorm_lora_shrink(const void* x, const void* w, void* y, const void* A, float* t, int64_t M, int64_t H,
+                           int64_t ldx, int64_t ldy, float eps, int32_t r, int32_t split_k, void* stream);
+
+/*
  * bi_lora_expand -- y[M, N] += scale * bf16(t)[M, r] . B[r, N], in place
  *
  * Source: the same abstract ("low-rank LoRA multiplications").  The low-rank product

@@ -68,6 +68,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "bi_ctrl_gemm_splitk": ([P, P, P, I64, I64, I64, C, P, Z, P], C),
         "bi_ctrl_gemm_split_workspace_size": ([I64, I64, I64, I32], Z),
         "bi_ctrl_gemm_split": ([P, P, P, I64, I64, I64, C, I32, P, Z, P], C),
+        "bi_rmsnorm_lora_shrink": ([P, P, P, P, P, I64, I64, I64, I64, F, I32, I32, P], C),
         "bi_ctrl_decode_attn_adaptive_workspace_size": ([I64, I32], Z),
         "bi_ctrl_decode_attn_adaptive": ([P, P, P, P, P, I32, I64, I32, I32, F, P, C, P, Z, P], C),
         "bi_ctrl_wait_timeout_probe": ([ctypes.c_uint64, P], C),
@@ -186,6 +187,34 @@ def bi_lora_shrink(x: torch.Tensor, A: torch.Tensor, t: torch.Tensor | None = No
                                   _stream(stream))
     _check("bi_lora_shrink", st)
     return t
+
+
+def bi_rmsnorm_lora_shrink(x: torch.Tensor, w: torch.Tensor, A: torch.Tensor, y: torch.Tensor | None = None,
+                           t: torch.Tensor | None = None, eps: float = 1e-6, split_k: int = 8,
+                           stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """y = RMSNorm(x) * w and t = y @ A in one pass; bitwise bi_rmsnorm then bi_lora_shrink.
+    x, y bf16 [M, 4096] (row strides may exceed 4096), w bf16 [4096], A bf16 [4096, r], r 8 or 16."""
+    _rows(x, "x")
+    _bf16_2d(A, "A")
+    if y is None:
+        y = torch.empty_like(x, memory_format=torch.contiguous_format)
+    _rows(y, "y")
+    if x.dtype != torch.bfloat16 or y.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise ValueError("x, y and w must be bf16")
+    if w.dim() != 1 or not w.is_contiguous() or not w.is_cuda:
+        raise ValueError("w must be a contiguous 1-D CUDA tensor")
+    M, H = x.shape
+    H2, r = A.shape
+    if H != H2 or tuple(y.shape) != (M, H):
+        raise ValueError("shape mismatch")
+    if t is None:
+        t = torch.empty((M, r), dtype=torch.float32, device=x.device)
+    if t.dtype != torch.float32 or tuple(t.shape) != (M, r) or not t.is_contiguous():
+        raise ValueError("t must be a contiguous fp32 [M, r] tensor")
+    st = library().bi_rmsnorm_lora_shrink(_ptr(x), _ptr(w), _ptr(y), _ptr(A), _ptr(t), M, H, max(x.stride(0), H),
+                                          max(y.stride(0), H), float(eps), r, split_k, _stream(stream))
+    _check("bi_rmsnorm_lora_shrink", st)
+    return y, t
 
 
 def bi_lora_expand(t: torch.Tensor, B: torch.Tensor, y: torch.Tensor, scale: float = 1.0,

@@ -9,8 +9,8 @@
 // Shrink, t[M, r] = x[M, K] . A[K, r]:
 //   The partial P_s of slice s covers the contiguous K slice [s*K/split, (s+1)*K/split).  It is
 //   accumulated in fp32 from bf16 products in 16-deep K steps in ascending order, starting from
-//   zero: with mma.sync m16n8k16 at r = 8, 16, 32, with tcgen05.mma at r = 64 (below).  The output is t = ((P_0 + P_1) + P_2) + ... + P_{split-1}, every
-//   add rounded to nearest.  There is no atomic, and the split count and slice size depend only
+//   zero: with mma.sync m16n8k16 at r = 8, 16, 32, with tcgen05.mma at r = 64 (below).  The
+//   output is t = ((P_0 + P_1) + P_2) + ... + P_{split-1}, every add rounded to nearest.  There is no atomic, and the split count and slice size depend only
 //   on (K, split), never on M.  A thread-block cluster of `split` CTAs computes 128-row tiles:
 //   CTA s streams x and A of its slice through a TMA ring, eight compute warps own 16 rows each,
 //   and the partials meet on chip (distributed shared memory), never in HBM.  The ordered kernel

@@ -130,3 +130,23 @@ def test_gemm_split_plan_host(lib):
     assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 4096, 64, 1, 2, None, 0, None) == 1  # 1 K block
     assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 8, 28672, 4096, 1, 2, None, 0, None) == 2
     assert lib.bi_ctrl_gemm_split(P(a), P(a), P(a), 0, 4096, 4096, 1, 2, None, 0, None) == 0  # empty batch
+
+
+def test_fused_rmsnorm_shrink_host_checks(lib):
+    """bi_rmsnorm_lora_shrink refuses, before any launch, the shapes it does not fuse (they
+    take the two separate calls), bad arguments and misaligned rows; an empty batch is a no-op."""
+    a = 1 << 20
+    P = ctypes.c_void_p
+    ok = dict(M=8, H=4096, ldx=4096, ldy=4096, eps=1e-6, r=16, split=8)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return lib.bi_rmsnorm_lora_shrink(P(a), P(a), P(a), P(a), P(a), d["M"], d["H"], d["ldx"], d["ldy"],
+                                          d["eps"], d["r"], d["split"], None)
+    assert call(M=0) == 0
+    assert call(H=2048, ldx=2048, ldy=2048) == 2
+    assert call(r=32) == 2 and call(r=64) == 2
+    assert call(split=4) == 2
+    assert call(ldx=4100) == 3  # a row stride that is not 16 bytes
+    assert call(ldx=4000) == 1  # shorter than a row
+    assert call(eps=-1.0) == 1 and call(M=-1) == 1
