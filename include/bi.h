@@ -189,7 +189,7 @@ int bi_lora_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K,
  * the same order (bi_rmsnorm's per-row reduction tree for H = 4096; per K slice an mma.sync
  * chain of 16-deep steps from zero, then ((P_0 + P_1) + ...) + P_7).  Batch-invariant like
  * both.  Persistent CTAs walk 8-row tiles; which CTA takes a tile never changes a row's
- * arithmetic.  A stage that does not arrive in time sets bit 0x2 of the device error word.
+ * arithmetic.
  */
 int bi_rmsnorm_lora_shrink(const void* x, const void* w, void* y, const void* A, float* t, int64_t M, int64_t H,
                            int64_t ldx, int64_t ldy, float eps, int32_t r, int32_t split_k, void* stream);

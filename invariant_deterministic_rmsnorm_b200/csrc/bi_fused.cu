@@ -24,16 +24,17 @@
 // (staged through shared memory and taken with ldmatrix .trans, as the shrink kernel does).
 //
 // Data flow: persistent CTAs, one per SM, walk tiles of 8 rows (tile i, i + grid, ...).  A ring
-// of shared-memory stages holds whole rows of x, each row fetched by one bulk copy
-// (cp.async.bulk, 8 KB) that completes on the stage's mbarrier; the ring keeps several tiles in
-// flight while the CTA works on one.  Per tile: sums of squares, the inverse norms, y written
-// to HBM and back into the stage in place, the eight slice MMAs, the ordered combine, t stored.
-// Which CTA handles a tile never changes a row's arithmetic.  Every wait is bounded.
+// of shared-memory stages holds whole rows of x.  Every thread fetches the 16-byte vectors it
+// owns with cp.async (one commit group per tile), so the ring keeps two tiles of loads in flight
+// without holding them in registers while the CTA works on the third.  Per tile: sums of
+// squares, the inverse norms, y written to HBM and back into the stage in place, the eight
+// slice MMAs, the ordered combine, t stored.  Which CTA handles a tile never changes a row's
+// arithmetic.
 //
-// Measured on a B200 against the two calls launched back to back: about the same time up to
-// M = 4096, 7-10 % less at M = 8192.  One CTA of eight warps per SM (the resident A slices take
-// 128 registers a thread) leaves the row phases short of the parallelism that bi_rmsnorm's
-// eight CTAs per SM have.
+// Measured on a B200 against the two calls launched back to back: 4-20 % less time at
+// M = 256 ... 8192.  A tile costs about 3.4 us of latency-bound row and MMA work: one CTA of
+// eight warps per SM (the resident A slices take 128 registers a thread) has far less
+// parallelism than bi_rmsnorm's eight CTAs per SM.
 #include <mutex>
 #include "bi_common.cuh"
 #include "bi_sm100.cuh"
@@ -59,26 +60,31 @@ constexpr int FU_PITCH = FU_ROW_BYTES + 16;
 constexpr int FU_STAGE = FU_ROWS * FU_PITCH;  // 64 KB + 128 B
 constexpr int FU_STAGES = 3;                  // 192 KB of rows in flight
 
+// 16 bytes global -> shared without a register round trip (cached in L2 only)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
 template <int R>
 struct FusedLayout {
     static constexpr int P_OFF = FU_STAGES * FU_STAGE;
     static constexpr int P_BYTES = FU_SPLIT * FU_ROWS * R * 4;  // the slices' partials of a tile
-    static constexpr int BAR_OFF = P_OFF + P_BYTES;
-    static constexpr size_t BYTES = (size_t)BAR_OFF + FU_STAGES * 8 + 16;
+    static constexpr size_t BYTES = (size_t)P_OFF + P_BYTES;
 };
 
 template <int R>
 __global__ void __launch_bounds__(FU_THREADS, 1)
 rmsnorm_lora_shrink_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
                            __nv_bfloat16* __restrict__ y, const __nv_bfloat16* __restrict__ A, float* __restrict__ t,
-                           int M, int64_t ldx, int64_t ldy, float eps, int n_tiles, uint32_t* err) {
+                           int M, int64_t ldx, int64_t ldy, float eps, int n_tiles) {
     using L = FusedLayout<R>;
     extern __shared__ __align__(16) uint8_t smem[];
     float* P = reinterpret_cast<float*>(smem + L::P_OFF);  // [slice][row][R]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     __shared__ float warp_sums[FU_ROWS][FU_WARPS];
     __shared__ float inv_s[FU_ROWS];
-    __shared__ int abort_s;
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -86,16 +92,10 @@ rmsnorm_lora_shrink_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloa
     const int g = lane >> 2, q = lane & 3;  // the mma fragment's row group and column pair
     const uint32_t sbase = smem_u32(smem);
 
-    if (tid == 0) {
-        for (int s = 0; s < FU_STAGES; ++s) mbar_init(smem_u32(&full[s]), 1);
-        abort_s = 0;
-        fence_barrier_init();
-    }
     // the weights of this thread's two vectors, as raw bf16 pairs (bi_rmsnorm keeps them the same way)
     uint32_t wr[FU_VPT][4];
     // B fragments of this warp's K slice: step j, column block nt, k rows 2q, 2q+1 and 2q+8, 2q+9
     uint32_t bfr[FU_STEPS][R / 8][2];
-    __syncthreads();
     pdl_wait();  // x, w and A may come from the kernel before this one; it may still read y or t
     pdl_trigger();
 #pragma unroll
@@ -104,37 +104,41 @@ rmsnorm_lora_shrink_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloa
 #pragma unroll
         for (int k = 0; k < 4; ++k) wr[i][k] = __ldg(src + k);
     }
-    // A [H, R] through the (still empty) stages with 16-byte loads, then each warp's fragments with
-    // ldmatrix .trans: the same register contents bi_lora_shrink's kernel loads per step
+    // every thread fetches its own vectors of a tile's rows into a stage: one commit group per
+    // tile (empty past the last tile, so that the group count stays the same on every thread)
+    auto issue = [&](int tile, int stage) {
+        if (tile < n_tiles) {
+            const int row0 = tile * FU_ROWS;
+            const int rows = M - row0 < FU_ROWS ? M - row0 : FU_ROWS;
+            for (int r = 0; r < rows; ++r)
+#pragma unroll
+                for (int i = 0; i < FU_VPT; ++i) {
+                    const int v = tid + i * FU_THREADS;
+                    cp_async16(sbase + (uint32_t)(stage * FU_STAGE + r * FU_PITCH + v * 16),
+                               x + (int64_t)(row0 + r) * ldx + (int64_t)v * FU_VEC);
+                }
+        }
+        cp_async_commit();
+    };
+    // A [H, R] into stages 1 and 2 (still empty) while the first tile's rows come into stage 0;
+    // then each warp takes its fragments with ldmatrix .trans: the same register contents
+    // bi_lora_shrink's kernel loads per step
+    const uint32_t a_smem = sbase + (uint32_t)FU_STAGE;
+#pragma unroll 4
     for (int i = tid; i < FU_H * R * 2 / 16; i += FU_THREADS)
-        *reinterpret_cast<uint4*>(smem + i * 16) = __ldg(reinterpret_cast<const uint4*>(A) + i);
+        cp_async16(a_smem + (uint32_t)(i * 16), reinterpret_cast<const uint8_t*>(A) + (size_t)i * 16);
+    cp_async_commit();
+    issue(blockIdx.x, 0);
+    cp_async_wait<1>();  // A has landed (the first tile may still be in flight)
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < FU_STEPS; ++j) {
         const int krow = warp * FU_KS + j * 16 + (lane & 15);
 #pragma unroll
-        for (int nt = 0; nt < R / 8; ++nt) ldmatrix_x2_trans(sbase + (uint32_t)(krow * R * 2 + nt * 16), bfr[j][nt]);
+        for (int nt = 0; nt < R / 8; ++nt) ldmatrix_x2_trans(a_smem + (uint32_t)(krow * R * 2 + nt * 16), bfr[j][nt]);
     }
-    // the stages are refilled by the copy engine: order these generic accesses before its writes
-    fence_proxy_async_shared();
-    __syncthreads();
-
-    // the producer: thread 0 fetches the rows of a tile into a stage, one bulk copy per row
-    auto issue = [&](int tile, int stage) {
-        const int row0 = tile * FU_ROWS;
-        const int rows = M - row0 < FU_ROWS ? M - row0 : FU_ROWS;
-        const uint32_t bar = smem_u32(&full[stage]);
-        mbar_arrive_expect_tx(bar, (uint32_t)(rows * FU_ROW_BYTES));
-        for (int r = 0; r < rows; ++r)
-            bulk_load(sbase + (uint32_t)(stage * FU_STAGE + r * FU_PITCH), x + (int64_t)(row0 + r) * ldx,
-                      (uint32_t)FU_ROW_BYTES, bar);
-    };
-    if (tid == 0) {
-        for (int s = 0; s < FU_STAGES; ++s) {
-            const int tile = blockIdx.x + s * gridDim.x;
-            if (tile < n_tiles) issue(tile, s);
-        }
-    }
+    __syncthreads();  // every warp has its fragments before stages 1 and 2 are overwritten
+    for (int s = 1; s < FU_STAGES; ++s) issue(blockIdx.x + s * gridDim.x, s);
 
     const float h_float = (float)FU_H;
     int j = 0;
@@ -142,12 +146,9 @@ rmsnorm_lora_shrink_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloa
         const int stage = j % FU_STAGES;
         const int row0 = tile * FU_ROWS;
         const int rows = M - row0 < FU_ROWS ? M - row0 : FU_ROWS;
-        const bool ok = mbar_wait(smem_u32(&full[stage]), (uint32_t)(j / FU_STAGES) & 1u, nullptr);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) atomicOr(err, bi::DEVERR_WAIT_FULL);
-            abort_s = 1;
-            break;
-        }
+        // this thread's vectors of the tile have landed (at most the two later tiles' groups pend);
+        // phases 1 and 3 read only those, and the barrier after phase 3 publishes y to the MMA warps
+        cp_async_wait<FU_STAGES - 1>();
 
         const uint8_t* st = smem + stage * FU_STAGE;  // this tile's rows, row r at r * FU_PITCH
         // 1. per row: this thread's sum of squares, vectors in order, elements in order; the warp
@@ -287,29 +288,17 @@ rmsnorm_lora_shrink_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloa
             for (int sl = 1; sl < FU_SPLIT; ++sl) v = __fadd_rn(v, P[(sl * FU_ROWS + r) * R + c]);
             t[(int64_t)(row0 + r) * R + c] = v;
         }
-        // 6. the stage is free once every thread's generic reads and writes of it are ordered
-        //    before the refill's async-proxy writes; the barrier also retires P and the sums
-        fence_proxy_async_shared();
+        // 6. every read of the stage (the MMA warps' included) is done: refill it
         __syncthreads();
-        if (tid == 0 && tile + FU_STAGES * (int)gridDim.x < n_tiles) issue(tile + FU_STAGES * (int)gridDim.x, stage);
+        issue(tile + FU_STAGES * (int)gridDim.x, stage);
     }
-    if (abort_s && tid == 0) {
-        // copies still in flight land before the shared memory is released (bounded waits)
-        const int done = j;
-        for (int jj = done; jj < done + FU_STAGES; ++jj) {
-            const int tl = blockIdx.x + jj * (int)gridDim.x;
-            if (tl >= n_tiles) break;
-            (void)mbar_wait(smem_u32(&full[jj % FU_STAGES]), (uint32_t)(jj / FU_STAGES) & 1u, nullptr);
-        }
-    }
+    cp_async_wait<0>();  // nothing may still write this CTA's shared memory when it exits
 }
 
 template <int R>
 int launch_fused(const void* x, const void* w, void* y, const void* A, float* t, int64_t M, int64_t ldx,
                  int64_t ldy, float eps, cudaStream_t s) {
     using L = FusedLayout<R>;
-    uint32_t* err = bi::device_error_word();
-    if (!err) return BI_ERR_CUDA;
     static std::once_flag once[64];
     static bool attr_ok[64];
     static int sms_cached[64];
@@ -326,7 +315,7 @@ int launch_fused(const void* x, const void* w, void* y, const void* A, float* t,
     if (bi::launch_pdl(rmsnorm_lora_shrink_kernel<R>, dim3((unsigned)grid), dim3(FU_THREADS), L::BYTES, s, 0u,
                        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w),
                        static_cast<__nv_bfloat16*>(y), static_cast<const __nv_bfloat16*>(A), t, (int)M, ldx, ldy, eps,
-                       (int)n_tiles, err) != cudaSuccess)
+                       (int)n_tiles) != cudaSuccess)
         return BI_ERR_CUDA;
     return bi::launch_status();
 }
