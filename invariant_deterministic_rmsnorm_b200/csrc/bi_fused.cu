@@ -27,12 +27,12 @@
 // of shared-memory stages holds whole rows of x.  Every thread fetches the 16-byte vectors it
 // owns with cp.async (one commit group per tile), so the ring keeps two tiles of loads in flight
 // without holding them in registers while the CTA works on the third.  Per tile: sums of
-// squares, the inverse norms, y written to HBM and back into the stage in place, the eight
-// slice MMAs, the ordered combine, t stored.  Which CTA handles a tile never changes a row's
+// squares, the inverse norms, y over x in the stage (and from there to HBM, one bulk copy per
+// row), the eight slice MMAs, the ordered combine, t stored.  Which CTA handles a tile never changes a row's
 // arithmetic.
 //
-// Measured on a B200 against the two calls launched back to back: 4-20 % less time at
-// M = 256 ... 8192.  A tile costs about 3.4 us of latency-bound row and MMA work: one CTA of
+// Measured on a B200 against the two calls launched back to back: the same time at M = 256,
+// 12-19 % less at M = 1024 ... 8192.  A tile costs about 3.4 us of latency-bound row and MMA work: one CTA of
 // eight warps per SM (the resident A slices take 128 registers a thread) has far less
 // parallelism than bi_rmsnorm's eight CTAs per SM.
 #include <mutex>
@@ -67,6 +67,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+// `bytes` (a multiple of 16, both addresses 16-byte aligned) shared -> global by the copy engine
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :: "l"(reinterpret_cast<uint64_t>(dst)), "r"(src), "r"(bytes) : "memory");
+}
 
 template <int R>
 struct FusedLayout {
@@ -227,7 +232,6 @@ rmsnorm_lora_shrink_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloa
                 for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], inv), wf[i][e]);
                 const uint4 o = make_uint4(bi::pack_bf16x2(f[0], f[1]), bi::pack_bf16x2(f[2], f[3]),
                                            bi::pack_bf16x2(f[4], f[5]), bi::pack_bf16x2(f[6], f[7]));
-                bi::st_stream_v4(y + (int64_t)(row0 + r) * ldy + (int64_t)v * FU_VEC, o);
                 *reinterpret_cast<uint4*>(smem + stage * FU_STAGE + r * FU_PITCH + v * 16) = o;
             };
             if (rows == FU_ROWS) {
@@ -251,7 +255,16 @@ rmsnorm_lora_shrink_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloa
                         norm_row(r, i, *reinterpret_cast<const uint4*>(st + r * FU_PITCH + (tid + i * FU_THREADS) * 16));
             }
         }
+        // y leaves for HBM from the stage, one bulk copy per row (the copy engine reads what the
+        // threads wrote: their generic writes are ordered before its async-proxy reads)
+        fence_proxy_async_shared();
         __syncthreads();
+        if (tid == 0) {
+            for (int r = 0; r < rows; ++r)
+                bulk_store(y + (int64_t)(row0 + r) * ldy, sbase + (uint32_t)(stage * FU_STAGE + r * FU_PITCH),
+                           (uint32_t)FU_ROW_BYTES);
+            bulk_commit();
+        }
         // 4. warp s: the partial of K slice s over the tile's rows, 32 mma steps from zero.  Row g of
         //    the fragment is tile row g (zero past the last row), rows g + 8 are zero.
         {
@@ -288,11 +301,13 @@ rmsnorm_lora_shrink_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloa
             for (int sl = 1; sl < FU_SPLIT; ++sl) v = __fadd_rn(v, P[(sl * FU_ROWS + r) * R + c]);
             t[(int64_t)(row0 + r) * R + c] = v;
         }
-        // 6. every read of the stage (the MMA warps' included) is done: refill it
+        // 6. every read of the stage (the MMA warps' and the copy engine's included) is done: refill it
+        if (tid == 0) bulk_wait_read();
         __syncthreads();
         issue(tile + FU_STAGES * (int)gridDim.x, stage);
     }
     cp_async_wait<0>();  // nothing may still write this CTA's shared memory when it exits
+    if (tid == 0) bulk_wait_all();  // and y has reached global memory
 }
 
 template <int R>
