@@ -1403,12 +1403,28 @@ def run_one_op(args):
     device = torch.device("cuda", 0)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
-        ops, _ = build_ops(device, stream, args.attn_batch, args.lora_rank, args.tokens)
-        op = next(o for o in ops if o["name"] == args.op)
-        for k in range(args.launches):
-            op["launch"](k)
+        if args.op == "rmsnorm_lora_shrink":
+            # the fused RMSNorm + shrink (not an op of the step): the step's RMSNorm input and weight,
+            # the LoRA A of the step's rank, rotating inputs
+            from invariant_deterministic_rmsnorm_b200 import binding as B
+            M, H, r = args.tokens, HIDDEN, args.lora_rank
+            x_np, w_np = inputs.rmsnorm_case(M, H, "bf16")
+            xs = [_to_dev(x_np, device) for _ in range(ROTATE)]
+            w = _to_dev(w_np, device)
+            A_l = _to_dev(inputs.normal_bf16(inputs.SEED_WEIGHTS + 20, (H, r), 0.0, 0.02), device)
+            y = torch.empty_like(xs[0])
+            t = torch.empty((M, r), dtype=torch.float32, device=device)
+            for k in range(args.launches):
+                B.bi_rmsnorm_lora_shrink(xs[k % ROTATE], w, A_l, y=y, t=t, eps=EPS, stream=stream)
+            desc = f"x bf16 [{M},{H}] -> y bf16 and t fp32 [{M},{r}] = y A, split-K 8, one pass"
+        else:
+            ops, _ = build_ops(device, stream, args.attn_batch, args.lora_rank, args.tokens)
+            op = next(o for o in ops if o["name"] == args.op)
+            for k in range(args.launches):
+                op["launch"](k)
+            desc = op["desc"]
     torch.cuda.synchronize()
-    print(json.dumps({"op": args.op, "launches": args.launches, "desc": op["desc"]}), flush=True)
+    print(json.dumps({"op": args.op, "launches": args.launches, "desc": desc}), flush=True)
 
 
 def main():
@@ -1440,7 +1456,7 @@ def main():
     ap.add_argument("--contrast-batches", type=int, nargs="+", default=[1, 8, 32, 128])
     ap.add_argument("--op", default=None,
                     choices=["rmsnorm", "gemm_qkv", "lora_shrink", "lora_expand", "gemm_up", "gemm_down",
-                             "decode_attn"],
+                             "decode_attn", "rmsnorm_lora_shrink"],
                     help="launch only this op of the step, --launches times, and exit (for profiler captures)")
     ap.add_argument("--launches", type=int, default=4)
     ap.add_argument("--tokens", type=int, default=M_TOKENS,
