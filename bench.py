@@ -1059,9 +1059,10 @@ def run_sweep(args):
     kv_len = inputs.kv_lengths(128)
     indptr, T = inputs.kv_layout(kv_len, 256)
     g = torch.Generator(device=device).manual_seed(5)
-    kc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
-    vc = torch.randn((T, 8, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
-    qa = torch.randn((128, 32, 128), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    # drawn straight into bf16 buffers: no fp32 temporaries twice the cache's size beside it
+    kc = torch.empty((T, 8, 128), device=device, dtype=torch.bfloat16).normal_(generator=g)
+    vc = torch.empty((T, 8, 128), device=device, dtype=torch.bfloat16).normal_(generator=g)
+    qa = torch.empty((128, 32, 128), device=device, dtype=torch.bfloat16).normal_(generator=g)
     ip_d = torch.tensor(indptr, dtype=torch.int32, device=device)
     ln_d = torch.tensor(kv_len, dtype=torch.int32, device=device)
     table = []
