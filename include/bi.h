@@ -158,9 +158,10 @@ int bi_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t
  * accumulator per slice) at r = 64.  t = ((P_0 + P_1) + ...) + P_{split_k - 1}, each add
  * rounded to nearest.  No atomics.  The partials meet on chip (distributed shared memory of
  * a thread-block cluster), and every CTA of the cluster adds all slices of its share of a
- * 128-row tile's rows.  The arithmetic depends on (K, r, split_k) only; the cluster shape of
- * the r = 64 kernel (split_k CTAs of one slice, or split_k / 2 of two) follows the number of
- * tiles and gives the same bits either way.
+ * tile's rows (tiles of 128 rows at r = 8 and 64, of 64 rows at r = 16 and 32).  The arithmetic
+ * depends on (K, r, split_k) only; neither the tile height nor the cluster shape of the r = 64
+ * kernel (split_k CTAs of one slice, or split_k / 2 of two, by the number of tiles) changes a
+ * row's bits.
  */
 size_t bi_lora_shrink_workspace_size(int64_t M, int64_t K, int32_t r, int32_t split_k);
 int bi_lora_shrink(const void* x, const void* A, float* t, int64_t M, int64_t K, int32_t r, int32_t split_k,

@@ -10,10 +10,11 @@
 //   The partial P_s of slice s covers the contiguous K slice [s*K/split, (s+1)*K/split).  It is
 //   accumulated in fp32 from bf16 products in 16-deep K steps in ascending order, starting from
 //   zero: with mma.sync m16n8k16 at r = 8, 16, 32, with tcgen05.mma at r = 64 (below).  The
-//   output is t = ((P_0 + P_1) + P_2) + ... + P_{split-1}, every add rounded to nearest.  There is no atomic, and the split count and slice size depend only
-//   on (K, split), never on M.  A thread-block cluster of `split` CTAs computes 128-row tiles:
-//   CTA s streams x and A of its slice through a TMA ring, eight compute warps own 16 rows each,
-//   and the partials meet on chip (distributed shared memory), never in HBM.  The ordered kernel
+//   output is t = ((P_0 + P_1) + P_2) + ... + P_{split-1}, every add rounded to nearest.  There
+//   is no atomic, and the split count and slice size depend only on (K, split), never on M.  A
+//   thread-block cluster of `split` CTAs computes tiles of 64 or 128 rows (by r): CTA s streams x
+//   and A of its slice through a TMA ring, each compute warp owns 16 rows, and the partials meet
+//   on chip (distributed shared memory), never in HBM.  The ordered kernel
 //   (lora_shrink_ordered_kernel) is persistent and spreads the combine over every CTA of the
 //   cluster; the atomic comparator (lora_shrink_atomic_kernel) adds the partials into t with
 //   floating-point atomics instead.
@@ -172,37 +173,48 @@ lora_shrink_atomic_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_
 // The batch-invariant shrink.  Each output element is computed exactly as described at the top
 // of this file: slice s's partial is one mma.sync chain over its K slice, and the partials are
 // added in slice order.  What this kernel changes is where and when that happens:
-//   - Persistent clusters.  A cluster of `split` CTAs (CTA s = slice s) walks 128-row tiles
-//     c, c + clusters, ...; its producer warp keeps one TMA ring streaming across tiles, so a
-//     cluster's second tile loads while its first is being combined.
-//   - Distributed, pushed combine.  Compute warp w owns rows [16w, 16w + 16) of the tile.  When
-//     its chain ends, it stores its fragment of the partial straight into the shared memory of
-//     the CTA that combines those rows (CTA d = w * split / 8 combines rows
-//     [128 d / split, 128 (d + 1) / split)), and every lane then arrives, with release semantics
-//     at cluster scope, on d's receive barrier: each lane publishes its own stores.  A combiner
-//     warp in every CTA waits for the 8 x 32 arrivals (acquire), adds its rows' split partials
-//     from its own shared memory in slice order, and writes t.  Every CTA combines; no CTA reads
-//     a peer's shared memory.
-//   - Receive buffers rotate (two for r <= 16, one above), and a combiner hands a buffer back to
-//     the senders with a remote arrive once it has read it.
+//   - Persistent clusters.  A cluster of `split` CTAs (CTA s = slice s) walks tiles c,
+//     c + clusters, ...; its producer warp keeps one TMA ring streaming across tiles, so a
+//     cluster's next tile loads while its last one is being exchanged and combined.  Tiles have
+//     TM = 64 rows from r = 16 (a cluster then has two at M = 4096 on this GPU, where one tile of
+//     128 left that tail bare, and twice the CTAs share a small batch) and 128 rows at r = 8; a
+//     row's arithmetic does not depend on the tile height.
+//   - Distributed, pushed combine.  Compute warp w owns rows [16w, 16w + 16) of the tile; CTA d
+//     combines rows [TM d / split, TM (d + 1) / split).  When its chain ends, a warp stages its
+//     rows of the partial in its own shared memory as the combining CTA's buffer holds them and
+//     sends them with one bulk copy per combining CTA (two when a CTA combines 8 rows), which
+//     completes on that CTA's receive barrier.  A combiner warp in every CTA waits for the bytes,
+//     adds its rows' split partials from its own shared memory in slice order, writes t, and
+//     hands the buffer back to every sender with a remote arrive.  No CTA reads a peer's shared
+//     memory.
 // Every wait is bounded.  A cluster barrier at the end keeps each CTA's shared memory alive until
 // no peer can still write into it.
-constexpr int SO_CWARPS = 8;
-constexpr int SO_THREADS = (SO_CWARPS + 2) * 32;  // compute warps, a producer warp, a combiner warp
+constexpr int SO_MAX_STAGES = 8;   // a whole 512-column slice of a tile in flight
+
+// Tile height by rank (a row's arithmetic does not depend on it): 64 rows from r = 16, where
+// the measured shrink is 2-20 % faster than with 128-row tiles, and 128 rows at r = 8, where it
+// is 2-6 % slower.
+template <int R>
+struct OrderedShape {
+    static constexpr int TM = R >= 16 ? 64 : 128;           // rows per tile
+    static constexpr int CWARPS = TM / 16;                   // compute warps, 16 rows each
+    static constexpr int THREADS = (CWARPS + 2) * 32;        // compute warps, a producer warp, a combiner warp
+};
 
 template <int R>
 struct OrderedLayout {
-    static constexpr int X_STAGE = SH_TM * SH_KC * 2;  // 16 KB, 128B-swizzled rows of 64 K
+    static constexpr int SO_TM = OrderedShape<R>::TM;
+    static constexpr int X_STAGE = SO_TM * SH_KC * 2;  // 8 or 16 KB, 128B-swizzled rows of 64 K
     static constexpr int A_STAGE = SH_KC * R * 2;
-    static constexpr int STAGE = X_STAGE + A_STAGE;
+    static constexpr int STAGE = X_STAGE + A_STAGE;    // a multiple of 1 KB
     static constexpr int NB = 1;                       // receive buffers
-    static constexpr int RECV = SH_TM * R * 4;         // one buffer: [slice][rows this CTA combines][R] fp32
-    // every compute warp stages its 16 rows of partials here before one bulk copy sends them
-    static constexpr int STAGING = SH_TM * R * 4;
+    static constexpr int RECV = SO_TM * R * 4;         // one buffer: [slice][rows this CTA combines][R] fp32
+    // every compute warp stages its 16 rows of partials here before its bulk copies send them
+    static constexpr int STAGING = SO_TM * R * 4;
     // two CTAs per SM: at most 112 KB each, including the 1 KB alignment pad and the barriers
     static constexpr int BUDGET = 112 * 1024 - 1024 - 256;
     static constexpr int STAGES_FIT = (BUDGET - NB * RECV - STAGING) / STAGE;
-    static constexpr int STAGES = STAGES_FIT > SH_MAX_STAGES ? SH_MAX_STAGES : STAGES_FIT;
+    static constexpr int STAGES = STAGES_FIT > SO_MAX_STAGES ? SO_MAX_STAGES : STAGES_FIT;
     static_assert(STAGES >= 3, "the ring needs at least three stages");
     static constexpr int RECV_OFF = STAGES * STAGE;
     static constexpr int STAGING_OFF = RECV_OFF + NB * RECV;
@@ -214,10 +226,12 @@ struct OrderedLayout {
 };
 
 template <int R>
-__global__ void __launch_bounds__(SO_THREADS, 2)
+__global__ void __launch_bounds__(OrderedShape<R>::THREADS, 2)
 lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
                            float* __restrict__ t, int M, int KS, int split, int n_tiles, uint32_t* err) {
     using L = OrderedLayout<R>;
+    constexpr int SO_TM = OrderedShape<R>::TM;
+    constexpr int SO_CWARPS = OrderedShape<R>::CWARPS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* recv = reinterpret_cast<float*>(base + L::RECV_OFF);
@@ -234,7 +248,7 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
     const uint32_t slice = cluster_ctarank();
     const int kbase = (int)slice * KS;
     const int nchunks = KS / SH_KC;
-    const int rows_per = SH_TM / split;  // rows of a tile that each CTA combines
+    const int rows_per = SO_TM / split;  // rows of a tile that each CTA combines (8 or more)
 
     if (tid == 0) {
         for (int i = 0; i < L::STAGES; ++i) {
@@ -272,7 +286,7 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
                     uint8_t* sx = base + st * L::STAGE;
                     const uint32_t fb = smem_u32(&full[st]);
                     mbar_arrive_expect_tx(fb, L::STAGE);
-                    tma_load_2d(smem_u32(sx), &tmX, kbase + c * SH_KC, tile * SH_TM, fb);
+                    tma_load_2d(smem_u32(sx), &tmX, kbase + c * SH_KC, tile * SO_TM, fb);
                     tma_load_2d(smem_u32(sx + L::X_STAGE), &tmA, 0, kbase + c * SH_KC, fb);
                 }
             }
@@ -283,7 +297,7 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
         }
     } else if (warp == SO_CWARPS + 1) {
         // ------------------------------------------------ combiner: this CTA's rows of every tile
-        const uint32_t tile_bytes = (uint32_t)(SH_TM * R * 4);  // every slice of this CTA's rows
+        const uint32_t tile_bytes = (uint32_t)(SO_TM * R * 4);  // every slice of this CTA's rows
         if (lane == 0 && (int)blockIdx.x < n_tiles) mbar_arrive_expect_tx(smem_u32(&rfull[0]), tile_bytes);
         int j = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
@@ -295,8 +309,8 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
                 *abort = 1;
                 break;
             }
-            const float* rb = recv + b * (SH_TM * R);  // [slice][rows_per][R]
-            const int row0 = tile * SH_TM + (int)slice * rows_per;
+            const float* rb = recv + b * (SO_TM * R);  // [slice][rows_per][R]
+            const int row0 = tile * SO_TM + (int)slice * rows_per;
             for (int i = lane; i < rows_per * R / 4; i += 32) {
                 const int row = (4 * i) / R, col = (4 * i) % R;
                 float4 v = *reinterpret_cast<const float4*>(rb + row * R + col);
@@ -318,10 +332,11 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
         }
     } else {
         // ------------------------------------------------ compute warps
-        const int d = warp * split / SO_CWARPS;            // the CTA that combines this warp's rows
-        const int lrow0 = warp * 16 - d * rows_per;        // first of them inside d's share
-        const uint32_t peer_recv = mapa(smem_u32(recv), (uint32_t)d);
-        const uint32_t peer_rfull = mapa(smem_u32(rfull), (uint32_t)d);
+        // this warp's 16 rows go to one combining CTA, or to two when a CTA combines 8 rows
+        const int chunk = rows_per < 16 ? rows_per : 16;   // rows per destination
+        const int nd = 16 / chunk;                         // 1 or 2
+        const int d0 = warp * 16 / rows_per;               // the CTA that combines the first of them
+        const int lrow0 = warp * 16 - d0 * rows_per;       // their first row inside d0's share
         const uint32_t stg = smem_u32(staging + warp * 16 * R);  // this warp's 16 rows, as d holds them
         bool pending = false;  // lane 0 issued a copy whose source may still be read
         const int g = lane >> 2, q = lane & 3;
@@ -363,8 +378,10 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
             if (!ok) break;
             const int b = j % L::NB;
             const uint32_t par = (uint32_t)(j / L::NB) & 1u;
-            // d has read what this warp pushed into buffer b for tile j - NB
-            ok = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&rfree[b * SH_MAX_SPLIT + d]), par ^ 1u, abort));
+            // every destination has read what this warp pushed into its buffer b for tile j - NB
+            for (int k = 0; ok && k < nd; ++k)
+                ok = __all_sync(0xffffffffu, mbar_wait_cluster(smem_u32(&rfree[b * SH_MAX_SPLIT + d0 + k]), par ^ 1u,
+                                                                abort));
             if (!ok) {
                 if (lane == 0) atomicOr(err, bi::DEVERR_WAIT_CLUSTER);
                 *abort = 1;
@@ -385,8 +402,13 @@ lora_shrink_ordered_kernel(const __grid_constant__ CUtensorMap tmX, const __grid
             fence_proxy_async_shared();  // the copy engine reads what these generic stores wrote
             __syncwarp();
             if (lane == 0) {
-                const uint32_t dst = peer_recv + (uint32_t)((b * SH_TM * R + ((int)slice * rows_per + lrow0) * R) * 4);
-                bulk_copy_to_peer(dst, stg, (uint32_t)(16 * R * 4), peer_rfull + (uint32_t)b * 8u);
+                for (int k = 0; k < nd; ++k) {
+                    const uint32_t d = (uint32_t)(d0 + k);
+                    const uint32_t dst = mapa(smem_u32(recv), d) +
+                                         (uint32_t)((b * SO_TM * R + ((int)slice * rows_per + lrow0) * R) * 4);
+                    bulk_copy_to_peer(dst, stg + (uint32_t)(k * chunk * R * 4), (uint32_t)(chunk * R * 4),
+                                      mapa(smem_u32(rfull), d) + (uint32_t)b * 8u);
+                }
                 bulk_commit();
                 pending = true;
             }
@@ -942,7 +964,7 @@ int ordered_clusters(int split) {
         int n = 0;
         if (split == 1) {
             int per_sm = 0, sms = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lora_shrink_ordered_kernel<R>, SO_THREADS,
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lora_shrink_ordered_kernel<R>, OrderedShape<R>::THREADS,
                                                               L::BYTES) != cudaSuccess ||
                 cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
                 return -1;
@@ -950,7 +972,7 @@ int ordered_clusters(int split) {
         } else {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(1, (unsigned)split, 1);
-            cfg.blockDim = dim3(SO_THREADS, 1, 1);
+            cfg.blockDim = dim3(OrderedShape<R>::THREADS, 1, 1);
             cfg.dynamicSmemBytes = L::BYTES;
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -976,14 +998,14 @@ int launch_shrink_ordered(const void* x, const void* A, float* t, int64_t M, int
     if (fit <= 0) return BI_ERR_CUDA;
     CUtensorMap tmX, tmA;
     if (!bi::make_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2,
-                          SH_KC, SH_TM, CU_TENSOR_MAP_SWIZZLE_128B))
+                          SH_KC, OrderedShape<R>::TM, CU_TENSOR_MAP_SWIZZLE_128B))
         return BI_ERR_CUDA;
     if (!bi::make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, (uint64_t)R, (uint64_t)K, (uint64_t)R * 2, R,
                           SH_KC, bi::swizzle_for(R * 2)))
         return BI_ERR_CUDA;
-    const int n_tiles = (int)((M + SH_TM - 1) / SH_TM);
+    const int n_tiles = (int)((M + OrderedShape<R>::TM - 1) / OrderedShape<R>::TM);
     const int clusters = n_tiles < fit ? n_tiles : fit;
-    if (bi::launch_pdl(kern, dim3((unsigned)clusters, (unsigned)split), dim3(SO_THREADS), L::BYTES, s,
+    if (bi::launch_pdl(kern, dim3((unsigned)clusters, (unsigned)split), dim3(OrderedShape<R>::THREADS), L::BYTES, s,
                        (unsigned)split, tmX, tmA, t, (int)M, (int)(K / split), (int)split, n_tiles,
                        err) != cudaSuccess)
         return BI_ERR_CUDA;
