@@ -32,7 +32,7 @@
 // arithmetic.
 //
 // Measured on a B200 against the two calls launched back to back: the same time at M = 256,
-// 12-19 % less at M = 1024 ... 8192.  A tile costs about 3.4 us of latency-bound row and MMA work: one CTA of
+// 9-26 % less at M = 1024 ... 8192 (the spread is between boxes).  A tile costs about 3.4 us of latency-bound row and MMA work: one CTA of
 // eight warps per SM (the resident A slices take 128 registers a thread) has far less
 // parallelism than bi_rmsnorm's eight CTAs per SM.
 #include <mutex>
