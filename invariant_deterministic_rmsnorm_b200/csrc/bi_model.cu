@@ -78,6 +78,43 @@ __global__ void rope_kernel(__nv_bfloat16* __restrict__ x, int64_t ld_row, int h
                           __fadd_rn(__fmul_rn(b1, cs.z), __fmul_rn(a1, cs.w)));
 }
 
+// The same rotation, eight pairs i .. i+7 (i a multiple of 8) of one head per thread, with
+// 16-byte loads and stores, for rows that are 16-byte aligned and head_dim a multiple of 16.
+// Element for element it runs rope_kernel's operations, so the two give the same bits.
+__global__ void rope8_kernel(__nv_bfloat16* __restrict__ x, int64_t ld_row, int heads, int D,
+                             const int32_t* __restrict__ pos, const float4* __restrict__ table, int64_t table_rows,
+                             uint32_t* err) {
+    pdl_wait();  // inputs may come from the kernel just before this one
+    pdl_trigger();
+    const int64_t t = blockIdx.x;
+    const int half = D / 2, octs = half / 8;  // pairs per head, eight at a time
+    const int j = blockIdx.y * blockDim.x + threadIdx.x;
+    if (j >= heads * octs) return;
+    const int32_t p = pos[t];
+    if (p < 0 || p >= table_rows) {
+        if (j == 0) atomicOr(err, bi::DEVERR_BAD_POSITION);  // position outside the table: row left as is
+        return;
+    }
+    const int h = j / octs, i = (j % octs) * 8;
+    const float4* cs = table + ((int64_t)p * half + i) / 2;  // (cos, sin) of pairs i, i+1 per float4
+    uint4* lo = reinterpret_cast<uint4*>(x + t * ld_row + (int64_t)h * D + i);
+    uint4* hi = reinterpret_cast<uint4*>(x + t * ld_row + (int64_t)h * D + half + i);
+    const uint4 av = *lo, bv = *hi;
+    const uint32_t a[4] = {av.x, av.y, av.z, av.w}, b[4] = {bv.x, bv.y, bv.z, bv.w};
+    uint32_t ro[4], rh[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 c = cs[q];
+        const float a0 = bi::bf16_lo(a[q]), a1 = bi::bf16_hi(a[q]), b0 = bi::bf16_lo(b[q]), b1 = bi::bf16_hi(b[q]);
+        ro[q] = bi::pack_bf16x2(__fsub_rn(__fmul_rn(a0, c.x), __fmul_rn(b0, c.y)),
+                                __fsub_rn(__fmul_rn(a1, c.z), __fmul_rn(b1, c.w)));
+        rh[q] = bi::pack_bf16x2(__fadd_rn(__fmul_rn(b0, c.x), __fmul_rn(a0, c.y)),
+                                __fadd_rn(__fmul_rn(b1, c.z), __fmul_rn(a1, c.w)));
+    }
+    *lo = make_uint4(ro[0], ro[1], ro[2], ro[3]);
+    *hi = make_uint4(rh[0], rh[1], rh[2], rh[3]);
+}
+
 // ------------------------------------------------------------------ KV append
 // dst[dst_row[t], :] = src[t, :] for one packed row of `row_elems` bf16 (all kv heads of a token).
 __global__ void kv_append_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src,
@@ -228,10 +265,12 @@ BI_API int bi_rope(void* x, int64_t T, int64_t ld_row, int32_t heads, int32_t he
     if (!bi::aligned16(table) || (reinterpret_cast<uintptr_t>(x) & 3u) || ld_row % 2 != 0) return BI_ERR_MISALIGNED;
     uint32_t* err = bi::device_error_word();
     if (!err) return BI_ERR_CUDA;
-    const int work = heads * (head_dim / 4);
+    // 16-byte accesses where the layout allows them (the same bits either way)
+    const bool vec = bi::aligned16(x) && ld_row % 8 == 0 && head_dim % 16 == 0;
+    const int work = heads * (head_dim / (vec ? 16 : 4));
     if ((work + 127) / 128 > 65535) return BI_ERR_UNSUPPORTED_SHAPE;
     dim3 grid((unsigned)T, (unsigned)((work + 127) / 128));
-    if (bi::launch_pdl(rope_kernel, dim3(grid), dim3(128), 0, bi::as_stream(stream), 0u,
+    if (bi::launch_pdl(vec ? rope8_kernel : rope_kernel, dim3(grid), dim3(128), 0, bi::as_stream(stream), 0u,
                        static_cast<__nv_bfloat16*>(x), ld_row, heads, head_dim, pos,
                        static_cast<const float4*>(table), table_rows, err) != cudaSuccess)
         return BI_ERR_CUDA;

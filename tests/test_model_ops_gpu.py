@@ -59,6 +59,23 @@ def test_rope_parity(heads, ld):
     assert np.array_equal(got[0], x[0])  # position 0 is the identity
 
 
+def test_rope_16_byte_and_4_byte_paths_give_the_same_bits():
+    """Rows that are 16-byte aligned (row stride a multiple of 8) take the kernel with 16-byte
+    accesses; an even row stride that is not a multiple of 8 takes the 4-byte kernel.  Both run
+    the same operations on every element."""
+    T, D, heads = 257, 128, 40
+    x = inputs.normal_bf16(34, (T, heads * D))
+    pos = np.random.default_rng(35).integers(0, 2200, T).astype(np.int32)
+    table = binding.bi_rope_table(2200, D, 500000.0)
+    rows = {}
+    for ld in (6144, 6146):
+        buf = np.zeros((T, ld), np.uint16)
+        buf[:, :heads * D] = x
+        rows[ld] = host(binding.bi_rope(dev(buf), dev(pos), heads, table, D))[:, :heads * D]
+    assert np.array_equal(rows[6144], rows[6146])
+    assert not np.array_equal(rows[6144], x)  # the rotation did run
+
+
 def test_rope_table_and_bad_position():
     t = host(binding.bi_rope_table(3000, 128, 500000.0)).astype(np.float64)
     i = np.arange(64)
